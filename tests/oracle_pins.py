@@ -1,0 +1,268 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each ``pin_*`` function takes a compiled oracle library handle (the real one,
+or a deliberately broken variant built by the mutation test) and raises
+AssertionError when the oracle disagrees with what the method's definition
+and mathematics fix:
+
+* brute force: the full token score matrix from a library matmul, max-pooled
+  by reshaping, and the kept set decided by COUNTING better candidates (no
+  sort), for tiny inputs ("MiniMax Sparse Attention", Summary: max-pooled
+  token-level index scores, per-group Top-k, current block kept);
+* the dense limit: with every causal block kept, the output is dense causal
+  GQA attention, computed by torch's scaled_dot_product_attention in fp64;
+* masked attention: for any kept set, the output is scaled_dot_product_attention
+  with a boolean mask that allows exactly the kept blocks' causal tokens;
+* closed forms and invariants: all-equal index scores keep blocks
+  {0..k-2} plus the current one; constant values give a constant output; a
+  single attended key gives that key's value; LSE brackets;
+* exactness of the inputs' grid: bf16 and fp32 copies of the same grid
+  values give bit-identical oracle results.
+
+Inputs are small (a few hundred tokens) so every pin runs in well under a
+second on CPU.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle as orc
+
+
+def _grid(rng, shape):
+    return (rng.integers(-4, 5, size=shape).astype(np.float32) / 4.0)
+
+
+def brute_block_scores(q_idx, k_idx, T, block):
+    """[B, T, G, NB] block scores from a full fp64 score matrix (numpy)."""
+    B, _, G, _ = q_idx.shape
+    S = k_idx.shape[1]
+    NB = -(-S // block)
+    s = np.einsum("btgi,bji->btgj", q_idx.astype(np.float64), k_idx.astype(np.float64))
+    pos = S - T + np.arange(T)
+    causal = np.arange(S)[None, :] <= pos[:, None]            # [T, S]
+    s = np.where(causal[None, :, None, :], s, -np.inf)
+    pad = NB * block - S
+    s = np.concatenate([s, np.full(s.shape[:-1] + (pad,), -np.inf)], axis=-1)
+    return s.reshape(B, T, G, NB, block).max(axis=-1)
+
+
+def brute_kept_sets(bs_row, cb, k):
+    """Kept set by counting: n < cb is kept iff fewer than k-1 candidates
+    beat it (higher score, or equal score and lower id)."""
+    kept = {cb}
+    for n in range(cb):
+        better = sum(1 for m in range(cb)
+                     if bs_row[m] > bs_row[n] or (bs_row[m] == bs_row[n] and m < n))
+        if better < k - 1:
+            kept.add(n)
+    return kept
+
+
+def _rows_all(B, T):
+    return np.arange(B * T, dtype=np.int64)
+
+
+def pin_brute_force_selection(lib):
+    rng = np.random.default_rng(7)
+    cases = [  # B, T, S, G, d_idx, block, k
+        (2, 96, 96, 2, 4, 16, 3),
+        (1, 40, 200, 3, 4, 16, 5),     # T < S (bottom-right alignment), S % block != 0
+        (1, 64, 64, 1, 8, 8, 8),
+    ]
+    for B, T, S, G, d_idx, block, k in cases:
+        q = _grid(rng, (B, T, G, d_idx))
+        kk = _grid(rng, (B, S, d_idx))
+        rows = _rows_all(B, T)
+        bs = orc.block_scores(q.reshape(B * T, G, d_idx), kk, rows, T=T, block=block, lib=lib)
+        ref = brute_block_scores(q, kk, T, block).reshape(B * T, G, -1)
+        assert np.array_equal(bs, ref), "block scores differ from brute force"
+        ids = orc.select_blocks(bs, rows, T=T, S=S, block=block, topk=k, lib=lib)
+        for ri in range(B * T):
+            t = ri % T
+            cb = (S - T + t) // block
+            for g in range(G):
+                want = brute_kept_sets(ref[ri, g], cb, k)
+                got = ids[ri, g]
+                n_kept = min(k, cb + 1)
+                assert list(got[:n_kept]) == sorted(want), (ri, g, got, sorted(want))
+                assert np.all(got[n_kept:] == -1)
+
+
+def _sdpa_reference(Q, K, V, allowed, scale):
+    """O and LSE by torch scaled_dot_product_attention (fp64) with a boolean
+    mask allowed [B, T, Hq, S]; GQA by repeating each KV head over its group."""
+    B, T, Hq, d = Q.shape
+    Hkv = K.shape[2]
+    R = Hq // Hkv
+    q = torch.from_numpy(Q.astype(np.float64)).permute(0, 2, 1, 3)          # B Hq T d
+    k = torch.from_numpy(K.astype(np.float64)).permute(0, 2, 1, 3).repeat_interleave(R, dim=1)
+    v = torch.from_numpy(V.astype(np.float64)).permute(0, 2, 1, 3).repeat_interleave(R, dim=1)
+    m = torch.from_numpy(allowed).permute(0, 2, 1, 3)                      # B Hq T S
+    O = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)
+    s = (q @ k.transpose(-1, -2)) * scale
+    lse = torch.logsumexp(s.masked_fill(~m, float("-inf")), dim=-1)
+    return O.permute(0, 2, 1, 3).numpy(), lse.permute(0, 2, 1).numpy()
+
+
+def _allowed_from_ids(ids, B, T, S, Hq, Hkv, block):
+    """Boolean [B, T, Hq, S]: token j allowed iff its block is kept and j <= p(t)."""
+    R = Hq // Hkv
+    allowed = np.zeros((B, T, Hq, S), dtype=bool)
+    tok_block = np.arange(S) // block
+    for b in range(B):
+        for t in range(T):
+            p = S - T + t
+            for h in range(Hq):
+                kept = [n for n in ids[b * T + t, h // R] if n >= 0]
+                allowed[b, t, h] = np.isin(tok_block, kept) & (np.arange(S) <= p)
+    return allowed
+
+
+def pin_dense_limit(lib):
+    rng = np.random.default_rng(11)
+    for B, T, S, Hq, Hkv, d, block in [(1, 48, 48, 4, 2, 8, 8), (2, 20, 70, 6, 3, 16, 16)]:
+        NB = -(-S // block)
+        Q = rng.standard_normal((B, T, Hq, d)).astype(np.float32)
+        K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+        V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+        rows = _rows_all(B, T)
+        ids = np.tile(np.arange(NB, dtype=np.int32), (B * T, Hkv, 1))     # every block kept
+        O, lse = orc.attention(Q.reshape(B * T, Hq, d), K, V, ids, rows, T=T, block=block, lib=lib)
+        allowed = _allowed_from_ids(ids, B, T, S, Hq, Hkv, block)
+        pos = S - T + np.arange(T)
+        dense = np.arange(S)[None, :] <= pos[:, None]
+        assert np.array_equal(allowed, np.broadcast_to(dense[None, :, None, :], allowed.shape))
+        O_ref, lse_ref = _sdpa_reference(Q, K, V, allowed, 1.0 / np.sqrt(d))
+        np.testing.assert_allclose(O, O_ref.reshape(B * T, Hq, d), rtol=0, atol=1e-10)
+        np.testing.assert_allclose(lse, lse_ref.reshape(B * T, Hq), rtol=0, atol=1e-10)
+        # the whole pass with k >= NB is dense causal attention too
+        q_idx = _grid(rng, (B * T, Hkv, 4))
+        k_idx = _grid(rng, (B, S, 4))
+        ids2, O2, lse2 = orc.forward(q_idx, k_idx, Q.reshape(B * T, Hq, d), K, V, rows, T=T,
+                                     block=block, topk=NB, lib=lib)
+        np.testing.assert_allclose(O2, O_ref.reshape(B * T, Hq, d), rtol=0, atol=1e-10)
+        np.testing.assert_allclose(lse2, lse_ref.reshape(B * T, Hq), rtol=0, atol=1e-10)
+
+
+def pin_masked_attention(lib):
+    """Sparse kept sets: equal to SDPA with the kept-block mask."""
+    rng = np.random.default_rng(13)
+    B, T, S, Hq, Hkv, d, d_idx, block, k = 1, 64, 64, 4, 2, 16, 4, 8, 3
+    Q = rng.standard_normal((B, T, Hq, d)).astype(np.float32)
+    K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    q_idx = _grid(rng, (B * T, Hkv, d_idx))
+    k_idx = _grid(rng, (B, S, d_idx))
+    rows = _rows_all(B, T)
+    ids, O, lse = orc.forward(q_idx, k_idx, Q.reshape(B * T, Hq, d), K, V, rows, T=T,
+                              block=block, topk=k, lib=lib)
+    allowed = _allowed_from_ids(ids, B, T, S, Hq, Hkv, block)
+    O_ref, lse_ref = _sdpa_reference(Q, K, V, allowed, 1.0 / np.sqrt(d))
+    np.testing.assert_allclose(O, O_ref.reshape(B * T, Hq, d), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse, lse_ref.reshape(B * T, Hq), rtol=0, atol=1e-10)
+    # an explicit scale is honoured
+    O3, lse3 = orc.attention(Q.reshape(B * T, Hq, d), K, V, ids, rows, T=T, block=block,
+                             scale=0.37, lib=lib)
+    O3_ref, lse3_ref = _sdpa_reference(Q, K, V, allowed, 0.37)
+    np.testing.assert_allclose(O3, O3_ref.reshape(B * T, Hq, d), rtol=0, atol=1e-10)
+    np.testing.assert_allclose(lse3, lse3_ref.reshape(B * T, Hq), rtol=0, atol=1e-10)
+
+
+def pin_closed_forms(lib):
+    rng = np.random.default_rng(17)
+    B, T, S, Hq, Hkv, d, d_idx, block, k = 1, 80, 120, 4, 2, 8, 4, 8, 4
+    NB = -(-S // block)
+    rows = _rows_all(B, T)
+    # all-equal index scores: the tie-break alone decides -> {0..k-2} + {cb}
+    q0 = np.zeros((B * T, Hkv, d_idx), np.float32)
+    kk = _grid(rng, (B, S, d_idx))
+    bs = orc.block_scores(q0, kk, rows, T=T, block=block, lib=lib)
+    ids = orc.select_blocks(bs, rows, T=T, S=S, block=block, topk=k, lib=lib)
+    for ri in range(B * T):
+        cb = (S - T + ri) // block
+        want = sorted(set(range(min(k - 1, cb))) | {cb})
+        for g in range(Hkv):
+            assert list(ids[ri, g, :len(want)]) == want
+            assert np.all(ids[ri, g, len(want):] == -1)
+            # only blocks with a causal token score finitely
+            assert np.all(np.isfinite(bs[ri, g, :cb + 1])) and np.all(bs[ri, g, cb + 1:] == -np.inf)
+    # constant values per (KV head, channel): output equals that constant
+    Q = rng.standard_normal((B * T, Hq, d)).astype(np.float32)
+    K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    c = rng.standard_normal((Hkv, d)).astype(np.float32)
+    V = np.broadcast_to(c, (B, S, Hkv, d)).copy()
+    O, lse = orc.attention(Q, K, V, ids, rows, T=T, block=block, lib=lib)
+    R = Hq // Hkv
+    for h in range(Hq):
+        np.testing.assert_allclose(O[:, h, :], np.broadcast_to(c[h // R], (B * T, d)),
+                                   rtol=0, atol=1e-12)
+    # random values: output inside the per-channel hull of the attended rows,
+    # and max_j s_j <= lse <= max_j s_j + log(#keys)
+    V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    O, lse = orc.attention(Q, K, V, ids, rows, T=T, block=block, lib=lib)
+    for ri in range(B * T):
+        p = S - T + ri
+        for h in range(Hq):
+            g = h // R
+            keys = [j for n in ids[ri, g] if n >= 0
+                    for j in range(n * block, min((n + 1) * block, S)) if j <= p]
+            vv = V[0, keys, g, :].astype(np.float64)
+            assert np.all(O[ri, h] >= vv.min(0) - 1e-12) and np.all(O[ri, h] <= vv.max(0) + 1e-12)
+            s = (K[0, keys, g, :].astype(np.float64) @ Q[ri, h].astype(np.float64)) / np.sqrt(d)
+            assert s.max() - 1e-12 <= lse[ri, h] <= s.max() + np.log(len(keys)) + 1e-12
+    # a query at position 0 attends exactly one key: O = V[0], lse = s_0
+    T1, S1 = 4, 4
+    Q1 = rng.standard_normal((T1, Hq, d)).astype(np.float32)
+    K1 = rng.standard_normal((1, S1, Hkv, d)).astype(np.float32)
+    V1 = rng.standard_normal((1, S1, Hkv, d)).astype(np.float32)
+    ids1 = np.zeros((T1, Hkv, 1), np.int32)
+    O1, lse1 = orc.attention(Q1, K1, V1, ids1, np.arange(T1), T=T1, block=block, lib=lib)
+    for h in range(Hq):
+        g = h // R
+        np.testing.assert_allclose(O1[0, h], V1[0, 0, g], rtol=0, atol=1e-12)
+        s0 = float(Q1[0, h].astype(np.float64) @ K1[0, 0, g].astype(np.float64)) / np.sqrt(d)
+        np.testing.assert_allclose(lse1[0, h], s0, rtol=0, atol=1e-12)
+
+
+def pin_permutation_invariance(lib):
+    rng = np.random.default_rng(19)
+    B, T, S, Hq, Hkv, d, block, k = 1, 64, 64, 4, 2, 8, 8, 4
+    rows = _rows_all(B, T)
+    Q = rng.standard_normal((B * T, Hq, d)).astype(np.float32)
+    K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    q_idx = _grid(rng, (B * T, Hkv, 4))
+    k_idx = _grid(rng, (B, S, 4))
+    ids, O, lse = orc.forward(q_idx, k_idx, Q, K, V, rows, T=T, block=block, topk=k, lib=lib)
+    perm = ids.copy()
+    for ri in range(B * T):
+        for g in range(Hkv):
+            rng.shuffle(perm[ri, g])
+    O2, lse2 = orc.attention(Q, K, V, perm, rows, T=T, block=block, lib=lib)
+    np.testing.assert_allclose(O2, O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse2, lse, rtol=0, atol=1e-12)
+
+
+def pin_bf16_widening(lib):
+    """The same grid values stored as bf16 and as fp32 give identical results
+    (bf16 -> fp64 widening is exact)."""
+    rng = np.random.default_rng(23)
+    B, T, S, Hq, Hkv, d, d_idx, block, k = 1, 48, 48, 4, 2, 8, 8, 8, 3
+    rows = _rows_all(B, T)
+    q_idx = torch.from_numpy(_grid(rng, (B * T, Hkv, d_idx)))
+    k_idx = torch.from_numpy(_grid(rng, (B, S, d_idx)))
+    Q = torch.randn(B * T, Hq, d, generator=torch.Generator().manual_seed(3)).bfloat16()
+    K = torch.randn(B, S, Hkv, d, generator=torch.Generator().manual_seed(4)).bfloat16()
+    V = torch.randn(B, S, Hkv, d, generator=torch.Generator().manual_seed(5)).bfloat16()
+    a = orc.forward(q_idx.bfloat16(), k_idx.bfloat16(), Q, K, V, rows, T=T, block=block,
+                    topk=k, lib=lib, want_scores=True)
+    b = orc.forward(q_idx, k_idx, Q.float(), K.float(), V.float(), rows, T=T, block=block,
+                    topk=k, lib=lib, want_scores=True)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y), "bf16 and fp32 copies of the same values disagree"
+
+
+ALL_PINS = [pin_brute_force_selection, pin_dense_limit, pin_masked_attention,
+            pin_closed_forms, pin_permutation_invariance, pin_bf16_widening]
