@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the MSA-style block-sparse attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one msa_forward over one batch of the 128K-token prefill
+workload (B=1, T=S=131072, Hq=64, Hkv=8, d=128, d_idx=64, B_k=128, k=32,
+bf16): index block scores, per-group Top-k with the current block kept,
+sparse attention with LSE.  The 128K decode workload (64 sequences x 1
+token, S=131072, Hq=32, Hkv=8, B_k=64, k=32) is timed the same way and
+reported under "decode".  Inputs are synthetic, seeded, and resident in HBM
+before timing; they are larger than L2 (126 MB), so no flush is needed.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own
+independent problem (weak scaling, no data-path collective); the time is the
+max over ranks and `value` counts the tokens of all ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores on a bounded
+row sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "prefill_128k"
+DECODE = "decode_128k"
+
+
+# ---------------------------------------------------------------- accounting
+
+def attended_keys(w) -> np.ndarray:
+    """Causal keys each query attends under per-group Top-k with the current
+    block kept: (kept blocks - 1) full blocks plus the causal part of the
+    current block.  Shape [T]."""
+    p = w.S - w.T + np.arange(w.T, dtype=np.int64)
+    cb = p // w.block
+    kept = np.minimum(w.topk, cb + 1)
+    return (kept - 1) * w.block + (p - cb * w.block + 1)
+
+
+def attention_flops(w) -> float:
+    """4 d flops per (query head, attended key): QK^T and PV."""
+    return float(w.B * w.Hq * 4 * w.d * attended_keys(w).sum())
+
+
+def index_flops(w) -> float:
+    """2 d_idx flops per (query, group, causal key)."""
+    p = w.S - w.T + np.arange(w.T, dtype=np.int64)
+    return float(w.B * w.G * 2 * w.d_idx * (p + 1).sum())
+
+
+def decode_bytes(w) -> float:
+    """HBM bytes a decode step must move: all index keys, the kept K/V
+    blocks, the index queries, Q, O, LSE, block scores and ids."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    kept_tokens = attended_keys(w).sum()            # per (sequence, group)
+    kv = w.B * w.G * kept_tokens * w.d * e * 2
+    kidx = w.B * w.S * w.d_idx * e
+    small = w.B * w.T * (w.G * w.d_idx * e + 2 * w.Hq * w.d * e + w.Hq * 4)
+    bs = w.B * w.T * w.G * w.NB * 4 * 2 + w.B * w.T * w.G * w.topk * 4 * 2
+    return float(kv + kidx + small + bs)
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons during a timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU timing
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=600),
+            device_id=torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+    rank = int(os.environ.get("RANK", "0"))
+    return rank, ws
+
+
+def _barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class Problem:
+    """Device-resident inputs, outputs and workspace of one workload."""
+
+    def __init__(self, name: str, seed: int):
+        import block_sparse_long_03_b200 as msa
+        from block_sparse_long_03_b200 import synthetic
+        self.msa = msa
+        self.w = w = synthetic.WORKLOADS[name]
+        self.inp = synthetic.make_inputs(w, seed, device="cuda")
+        i = self.inp
+        self.params = msa.params_from(i.q_idx, i.Q, i.K, block=w.block, topk=w.topk)
+        self.O = torch.empty_like(i.Q)
+        self.lse = torch.empty(i.Q.shape[:3], dtype=torch.float32, device="cuda")
+        self.ids = torch.empty((w.B, w.T, w.G, w.topk), dtype=torch.int32, device="cuda")
+        self.ws = msa.alloc_workspace(self.params, msa.MSA_WS_FORWARD)
+        self.ws_attn = msa.alloc_workspace(self.params, msa.MSA_WS_SPARSE_ATTN)
+        self.bs = torch.empty((w.B, w.T, w.G, w.NB), dtype=torch.float32, device="cuda")
+
+    def step(self, stream=None):
+        i = self.inp
+        self.msa.msa_forward(self.params, i.q_idx, i.k_idx, i.Q, i.K, i.V, self.ids, self.O,
+                             self.lse, self.ws, stream)
+
+    def stage_times_ms(self, reps: int) -> dict:
+        """Average device time of each call of the path, launched on its own."""
+        m, i, s = self.msa, self.inp, torch.cuda.current_stream()
+        stages = {
+            "index_block_scores": lambda: m.msa_index_block_scores(self.params, i.q_idx, i.k_idx,
+                                                                   self.bs),
+            "topk_blocks": lambda: m.msa_topk_blocks(self.params, self.bs, self.ids),
+            "sparse_attn_fwd": lambda: m.msa_sparse_attn_fwd(self.params, i.Q, i.K, i.V, self.ids,
+                                                             self.O, self.lse, self.ws_attn),
+        }
+        out = {}
+        for name, fn in stages.items():
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(reps):
+                fn()
+            e1.record(s)
+            torch.cuda.synchronize()
+            out[name] = e0.elapsed_time(e1) / reps
+        return out
+
+    def free(self):
+        for f in ("inp", "O", "lse", "ids", "ws", "ws_attn", "bs"):
+            setattr(self, f, None)
+        torch.cuda.empty_cache()
+
+
+def time_steps(fn, steps: int, warmup: int, ws: int):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    return _max_over_ranks(e0.elapsed_time(e1) / steps, ws)
+
+
+def e2e_prefill(prob: Problem, steps: int, warmup: int, ws: int) -> dict:
+    """Same metric through the public call with HOST buffers: each step copies
+    the inputs from pinned host memory, runs msa_forward and reads O and LSE
+    back into pinned host memory."""
+    i = prob.inp
+    host_in = [x.cpu().pin_memory() for x in (i.q_idx, i.k_idx, i.Q, i.K, i.V)]
+    dev_in = [torch.empty_like(x) for x in (i.q_idx, i.k_idx, i.Q, i.K, i.V)]
+    host_O = torch.empty(prob.O.shape, dtype=prob.O.dtype, pin_memory=True)
+    host_lse = torch.empty(prob.lse.shape, dtype=prob.lse.dtype, pin_memory=True)
+    m = prob.msa
+
+    def step():
+        for d_, h_ in zip(dev_in, host_in):
+            d_.copy_(h_, non_blocking=True)
+        m.msa_forward(prob.params, *dev_in, prob.ids, prob.O, prob.lse, prob.ws)
+        host_O.copy_(prob.O, non_blocking=True)
+        host_lse.copy_(prob.lse, non_blocking=True)
+
+    ms = time_steps(step, steps, warmup, ws)
+    w = prob.w
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = host_O.numel() * host_O.element_size() + host_lse.numel() * host_lse.element_size()
+    del dev_in
+    return {"value": ws * w.B * w.T / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+def oracle_sample(name: str, budget_s: float, max_rows: int = 4096, seed: int = 7,
+                  host=None):
+    """Run the fp64 oracle (as it stands) on seeded rows of the workload until
+    about `budget_s` seconds of CPU work are done.  Returns (rows/s, rows,
+    seconds, threads).  Inputs are generated on the host with the same recipe."""
+    import oracle
+    from block_sparse_long_03_b200 import synthetic
+    w = synthetic.WORKLOADS[name]
+    if host is None:
+        host = synthetic.make_inputs(w, seed, device="cpu") if w.B * w.T * w.Hq * w.d < 3e9 \
+            else None
+    if host is None:
+        raise RuntimeError("workload too large to generate on the host")
+    rng = np.random.default_rng(seed)
+    done, elapsed, batch = 0, 0.0, 2
+    while elapsed < budget_s and done < max_rows:
+        rows = np.sort(rng.integers(0, w.B * w.T, size=batch))
+        for b in np.unique(rows // w.T):
+            ts = rows[rows // w.T == b] % w.T
+            tt = torch.from_numpy(ts)
+            t0 = time.perf_counter()
+            oracle.forward(host.q_idx[b].index_select(0, tt), host.k_idx[b:b + 1],
+                           host.Q[b].index_select(0, tt), host.K[b:b + 1], host.V[b:b + 1], ts,
+                           T=w.T, block=w.block, topk=w.topk)
+            elapsed += time.perf_counter() - t0
+        done += batch
+        batch = min(batch * 2, 64)
+    return done / elapsed, done, elapsed, oracle.num_threads()
+
+
+def run_reference(args, rank: int, ws: int):
+    if rank != 0:
+        return
+    from block_sparse_long_03_b200 import synthetic
+    w = synthetic.WORKLOADS[args.workload]
+    host = synthetic.make_inputs(w, 7, device="cpu")
+    budget = float(os.environ.get("MSA_REF_STEP_SECONDS", "8"))
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, 0.5, max_rows=2, host=host)
+    rates, rows_total, secs_total, threads = [], 0, 0.0, 1
+    for _ in range(args.steps):
+        rate, rows, secs, threads = oracle_sample(args.workload, budget / max(args.steps, 1),
+                                                  host=host)
+        rates.append(rate)
+        rows_total += rows
+        secs_total += secs
+    value = rows_total / secs_total
+    sample = (f"{rows_total} seeded query rows of {w.name} (all {w.Hq} heads each), "
+              f"{secs_total:.1f} s of oracle time")
+    line = {
+        "impl": "reference", "metric": "MSA prefill tokens/s @128K", "value": value,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs_total / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "d": w.d, "d_idx": w.d_idx, "block": w.block, "topk": w.topk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- main
+
+def run_ours(args, rank: int, ws: int):
+    import block_sparse_long_03_b200 as msa
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    pk = peaks()
+    prob = Problem(args.workload, seed=rank)
+    w = prob.w
+    launches0 = msa.msa_kernel_launches()
+    with ClockSampler(local) as clk:
+        ms = time_steps(prob.step, args.steps, args.warmup, ws)
+    timed_launches = msa.msa_kernel_launches() - launches0
+    per_step = timed_launches / float(args.steps + args.warmup)
+    value = ws * w.B * w.T / (ms / 1e3)
+    stages = prob.stage_times_ms(max(2, args.steps))
+    attn_fl, idx_fl = attention_flops(w), index_flops(w)
+    dominant = max(stages, key=stages.get)
+    if dominant == "index_block_scores":
+        ach = idx_fl / (stages[dominant] / 1e3) / 1e12
+    else:
+        ach = attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12
+        dominant = "sparse_attn_fwd"
+    roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,
+            "peak_source": pk["source"] + " bf16 burst (of " + pk["source"] + ")",
+            "stage_ms": stages,
+            "attention_tflops": attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12,
+            "index_tflops": idx_fl / (stages["index_block_scores"] / 1e3) / 1e12}
+    e2e = None if args.no_e2e else e2e_prefill(prob, max(1, min(args.steps, 3)), 1, ws)
+    prob.free()
+    del prob
+
+    decode = None
+    if not args.no_decode:
+        dp = Problem(DECODE, seed=100 + rank)
+        with ClockSampler(local) as dclk:
+            dms = time_steps(dp.step, max(args.steps, 10), args.warmup, ws)
+        dst = dp.stage_times_ms(max(args.steps, 10))
+        db = decode_bytes(dp.w)
+        decode = {"workload": DECODE, "us_per_step": dms * 1e3, "bytes_per_step": db,
+                  "achieved_gbs": db / (dms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+                  "frac": db / (dms / 1e3) / 1e9 / pk["hbm_gbs"], "stage_ms": dst,
+                  "clocks": dclk.summary()}
+        dp.free()
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, rows, secs, threads = oracle_sample(args.workload, args.cpu_seconds)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{rows} seeded query rows of {w.name}, {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": "MSA prefill tokens/s @128K", "value": value, "unit": "tokens/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; Q/K/V ~ N(0,1), index q/k on a 1/4 grid, hot blocks)",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq,
+                       "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx, "block": w.block,
+                       "topk": w.topk, "parallelism": f"replicas x{ws}",
+                       "l2": "inputs larger than L2 (Q alone 2 GiB); no flush"},
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(round(per_step * args.steps)),
+            "clocks": clk.summary(), "decode": decode,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=PREFILL)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, ws = _dist()
+    try:
+        run_ours(args, rank, ws)
+    finally:
+        if ws > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,190 @@
+"""Thin Python binding of the C ABI in ``include/msa.h``.
+
+Argument marshalling only: every function takes torch CUDA tensors, checks
+dtypes and shapes, and passes raw device pointers plus the current CUDA
+stream to ``libmsa.so``.  All computation happens in the library's CUDA
+kernels.  If the library is missing the import fails loudly; there is no
+fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmsa.so")
+
+MSA_OK = 0
+MSA_F32, MSA_BF16 = 0, 1
+MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD = 0, 1
+STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
+                4: "MSA_ERR_DEVICE_TIMEOUT", 5: "MSA_ERR_WORKSPACE", 6: "MSA_ERR_BAD_BLOCK_IDS"}
+
+# Every symbol the header declares (checked by the CPU test suite).
+EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
+           "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
+           "msa_kernel_launches")
+
+
+class MsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class Params(ctypes.Structure):
+    """msa_params_t."""
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "T", "S", "Hq", "Hkv", "d", "d_idx", "block", "topk", "dtype")] + \
+               [("scale", ctypes.c_float)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
+                          "(run python -m block_sparse_long_03_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, P = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Params)
+    st = ctypes.c_int
+    lib.msa_status_string.argtypes = [st]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_index_block_scores.argtypes = [P, vp, vp, vp, vp]
+    lib.msa_topk_blocks.argtypes = [P, vp, vp, vp]
+    lib.msa_workspace_size.argtypes = [P, ctypes.c_int]
+    lib.msa_workspace_size.restype = sz
+    lib.msa_sparse_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_get_device_error.argtypes = [vp, vp]
+    lib.msa_kernel_launches.argtypes = []
+    lib.msa_kernel_launches.restype = ctypes.c_uint64
+    for name in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd",
+                 "msa_forward", "msa_get_device_error"):
+        getattr(lib, name).restype = st
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.msa_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != MSA_OK:
+        raise MsaError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def make_params(*, B, T, S, Hq, Hkv, d, d_idx, block, topk, dtype, scale=0.0) -> Params:
+    code = {torch.float32: MSA_F32, torch.bfloat16: MSA_BF16}[dtype]
+    return Params(B, T, S, Hq, Hkv, d, d_idx, block, topk, code, float(scale))
+
+
+def params_from(q_idx, Q, K, *, block: int, topk: int, scale: float = 0.0) -> Params:
+    B, T, Hq, d = Q.shape
+    S, Hkv = K.shape[1], K.shape[2]
+    return make_params(B=B, T=T, S=S, Hq=Hq, Hkv=Hkv, d=d, d_idx=q_idx.shape[-1], block=block,
+                       topk=topk, dtype=Q.dtype, scale=scale)
+
+
+def msa_workspace_size(params: Params, which: int) -> int:
+    return int(lib.msa_workspace_size(ctypes.byref(params), int(which)))
+
+
+def alloc_workspace(params: Params, which: int, device=None) -> torch.Tensor:
+    n = msa_workspace_size(params, which)
+    if n == 0:
+        raise MsaError(1, "msa_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def msa_index_block_scores(params: Params, q_idx, k_idx, block_scores, stream=None):
+    _check(lib.msa_index_block_scores(ctypes.byref(params), _ptr(q_idx), _ptr(k_idx),
+                                      _ptr(block_scores), _stream(stream)),
+           "msa_index_block_scores")
+
+
+def msa_topk_blocks(params: Params, block_scores, block_ids, stream=None):
+    _check(lib.msa_topk_blocks(ctypes.byref(params), _ptr(block_scores), _ptr(block_ids),
+                               _stream(stream)), "msa_topk_blocks")
+
+
+def msa_sparse_attn_fwd(params: Params, Q, K, V, block_ids, O, lse, workspace, stream=None):
+    _check(lib.msa_sparse_attn_fwd(ctypes.byref(params), _ptr(Q), _ptr(K), _ptr(V),
+                                   _ptr(block_ids), _ptr(O), _ptr(lse), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "msa_sparse_attn_fwd")
+
+
+def msa_forward(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, workspace,
+                stream=None):
+    _check(lib.msa_forward(ctypes.byref(params), _ptr(q_idx), _ptr(k_idx), _ptr(Q), _ptr(K),
+                           _ptr(V), _ptr(block_ids), _ptr(O), _ptr(lse), _ptr(workspace),
+                           workspace.numel(), _stream(stream)), "msa_forward")
+
+
+def msa_get_device_error(workspace, stream=None) -> int:
+    """The status recorded on the device by the last call that used `workspace`."""
+    return int(lib.msa_get_device_error(_ptr(workspace), _stream(stream)))
+
+
+def msa_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib.msa_kernel_launches())
+
+
+# ---- convenience wrappers that allocate outputs with torch ----------------
+
+def index_block_scores(q_idx, k_idx, *, block: int, T: int | None = None):
+    B, T_, G, d_idx = q_idx.shape
+    S = k_idx.shape[1]
+    p = make_params(B=B, T=T_, S=S, Hq=G, Hkv=G, d=64, d_idx=d_idx, block=block, topk=1,
+                    dtype=q_idx.dtype)
+    bs = torch.empty((B, T_, G, S // block), dtype=torch.float32, device=q_idx.device)
+    msa_index_block_scores(p, q_idx, k_idx, bs)
+    return bs
+
+
+def topk_blocks(block_scores, *, S: int, block: int, topk: int):
+    B, T, G, NB = block_scores.shape
+    p = make_params(B=B, T=T, S=S, Hq=G, Hkv=G, d=64, d_idx=16, block=block, topk=topk,
+                    dtype=torch.float32)
+    ids = torch.empty((B, T, G, topk), dtype=torch.int32, device=block_scores.device)
+    msa_topk_blocks(p, block_scores, ids)
+    return ids
+
+
+def sparse_attn_fwd(Q, K, V, block_ids, *, block: int, scale: float = 0.0):
+    B, T, Hq, d = Q.shape
+    S, Hkv = K.shape[1], K.shape[2]
+    p = make_params(B=B, T=T, S=S, Hq=Hq, Hkv=Hkv, d=d, d_idx=16, block=block,
+                    topk=block_ids.shape[-1], dtype=Q.dtype, scale=scale)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, T, Hq), dtype=torch.float32, device=Q.device)
+    ws = alloc_workspace(p, MSA_WS_SPARSE_ATTN, Q.device)
+    msa_sparse_attn_fwd(p, Q, K, V, block_ids, O, lse, ws)
+    return O, lse, ws
+
+
+def forward(q_idx, k_idx, Q, K, V, *, block: int, topk: int, scale: float = 0.0):
+    """The whole forward pass; returns (O, lse, block_ids, workspace)."""
+    p = params_from(q_idx, Q, K, block=block, topk=topk, scale=scale)
+    O = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
+    ids = torch.empty((*Q.shape[:2], K.shape[2], topk), dtype=torch.int32, device=Q.device)
+    ws = alloc_workspace(p, MSA_WS_FORWARD, Q.device)
+    msa_forward(p, q_idx, k_idx, Q, K, V, ids, O, lse, ws)
+    return O, lse, ids, ws

@@ -1,0 +1,56 @@
+// msa_internal.cuh -- declarations shared by the library's translation units.
+// Not part of the public interface (that is include/msa.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/msa.h"
+
+namespace msa {
+
+// Shapes after host-side validation, with derived sizes.
+struct Shape {
+    int B, T, S, Hq, Hkv, G, R, d, d_idx, block, topk, NB;
+    int dtype;          // MSA_F32 or MSA_BF16
+    float scale;        // resolved softmax scale
+    int64_t rows() const { return (int64_t)B * T; }          // query tokens
+    int64_t index_rows() const { return rows() * G; }        // (token, group) rows
+};
+
+// Device error word: the first 256 bytes of every workspace.
+//   word[0]: first recorded msa_status_t (0 = none)
+//   word[1]: number of caller block ids skipped as invalid
+//   word[2]: number of bounded device waits that gave up
+constexpr size_t kErrorBytes = 256;
+
+__device__ __forceinline__ void record_error(uint32_t *err, uint32_t code, int counter) {
+    if (err == nullptr) return;
+    atomicCAS(err, 0u, code);
+    atomicAdd(err + counter, 1u);
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Every kernel launch of the library is counted (msa_kernel_launches).
+void count_launches(int n);
+
+// Launchers (each returns a cudaError_t from the launch).
+cudaError_t launch_index_scores_simt(const Shape &s, const void *q_idx, const void *k_idx,
+                                     float *bs, cudaStream_t st);
+cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st);
+cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
+                             const int32_t *ids, void *O, float *lse, uint32_t *err,
+                             cudaStream_t st);
+
+}  // namespace msa

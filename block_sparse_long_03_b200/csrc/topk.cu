@@ -1,0 +1,135 @@
+// topk.cu -- per-group Top-k over blocks with the current block forced.
+//
+// ("MiniMax Sparse Attention", Summary, second paragraph: each GQA group
+// picks its own Top-k blocks and the block containing the current position
+// is always kept; Key points, benchmark configuration: the current block is
+// one of the k.)
+//
+// For row (b, t, g) with cb = p(t) / block, the kept set is cb plus the
+// M = topk - 1 best candidates n < cb, ranked by (score descending, id
+// ascending).  Scores are compared as fp32 bit patterns mapped to an
+// order-preserving uint32 -- nothing is exponentiated.
+//
+// One warp per row.  The candidates' ordered keys are staged in shared
+// memory, then a 4-pass radix select (8 bits per pass, warp-private
+// histogram) finds the M-th largest score u*.  Every candidate above u* is
+// kept, and of the candidates equal to u* the lowest ids are kept until M is
+// reached.  A final pass in ascending id order emits the kept ids with
+// ballots, so the output is ascending without a sort; cb is appended last
+// (it is larger than every candidate) and unused slots get -1.
+#include "msa_internal.cuh"
+
+namespace msa {
+namespace {
+
+__device__ __forceinline__ uint32_t ordered_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids,
+                            int64_t nrows, int T_, int S, int G, int NB, int block, int topk,
+                            int warps_per_cta) {
+    extern __shared__ uint32_t sm[];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t r = (int64_t)blockIdx.x * warps_per_cta + warp;
+    if (r >= nrows) return;
+    uint32_t *keys = sm + (size_t)warp * (NB + 256);
+    uint32_t *hist = keys + NB;
+    const int t = (int)((r / G) % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int M = topk - 1;
+    int32_t *out = ids + r * topk;
+    const unsigned lt_mask = (1u << lane) - 1u;
+
+    if (M == 0) {                     // only the forced block
+        if (lane == 0) out[0] = cb;
+        return;
+    }
+    if (cb <= M) {                    // every causal block is kept
+        for (int i = lane; i < topk; i += 32) out[i] = (i <= cb) ? i : -1;
+        return;
+    }
+    const float *row = bs + r * NB;
+    for (int n = lane; n < cb; n += 32) keys[n] = ordered_key(row[n]);
+    __syncwarp();
+
+    uint32_t prefix = 0, mask = 0;
+    int remaining = M;                // how many still to take at or below prefix
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = lane; i < 256; i += 32) hist[i] = 0;
+        __syncwarp();
+        for (int n = lane; n < cb; n += 32) {
+            const uint32_t v = keys[n];
+            if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        // lane L owns digits [8L, 8L + 8); suffix sums over digits, high to low
+        uint32_t c[8], lane_sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { c[i] = hist[lane * 8 + i]; lane_sum += c[i]; }
+        uint32_t above = 0;           // count in lanes > this lane
+        {
+            uint32_t incl = lane_sum; // inclusive suffix sum over lanes >= lane
+#pragma unroll
+            for (int off = 1; off < 32; off *= 2) {
+                const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += o;
+            }
+            above = incl - lane_sum;
+        }
+        // the digit D where the running count from the top first reaches `remaining`
+        int found = -1;
+        uint32_t gt_count = 0;
+        if (above < (uint32_t)remaining && above + lane_sum >= (uint32_t)remaining) {
+            uint32_t acc = above;
+            for (int i = 7; i >= 0; --i) {
+                if (acc + c[i] >= (uint32_t)remaining) { found = lane * 8 + i; gt_count = acc; break; }
+                acc += c[i];
+            }
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = __ffs(who) - 1;
+        const int digit = __shfl_sync(0xffffffffu, found, src);
+        gt_count = __shfl_sync(0xffffffffu, gt_count, src);
+        prefix |= (uint32_t)digit << shift;
+        mask |= 255u << shift;
+        remaining -= (int)gt_count;
+        __syncwarp();
+    }
+    // prefix == u*, `remaining` ties at u* are to be taken, lowest ids first
+    int ties_seen = 0, written = 0;
+    for (int base = 0; base < cb; base += 32) {
+        const int n = base + lane;
+        const uint32_t v = (n < cb) ? keys[n] : 0u;
+        const bool eq = (n < cb) && v == prefix;
+        const unsigned eq_b = __ballot_sync(0xffffffffu, eq);
+        const int tie_rank = ties_seen + __popc(eq_b & lt_mask);
+        const bool take = (n < cb) && (v > prefix || (eq && tie_rank < remaining));
+        const unsigned tk_b = __ballot_sync(0xffffffffu, take);
+        const int pos = written + __popc(tk_b & lt_mask);
+        if (take && pos < M) out[pos] = n;
+        ties_seen += __popc(eq_b);
+        written += __popc(tk_b);
+    }
+    if (lane == 0) out[M] = cb;
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st) {
+    const int64_t nrows = s.index_rows();
+    const size_t per_warp = sizeof(uint32_t) * ((size_t)s.NB + 256);
+    int warps = 8;
+    while (warps > 1 && per_warp * warps > 200 * 1024) warps /= 2;
+    if (per_warp * warps > 220 * 1024) return cudaErrorInvalidConfiguration;
+    const size_t smem = per_warp * warps;
+    cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t grid = (nrows + warps - 1) / warps;
+    topk_kernel<<<(unsigned)grid, warps * 32, smem, st>>>(bs, ids, nrows, s.T, s.S, s.G, s.NB,
+                                                          s.block, s.topk, warps);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -6,7 +6,7 @@ check draw their inputs from here, and the same tensors feed both the CUDA
 library and the fp64 oracle.
 
 Value recipe (the pages fix no data, so these are stated choices):
-  * Q, K, V ~ N(0, 1), rounded to the workload dtype;
+  * Q, K, V ~ N(0, 1), drawn in the workload dtype;
   * index queries and keys q_idx, k_idx = randint[-4, 4] / 4, so that every
     index dot product is a multiple of 1/32 well inside fp32's exact range;
   * "hot" blocks (prefill workloads): a shared seeded direction u with
@@ -111,19 +111,20 @@ def make_inputs(w: Workload, seed: int, device="cpu") -> Inputs:
             mark[ids] = True
         tok = mark.repeat_interleave(w.block)[:S]
         k_idx[:, tok, :] += u
-    Q = torch.randn((B, T, w.Hq, w.d), generator=gen, device=device, dtype=torch.float32)
-    K = torch.randn((B, S, w.Hkv, w.d), generator=gen, device=device, dtype=torch.float32)
-    V = torch.randn((B, S, w.Hkv, w.d), generator=gen, device=device, dtype=torch.float32)
     dt = w.dtype
-    return Inputs(q_idx.to(dt), k_idx.to(dt), Q.to(dt), K.to(dt), V.to(dt), hot, u)
+    Q = torch.randn((B, T, w.Hq, w.d), generator=gen, device=device, dtype=dt)
+    K = torch.randn((B, S, w.Hkv, w.d), generator=gen, device=device, dtype=dt)
+    V = torch.randn((B, S, w.Hkv, w.d), generator=gen, device=device, dtype=dt)
+    return Inputs(q_idx.to(dt), k_idx.to(dt), Q, K, V, hot, u)
 
 
 def sample_rows(w: Workload, n: int, seed: int = 1234) -> list:
     """Rows r = b * T + t for a sampled parity check: the first and last rows
-    of every batch entry, rows at block boundaries, plus seeded random rows."""
+    and rows at the first block boundary of the first and last batch entries,
+    plus `n` seeded random rows."""
     g = torch.Generator().manual_seed(seed)
     rows = set()
-    for b in range(w.B):
+    for b in sorted({0, w.B - 1}):
         base = b * w.T
         rows.update({base, base + w.T - 1})
         if w.T > 1:

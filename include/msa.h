@@ -1,0 +1,179 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) library for the forward pass of
+ * MiniMax-Sparse-Attention-style block-sparse grouped-query attention.
+ *
+ * The method ("MiniMax Sparse Attention -- paper by Lai et al. (2026)",
+ * section "Summary", second paragraph; section "Key points"): a light index
+ * branch scores every KV block for each query by max-pooling token-level dot
+ * products of an index query with index keys; each GQA group keeps its own
+ * Top-k blocks, the block holding the query's own position always among
+ * them; exact softmax attention then runs over the kept blocks only, and the
+ * log-sum-exp of that softmax is a forward output.
+ *
+ * Notation used below:
+ *   G = Hkv            one index head per GQA group; KV head g is group g
+ *   R = Hq / Hkv       query heads per group; head h is in group h / R
+ *   NB = S / block     KV blocks (S must be a multiple of block)
+ *   p(t) = S - T + t   absolute position of query t (bottom-right causal
+ *                      alignment; prefill with T == S gives p(t) = t)
+ *   cb(t) = p(t) / block   the query's own ("current") block
+ *
+ * Conventions shared by every call:
+ *   - Every tensor pointer is DEVICE memory, dense and row-major in the
+ *     layout stated at the call, 16-byte aligned.  The caller allocates and
+ *     owns all of it, workspace included; the library allocates nothing and
+ *     keeps no state between calls other than per-device launch settings.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  A returned MSA_OK means the work was
+ *     enqueued; device-side problems are recorded in the workspace's error
+ *     word and read back with msa_get_device_error.
+ *   - Invalid arguments are rejected on the host, before anything is
+ *     enqueued.  No C++ exception crosses this interface.
+ *   - Floating-point element type: MSA_BF16 (bf16 storage, fp32
+ *     accumulation) or MSA_F32 (fp32 throughout).  The index tensors, Q, K,
+ *     V and O all use params->dtype; block scores and LSE are always fp32;
+ *     block ids are int32.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_EXPORT __attribute__((visibility("default")))
+#else
+#define MSA_EXPORT
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MSA_OK = 0,
+    MSA_ERR_INVALID_ARG = 1,     /* null pointer, bad shape, misalignment     */
+    MSA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. d=96)     */
+    MSA_ERR_CUDA = 3,            /* a CUDA runtime call failed                */
+    MSA_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device wait gave up             */
+    MSA_ERR_WORKSPACE = 5,       /* workspace missing or too small            */
+    MSA_ERR_BAD_BLOCK_IDS = 6    /* caller ids out of range / not causal      */
+} msa_status_t;
+
+typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype_t;
+
+/* Shapes of one call.  All fields are required. */
+typedef struct {
+    int32_t B;       /* batch (independent sequences)                       */
+    int32_t T;       /* query tokens per sequence, 1 <= T <= S              */
+    int32_t S;       /* keys per sequence, a multiple of block              */
+    int32_t Hq;      /* query heads                                         */
+    int32_t Hkv;     /* KV heads = GQA groups = index heads; Hq % Hkv == 0  */
+    int32_t d;       /* head dimension: 64 or 128                           */
+    int32_t d_idx;   /* index head dimension: a multiple of 16, <= 128      */
+    int32_t block;   /* KV block size B_k: 64 or 128                        */
+    int32_t topk;    /* blocks kept per (query, group), current one included */
+    int32_t dtype;   /* msa_dtype_t                                         */
+    float scale;     /* softmax scale; <= 0 selects 1/sqrt(d)               */
+} msa_params_t;
+
+/* Human-readable name of a status code (static storage). */
+MSA_EXPORT const char *msa_status_string(msa_status_t status);
+
+/*
+ * Index branch: block scores ("Summary", second paragraph: blocks are
+ * scored by max-pooling token-level dot products).
+ *
+ *   block_scores[b, t, g, n] = max over j in block n with j <= p(t) of
+ *                              sum_i q_idx[b, t, g, i] * k_idx[b, j, i]
+ *   and -infinity when block n starts after p(t).
+ *
+ * q_idx        [B, T, G, d_idx]  dtype      (read)
+ * k_idx        [B, S, d_idx]     dtype      (read)
+ * block_scores [B, T, G, NB]     float32    (written)
+ * The token-level scores are never written to memory.
+ */
+MSA_EXPORT msa_status_t msa_index_block_scores(const msa_params_t *params, const void *q_idx,
+                                    const void *k_idx, float *block_scores, void *stream);
+
+/*
+ * Per-group Top-k over blocks with the current block forced ("Summary",
+ * second paragraph: each GQA group picks its own Top-k blocks and the block
+ * containing the current position is always kept; "Key points", benchmark
+ * configuration: the current block is one of the k).
+ *
+ * For each (b, t, g): kept = {cb(t)} united with the topk - 1 best blocks
+ * n < cb(t), best meaning the larger block score and, on equal scores, the
+ * lower block id.  min(topk, cb(t) + 1) ids are written in ascending order
+ * and the remaining slots are set to -1.  Scores are compared as fp32 and
+ * never exponentiated.
+ *
+ * block_scores [B, T, G, NB]    float32  (read; only n < cb(t) is read)
+ * block_ids    [B, T, G, topk]  int32    (written)
+ */
+MSA_EXPORT msa_status_t msa_topk_blocks(const msa_params_t *params, const float *block_scores,
+                             int32_t *block_ids, void *stream);
+
+/* Workspace needs, in bytes, of msa_sparse_attn_fwd (which = 0) and
+ * msa_forward (which = 1) for these shapes; 0 for invalid shapes. */
+#define MSA_WS_SPARSE_ATTN 0
+#define MSA_WS_FORWARD 1
+MSA_EXPORT size_t msa_workspace_size(const msa_params_t *params, int which);
+
+/*
+ * Main branch: exact softmax attention over the kept blocks ("Summary",
+ * second paragraph) with the log-sum-exp as a second output ("Key points",
+ * kernel design: LSE is fused into the forward pass).
+ *
+ * For each (b, t, h) with g = h / R and J = the tokens j <= p(t) of the
+ * blocks listed in block_ids[b, t, g, :] (entries < 0 are empty slots):
+ *   s_j = scale * sum_c Q[b, t, h, c] * K[b, j, g, c]
+ *   O[b, t, h, :] = sum_j softmax(s)_j V[b, j, g, :]
+ *   lse[b, t, h]  = log(sum_j exp(s_j))      (natural log)
+ * The order of the ids in a row does not matter.  Caller ids are not
+ * trusted: an id >= NB, or an id repeated within a row, is skipped (a repeat
+ * counts once) and the device error word records MSA_ERR_BAD_BLOCK_IDS.  An
+ * id above cb(t) holds no causal token and adds nothing.  A row with no
+ * attended key gets O = 0 and lse = -infinity.
+ *
+ * Q [B, T, Hq, d], K and V [B, S, Hkv, d] (dtype, read);
+ * block_ids [B, T, G, topk] int32 (read); O [B, T, Hq, d] (dtype, written);
+ * lse [B, T, Hq] float32 (written).
+ * workspace: device memory of at least msa_workspace_size(params, 0) bytes,
+ * 256-byte aligned; its first 256 bytes hold the device error word.
+ */
+MSA_EXPORT msa_status_t msa_sparse_attn_fwd(const msa_params_t *params, const void *Q, const void *K,
+                                 const void *V, const int32_t *block_ids, void *O, float *lse,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The whole forward pass: index scores, Top-k and sparse attention, fused
+ * where that pays.  Same meaning and layouts as the three calls above.
+ * block_ids may be NULL (the ids then live in the workspace only); when not
+ * NULL it receives the kept ids [B, T, G, topk].  workspace must hold
+ * msa_workspace_size(params, 1) bytes.
+ */
+MSA_EXPORT msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const void *k_idx,
+                         const void *Q, const void *K, const void *V, int32_t *block_ids,
+                         void *O, float *lse, void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * Read the device error word of a workspace (synchronises `stream`) and
+ * clear it.  Returns MSA_OK when no kernel recorded a problem, otherwise
+ * the recorded status (MSA_ERR_BAD_BLOCK_IDS, MSA_ERR_DEVICE_TIMEOUT).
+ */
+MSA_EXPORT msa_status_t msa_get_device_error(void *workspace, void *stream);
+
+/*
+ * Diagnostics: the number of CUDA kernels this library has launched in this
+ * process since it was loaded (all devices, all calls).  Lets a caller count
+ * the kernels a region of work issued.
+ */
+MSA_EXPORT uint64_t msa_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

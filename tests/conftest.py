@@ -25,3 +25,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionstart(session):
+    # The CUDA library and the oracle are built in-tree (nvcc cross-compiles
+    # sm_100a without a GPU); rebuild them if a source is newer.
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_msa_build", os.path.join(ROOT, "block_sparse_long_03_b200", "build.py"))
+    lib_build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(lib_build)
+    lib_build.build()
+    import oracle
+    oracle.build()

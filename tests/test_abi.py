@@ -1,0 +1,105 @@
+"""The C-ABI library loads and exports every symbol the header declares, and
+rejects invalid arguments on the host (no GPU is touched by these tests:
+every call here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MSA_EXPORT\s+[\w\s\*]*?\b(msa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_symbols()
+    for want in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd", "msa_forward",
+                 "msa_workspace_size", "msa_status_string", "msa_get_device_error",
+                 "msa_kernel_launches"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    import block_sparse_long_03_b200 as msa
+    from block_sparse_long_03_b200 import binding
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), f"{name} declared in msa.h but not exported"
+    assert set(declared_symbols()) == set(msa.EXPORTS)
+
+
+def _p(**kw):
+    import torch
+    from block_sparse_long_03_b200 import make_params
+    base = dict(B=1, T=256, S=256, Hq=8, Hkv=2, d=128, d_idx=64, block=128, topk=2,
+                dtype=torch.bfloat16)
+    base.update(kw)
+    return make_params(**base)
+
+
+def test_status_strings():
+    from block_sparse_long_03_b200 import binding
+    for code, name in binding.STATUS_NAMES.items():
+        assert binding.status_string(code).startswith(name)
+    assert "unknown" in binding.status_string(99)
+
+
+def test_workspace_sizes():
+    from block_sparse_long_03_b200 import binding
+    p = _p()
+    ws_attn = binding.msa_workspace_size(p, binding.MSA_WS_SPARSE_ATTN)
+    ws_fwd = binding.msa_workspace_size(p, binding.MSA_WS_FORWARD)
+    assert ws_attn >= 256 and ws_fwd >= 256
+    # forward holds at least the block scores and the ids
+    assert ws_fwd >= 256 + 4 * (1 * 256 * 2 * 2) + 4 * (1 * 256 * 2 * 2)
+    assert binding.msa_workspace_size(_p(T=0), binding.MSA_WS_FORWARD) == 0
+    assert binding.msa_workspace_size(p, 7) == 0
+
+
+BAD_SHAPES = [
+    (dict(T=0), 1), (dict(T=512), 1), (dict(Hq=6, Hkv=4), 1), (dict(topk=0), 1),
+    (dict(B=-1), 1), (dict(S=320), 2), (dict(d=96), 2), (dict(block=32), 2),
+    (dict(d_idx=24), 2), (dict(Hq=64, Hkv=2), 2), (dict(topk=1000), 2),
+]
+
+
+@pytest.mark.parametrize("kw,status", BAD_SHAPES)
+def test_bad_shapes_rejected_on_host(kw, status):
+    from block_sparse_long_03_b200 import binding
+    p = _p(**kw)
+    fake = ctypes.c_void_p(0x10000)       # never dereferenced: validation fails first
+    ws = ctypes.c_void_p(0x20000)
+    lib = binding.lib
+    assert lib.msa_index_block_scores(ctypes.byref(p), fake, fake, fake, None) == status
+    assert lib.msa_topk_blocks(ctypes.byref(p), fake, fake, None) == status
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, ws,
+                                   1 << 30, None) == status
+    assert lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, ws,
+                           1 << 30, None) == status
+
+
+def test_null_and_misaligned_pointers_rejected():
+    from block_sparse_long_03_b200 import binding
+    lib = binding.lib
+    p = _p()
+    ok = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)        # 8-byte aligned only
+    ws = ctypes.c_void_p(0x20000)
+    assert lib.msa_index_block_scores(None, ok, ok, ok, None) == 1
+    assert lib.msa_index_block_scores(ctypes.byref(p), None, ok, ok, None) == 1
+    assert lib.msa_index_block_scores(ctypes.byref(p), odd, ok, ok, None) == 1
+    assert lib.msa_topk_blocks(ctypes.byref(p), ok, None, None) == 1
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), ok, ok, ok, ok, ok, odd, ws, 1 << 30,
+                                   None) == 1
+    # workspace: null, misaligned, too small
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), ok, ok, ok, ok, ok, ok, None, 1 << 30,
+                                   None) == 5
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), ok, ok, ok, ok, ok, ok,
+                                   ctypes.c_void_p(0x20010), 1 << 30, None) == 5
+    assert lib.msa_forward(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, ws, 16, None) == 5
+    assert lib.msa_get_device_error(None, None) == 5
