@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
-           "msa_kernel_launches")
+           "msa_kernel_launches", "msa_forward_noalloc")
 
 
 class MsaError(RuntimeError):
@@ -44,7 +44,7 @@ class Params(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"CUDA library not built: {LIB_PATH} is missing "
-                          "(run python -m block_sparse_long_03_b200.build)")
+                          "(run python block_sparse_long_03_b200/build.py)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, sz, P = ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(Params)
     st = ctypes.c_int
@@ -57,6 +57,8 @@ def _load():
     lib.msa_sparse_attn_fwd.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_get_device_error.argtypes = [vp, vp]
+    lib.msa_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.msa_forward_noalloc.restype = st
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = ctypes.c_uint64
     for name in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd",

@@ -1,6 +1,6 @@
 """Build the CUDA library ``libmsa.so`` in-tree for sm_100a with nvcc.
 
-    python -m block_sparse_long_03_b200.build [--force]
+    python block_sparse_long_03_b200/build.py [--force]
 
 The library is the product: every kernel of the forward pass lives in
 ``csrc/*.cu`` and the C ABI is ``include/msa.h``.

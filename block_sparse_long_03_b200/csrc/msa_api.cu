@@ -166,3 +166,71 @@ msa_status_t msa_get_device_error(void *workspace, void *stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// msa_forward_noalloc: msa_forward for callers that cannot allocate device
+// memory (see include/msa.h).  Its scratch is a fixed file-scope device
+// array, so every GPU that loads this library holds kNoAllocScratchBytes for
+// the life of the process.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace msa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)MSA_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status_t msa_forward_noalloc(const msa_params_t *params, const void *q_idx,
+                                            const void *k_idx, const void *Q, const void *K,
+                                            const void *V, int32_t *block_ids, void *O,
+                                            float *lse, void *stream) {
+    Shape s;
+    msa_status_t rc = make_shape(params, &s);
+    if (rc != MSA_OK) return rc;
+    if (!q_idx || !k_idx || !Q || !K || !V || !O || !lse) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(Q) || !aligned16(K) ||
+        !aligned16(V) || !aligned16(O) || !aligned16(lse) ||
+        (block_ids && !aligned16(block_ids)))
+        return MSA_ERR_INVALID_ARG;
+    if (forward_ws(s) > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return MSA_ERR_CUDA;
+    cudaStream_t st = (cudaStream_t)stream;
+    char *ws = (char *)scratch;
+    uint32_t *err = (uint32_t *)ws;
+    float *bs = (float *)(ws + kErrorBytes);
+    int32_t *ids = block_ids ? block_ids
+                             : (int32_t *)(ws + kErrorBytes + align_up(block_score_bytes(s)));
+    cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);   // error word starts at zero
+    if (e == cudaSuccess) e = launch_index_scores_simt(s, q_idx, k_idx, bs, st);
+    if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
+    if (e == cudaSuccess) e = launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
+    return cuda_status(e);
+}

@@ -166,6 +166,38 @@ MSA_EXPORT msa_status_t msa_forward(const msa_params_t *params, const void *q_id
 MSA_EXPORT msa_status_t msa_get_device_error(void *workspace, void *stream);
 
 /*
+ * msa_forward for callers that cannot allocate device memory: code that
+ * runs where cudaMalloc is unavailable or forbidden (for example inside a
+ * host callback, a custom allocator's own hooks, or an embedding runtime
+ * that owns all device allocations), or that must not add allocations to a
+ * tightly budgeted process.  The paper has no counterpart of this call.
+ *
+ * Same meaning, layouts and outputs as msa_forward, but no workspace is
+ * passed: the block scores, ids and error word live in a fixed scratch
+ * array of MSA_NOALLOC_SCRATCH_BYTES that the library defines as a device
+ * global.  Every GPU that loads the library holds that array until the
+ * process exits.  The call itself allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine).
+ *   - Shapes whose scratch (msa_workspace_size(params, MSA_WS_FORWARD))
+ *     exceeds MSA_NOALLOC_SCRATCH_BYTES are rejected with MSA_ERR_WORKSPACE
+ *     before anything is enqueued.
+ *   - The first call on each device looks up the array's device address
+ *     (once per device, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps the last
+ *     call's contents.  Calls that may overlap on the GPU (different
+ *     streams, or host threads racing on the same device) race on it:
+ *     serialise them.
+ *   - The call clears the error word itself; the ids come from the call's
+ *     own Top-k, so no caller id is checked.
+ */
+#define MSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+MSA_EXPORT msa_status_t msa_forward_noalloc(const msa_params_t *params, const void *q_idx,
+                                            const void *k_idx, const void *Q, const void *K,
+                                            const void *V, int32_t *block_ids, void *O,
+                                            float *lse, void *stream);
+
+/*
  * Diagnostics: the number of CUDA kernels this library has launched in this
  * process since it was loaded (all devices, all calls).  Lets a caller count
  * the kernels a region of work issued.
