@@ -23,8 +23,9 @@ def _check_all_rows_valid(ids, w):
     valid = ids >= 0
     assert torch.equal(valid.sum(-1), n_keep.expand(B, T, G)), "wrong number of kept ids"
     slot = torch.arange(k, device=ids.device).view(1, 1, 1, k)
-    assert torch.equal(valid, slot < n_keep.unsqueeze(-1)), "ids not packed at the front"
-    big = torch.where(valid, ids, torch.full_like(ids, 1 << 30))
+    assert torch.equal(valid, (slot < n_keep.unsqueeze(-1)).expand_as(valid)), \
+        "ids not packed at the front"
+    big = torch.where(valid, ids, (1 << 30) + slot.expand_as(ids).to(ids.dtype))
     assert bool((big[..., 1:] > big[..., :-1]).all()), "ids not strictly ascending"
     assert bool((torch.where(valid, ids, cb.unsqueeze(-1)) <= cb.unsqueeze(-1)).all())
     last = ids.gather(-1, (n_keep - 1).unsqueeze(-1).expand(B, T, G, 1)).squeeze(-1)
