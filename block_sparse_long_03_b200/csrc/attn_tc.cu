@@ -1,0 +1,642 @@
+// attn_tc.cu -- sparse attention over the kept blocks on the tensor cores
+// (bf16 prefill), KV-block-outer.
+//
+// Main branch ("MiniMax Sparse Attention", Summary, second paragraph: exact
+// softmax attention restricted to the kept blocks; Key points, kernel design:
+// pre-scheduled chunks, a two-phase combine, and the LSE produced by the
+// forward pass).  For query (b, t), head h in group g, over the causal
+// tokens j <= p(t) of the kept blocks:
+//   O = sum_j softmax(scale * Q.K_j) V_j,   lse = log sum_j exp(scale * Q.K_j).
+//
+// Each (query, group) keeps its own blocks, so the query heads that share a
+// kept block are only the R = Hq/Hkv heads of one token -- too few rows for
+// a tensor-core tile.  The work is therefore turned around: for every
+// (batch, group, block n) the tokens that kept n are listed (a CSR built on
+// the device), and a tile is up to 128/R of those tokens times their R
+// heads = 128 rows, against the 128 (or 64) keys of block n:
+//   phase 1  S = Q K_n^T (tcgen05, SS), block-local softmax in registers,
+//            P (bf16) to TMEM, O_n = P V_n (tcgen05, A from TMEM), written as
+//            a normalised fp16 partial plus its LSE, one per (query, head,
+//            kept slot);
+//   phase 2  per (query, head): LSE-weighted combine of the partials of its
+//            kept slots -> O (bf16) and lse (fp32).
+// Work is chunked over query rows so the partial buffer stays bounded.
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include <algorithm>
+
+#include "tc.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kRows = 128;           // tile rows = tokens_per_tile * R
+constexpr int kThreads = 320;        // warp 0 load, warp 1 MMA, warps 2-9 softmax/epilogue
+constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Validity of slot `i` of a kept-id row, shared by every phase: in range, not
+// a repeat of an earlier slot, and holding at least one causal token.
+__device__ __forceinline__ bool slot_valid(const int32_t *row, int i, int NB, int cb,
+                                           bool *bad) {
+    const int n = row[i];
+    *bad = false;
+    if (n < 0) return false;
+    if (n >= NB) { *bad = true; return false; }
+    for (int k = 0; k < i; ++k)
+        if (row[k] == n) { *bad = true; return false; }
+    return n <= cb;
+}
+
+// ---------------------------------------------------------------- CSR build
+
+// counts[(b*G + g)*NB + n] += 1 for every valid kept slot of the chunk's rows.
+__global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restrict__ counts,
+                                 uint32_t *err, int64_t r0, int64_t rc, int T_, int S, int G,
+                                 int NB, int block, int topk) {
+    const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= rc * G) return;
+    const int64_t r = r0 + x / G;                 // b * T + t
+    const int g = (int)(x % G);
+    const int b = (int)(r / T_), t = (int)(r % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int32_t *row = ids + (r * G + g) * topk;
+    for (int i = 0; i < topk; ++i) {
+        bool bad;
+        if (slot_valid(row, i, NB, cb, &bad))
+            atomicAdd(&counts[((int64_t)b * G + g) * NB + row[i]], 1);
+        else if (bad)
+            record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+    }
+}
+
+// Single-CTA exclusive scans: offs = scan(counts), tile_offs = scan(ceil(counts / tpt)).
+// offs[L] and tile_offs[L] hold the totals.
+__global__ void csr_scan_kernel(const int *__restrict__ counts, int *__restrict__ offs,
+                                int *__restrict__ tile_offs, int L, int tpt) {
+    __shared__ int s_a[1024], s_b[1024];
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (L + nt - 1) / nt;
+    const int lo = min(L, tid * per), hi = min(L, lo + per);
+    int a = 0, b = 0;
+    for (int i = lo; i < hi; ++i) { a += counts[i]; b += (counts[i] + tpt - 1) / tpt; }
+    s_a[tid] = a;
+    s_b[tid] = b;
+    __syncthreads();
+    for (int off = 1; off < nt; off *= 2) {       // inclusive Hillis-Steele scan
+        const int va = tid >= off ? s_a[tid - off] : 0;
+        const int vb = tid >= off ? s_b[tid - off] : 0;
+        __syncthreads();
+        s_a[tid] += va;
+        s_b[tid] += vb;
+        __syncthreads();
+    }
+    int ea = s_a[tid] - a, eb = s_b[tid] - b;      // exclusive
+    for (int i = lo; i < hi; ++i) {
+        offs[i] = ea;
+        tile_offs[i] = eb;
+        ea += counts[i];
+        eb += (counts[i] + tpt - 1) / tpt;
+    }
+    if (tid == nt - 1) { offs[L] = s_a[nt - 1]; tile_offs[L] = s_b[nt - 1]; }
+}
+
+// entries[offs[list] + k] = (row - r0) << 8 | slot, for every valid kept slot.
+__global__ void csr_fill_kernel(const int32_t *__restrict__ ids, const int *__restrict__ offs,
+                                int *__restrict__ cursor, int *__restrict__ entries, int64_t r0,
+                                int64_t rc, int T_, int S, int G, int NB, int block, int topk) {
+    const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= rc * G) return;
+    const int64_t r = r0 + x / G;
+    const int g = (int)(x % G);
+    const int b = (int)(r / T_), t = (int)(r % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int32_t *row = ids + (r * G + g) * topk;
+    for (int i = 0; i < topk; ++i) {
+        bool bad;
+        if (!slot_valid(row, i, NB, cb, &bad)) continue;
+        const int64_t list = ((int64_t)b * G + g) * NB + row[i];
+        const int pos = atomicAdd(&cursor[list], 1);
+        entries[offs[list] + pos] = (int)(((r - r0) << 8) | i);
+    }
+}
+
+// tiles[tile_offs[list] + c] = {list, tokens in the tile, index of its first
+// entry, 0} for every tile of every list.
+__global__ void csr_tiles_kernel(const int *__restrict__ counts, const int *__restrict__ offs,
+                                 const int *__restrict__ tile_offs, int4 *__restrict__ tiles,
+                                 int L, int tpt) {
+    const int list = blockIdx.x * blockDim.x + threadIdx.x;
+    if (list >= L) return;
+    const int cnt = counts[list];
+    const int nt = (cnt + tpt - 1) / tpt;
+    const int base = tile_offs[list];
+    for (int c = 0; c < nt; ++c)
+        tiles[base + c] = make_int4(list, min(tpt, cnt - c * tpt), offs[list] + c * tpt, 0);
+}
+
+}  // namespace
+}  // namespace msa
+
+namespace msa {
+namespace {
+
+struct AttnArgs {
+    const __nv_bfloat16 *Q;     // [B, T, Hq, D]
+    const int *entries;         // CSR entries: (row - r0) << 8 | slot
+    const int4 *tiles;          // {list, count, first entry, 0} per tile
+    const int *n_tiles;         // device-side tile count
+    __half *part_o;             // [rc * G * topk * R, D] normalised partial outputs
+    float *part_lse;            // [rc * G * topk * R]
+    uint32_t *err;
+    int64_t r0;
+    int T, S, Hq, G, R, NB, topk, tpt;
+    float scale, scale_log2;
+};
+
+__device__ __forceinline__ int run_tile(int i) {
+    return (i / kRun) * (gridDim.x * kRun) + blockIdx.x * kRun + (i % kRun);
+}
+
+__device__ __forceinline__ int4 load_tile(const AttnArgs &a, int i, int total) {
+    const int tile = run_tile(i);
+    return tile < total ? a.tiles[tile] : make_int4(-1, 0, 0, 0);
+}
+
+template <int D, int BLOCK>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
+    constexpr int kAtoms = D / 64;
+    constexpr uint32_t kQBytes = kRows * D * 2;
+    constexpr uint32_t kKBytes = BLOCK * D * 2;
+    constexpr uint32_t kAccCols = 256;            // S (BLOCK) + O (D) per accumulator set
+    static_assert(BLOCK + D <= (int)kAccCols, "TMEM budget");
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sQ = smem;                           // [2][kAtoms][128][64]
+    uint8_t *sK = sQ + 2 * kQBytes;               // [2][kAtoms][BLOCK][64]
+    uint8_t *sV = sK + 2 * kKBytes;               // [2][kAtoms][BLOCK][64]
+    uint64_t *bar = (uint64_t *)(sV + 2 * kKBytes);
+    uint64_t *q_full = bar, *q_empty = bar + 2, *kv_full = bar + 4, *kv_empty = bar + 6;
+    uint64_t *s_full = bar + 8, *p_full = bar + 10, *o_full = bar + 12, *acc_empty = bar + 14;
+    uint32_t *tmem_slot = (uint32_t *)(bar + 16);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 32);
+            tc::mbar_init(&q_empty[i], 1);
+            tc::mbar_init(&kv_full[i], 1);
+            tc::mbar_init(&kv_empty[i], 1);
+            tc::mbar_init(&s_full[i], 1);
+            tc::mbar_init(&p_full[i], 128);
+            tc::mbar_init(&o_full[i], 1);
+            tc::mbar_init(&acc_empty[i], 128);
+        }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total = *a.n_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------ loads: K/V blocks and Q rows by TMA
+        // The next tile's descriptor and entries are fetched one tile ahead.
+        int kvb = -1, cur_list = -1, kv_ph[2] = {0, 0}, q_ph[2] = {0, 0};
+        int4 nd = load_tile(a, 0, total);
+        int ne[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int tt = lane + 32 * k;
+            ne[k] = tt < nd.y ? a.entries[nd.z + tt] : 0;
+        }
+        for (int i = 0;; ++i) {
+            const int4 d = nd;
+            int e[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) e[k] = ne[k];
+            if (d.x < 0 || *abort_flag) break;
+            nd = load_tile(a, i + 1, total);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int tt = lane + 32 * k;
+                ne[k] = tt < nd.y ? a.entries[nd.z + tt] : 0;
+            }
+            const int list = d.x, count = d.y;
+            const int n = list % a.NB, g = (list / a.NB) % a.G, b = list / (a.NB * a.G);
+            if (list != cur_list) {
+                kvb = (kvb + 1) & 1;
+                cur_list = list;
+                if (lane == 0 && tc::mbar_wait(&kv_empty[kvb], kv_ph[kvb] ^ 1, a.err, abort_flag)) {
+                    tc::mbar_expect_tx(&kv_full[kvb], 2 * kKBytes);
+                    const int key0 = b * a.S + n * BLOCK;
+#pragma unroll
+                    for (int at = 0; at < kAtoms; ++at) {
+                        tc::tma_load_3d(sK + kvb * kKBytes + at * BLOCK * 128, &tm_k,
+                                        &kv_full[kvb], at * 64, g, key0);
+                        tc::tma_load_3d(sV + kvb * kKBytes + at * BLOCK * 128, &tm_v,
+                                        &kv_full[kvb], at * 64, g, key0);
+                    }
+                }
+                kv_ph[kvb] ^= 1;
+            }
+            const int qb = i & 1;
+            if (!tc::mbar_wait(&q_empty[qb], q_ph[qb] ^ 1, a.err, abort_flag)) break;
+            q_ph[qb] ^= 1;
+            uint8_t *dst = sQ + qb * kQBytes;
+            if (a.R >= 8) {
+                // One TMA box per token: its R heads x 64 channels, R * 128 bytes, so
+                // every box starts on a 1024-byte swizzle-atom boundary.
+                if (lane == 0) tc::mbar_expect_tx(&q_full[qb], (uint32_t)count * a.R * D * 2);
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int tt = lane + 32 * k;
+                    if (tt < count) {
+                        const int grow = (int)(a.r0 + (e[k] >> 8));
+#pragma unroll
+                        for (int at = 0; at < kAtoms; ++at)
+                            tc::tma_load_3d(dst + at * kRows * 128 + tt * a.R * 128, &tm_q,
+                                            &q_full[qb], at * 64, g * a.R, grow);
+                    }
+                }
+            } else {
+                // Fewer than 8 heads per token: a token's rows do not fill a swizzle
+                // atom, so the rows are gathered with 16-byte cp.async copies into
+                // the 128-byte-swizzled layout directly.
+                constexpr int kChunksPerRow = D / 8;
+                const int nchunks = count * a.R * kChunksPerRow;
+                for (int c = lane; c < nchunks; c += 32) {
+                    const int r = c / kChunksPerRow, cc = c % kChunksPerRow;
+                    const int tk = r / a.R, hh = r % a.R;
+                    const int eval = a.entries[d.z + tk];
+                    const int64_t grow = a.r0 + (eval >> 8);
+                    const __nv_bfloat16 *src =
+                        a.Q + (grow * a.Hq + (int64_t)g * a.R + hh) * D + cc * 8;
+                    const uint32_t sa = tc::smem_u32(dst + (cc / 8) * (kRows * 128) + r * 128 +
+                                                     (((cc % 8) ^ (r % 8)) * 16));
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(src)
+                                 : "memory");
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                tc::fence_proxy_async();
+                tc::mbar_arrive(&q_full[qb]);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
+            int kvb = -1, cur_list = -1, kv_ph[2] = {0, 0}, q_ph[2] = {0, 0};
+            int acc_ph[2] = {0, 0}, p_ph[2] = {0, 0};
+            int prev_acc = -1, prev_kvb = -1, prev_list = -1;
+            int next_list = load_tile(a, 0, total).x;
+            for (int i = 0;; ++i) {
+                const int list = next_list;
+                const bool have = list >= 0 && !*abort_flag;
+                if (have) {
+                    next_list = load_tile(a, i + 1, total).x;
+                    if (list != cur_list) {
+                        kvb = (kvb + 1) & 1;
+                        cur_list = list;
+                        kv_ph[kvb] ^= 1;
+                    }
+                    const int acc = i & 1, qb = i & 1;
+                    if (!tc::mbar_wait(&acc_empty[acc], acc_ph[acc] ^ 1, a.err, abort_flag)) break;
+                    acc_ph[acc] ^= 1;
+                    if (!tc::mbar_wait(&q_full[qb], q_ph[qb], a.err, abort_flag)) break;
+                    q_ph[qb] ^= 1;
+                    if (!tc::mbar_wait(&kv_full[kvb], kv_ph[kvb] ^ 1, a.err, abort_flag)) break;
+                    tc::tc_fence_after();
+                    const uint32_t qa = tc::smem_u32(sQ + qb * kQBytes);
+                    const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks) {
+                        const uint64_t ad =
+                            tc::sdesc_sw128(qa + (ks / 4) * kRows * 128 + (ks % 4) * 32, 16, 1024);
+                        const uint64_t bd =
+                            tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
+                        tc::mma_ss(tmem + acc * kAccCols, ad, bd, idesc_s, ks > 0);
+                    }
+                    tc::mma_commit(&q_empty[qb]);
+                    tc::mma_commit(&s_full[acc]);
+                }
+                if (prev_acc >= 0) {
+                    // O = P V for the previous tile (P from TMEM, V from shared memory)
+                    if (!tc::mbar_wait(&p_full[prev_acc], p_ph[prev_acc], a.err, abort_flag)) break;
+                    p_ph[prev_acc] ^= 1;
+                    tc::tc_fence_after();
+                    const uint32_t va = tc::smem_u32(sV + prev_kvb * kKBytes);
+#pragma unroll
+                    for (int ks = 0; ks < BLOCK / 16; ++ks) {
+                        const uint64_t bd = tc::sdesc_sw128(va + ks * 2048, BLOCK * 128, 1024);
+                        tc::mma_ts(tmem + prev_acc * kAccCols + BLOCK,
+                                   tmem + prev_acc * kAccCols + ks * 8, bd, idesc_o, ks > 0);
+                    }
+                    tc::mma_commit(&o_full[prev_acc]);
+                    if (list != prev_list) tc::mma_commit(&kv_empty[prev_kvb]);
+                }
+                if (!have) break;
+                prev_acc = i & 1;
+                prev_kvb = kvb;
+                prev_list = list;
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax + epilogue (two groups)
+        const int grp = (warp - 2) / 4;
+        const int quad = warp % 4;
+        const int row = quad * 32 + lane;
+        const int tt = row / a.R, h = row % a.R;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t tS = tmem + grp * kAccCols + lane_off;
+        const uint32_t tO = tS + BLOCK;
+        int ph = 0;
+        int4 nd = load_tile(a, grp, total);
+        int nent = tt < nd.y ? a.entries[nd.z + tt] : 0;
+        for (int i = grp;; i += 2) {
+            const int4 d = nd;
+            const int ent = nent;
+            if (d.x < 0 || *abort_flag) break;
+            nd = load_tile(a, i + 2, total);
+            nent = tt < nd.y ? a.entries[nd.z + tt] : 0;
+            const int list = d.x;
+            const int n = list % a.NB, g = (list / a.NB) % a.G;
+            const bool valid = tt < d.y;
+            const int t = (int)((a.r0 + (ent >> 8)) % a.T);
+            const int64_t p = (int64_t)a.S - a.T + t;
+            const int64_t j_base = (int64_t)n * BLOCK;
+            if (!tc::mbar_wait(&s_full[grp], ph, a.err, abort_flag)) break;
+            tc::tc_fence_after();
+            uint32_t sreg[BLOCK];
+#pragma unroll
+            for (int c = 0; c < BLOCK; c += 32) tc::tmem_ld32(tS + c, *(uint32_t(*)[32])(sreg + c));
+            tc::tmem_ld_wait();
+            const bool masked = valid && (j_base + BLOCK - 1 > p);
+            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+            if (!masked) {
+#pragma unroll
+                for (int c = 0; c < BLOCK; c += 4) {
+                    m0 = fmaxf(m0, __uint_as_float(sreg[c]));
+                    m1 = fmaxf(m1, __uint_as_float(sreg[c + 1]));
+                    m2 = fmaxf(m2, __uint_as_float(sreg[c + 2]));
+                    m3 = fmaxf(m3, __uint_as_float(sreg[c + 3]));
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < BLOCK; ++c)
+                    if (j_base + c <= p) m0 = fmaxf(m0, __uint_as_float(sreg[c]));
+            }
+            float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+            if (!valid) m = 0.f;
+            const float mb = m * a.scale_log2;
+            float l0 = 0.f, l1 = 0.f;
+            uint32_t preg[BLOCK / 2];
+#pragma unroll
+            for (int c = 0; c < BLOCK; c += 2) {
+                float p0 = exp2f(fmaf(__uint_as_float(sreg[c]), a.scale_log2, -mb));
+                float p1 = exp2f(fmaf(__uint_as_float(sreg[c + 1]), a.scale_log2, -mb));
+                if (!valid || (masked && j_base + c > p)) p0 = 0.f;
+                if (!valid || (masked && j_base + c + 1 > p)) p1 = 0.f;
+                l0 += p0;
+                l1 += p1;
+                __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+                preg[c / 2] = *(uint32_t *)&pk;
+            }
+            const float l = l0 + l1;
+#pragma unroll
+            for (int c = 0; c < BLOCK / 2; c += 32)
+                tc::tmem_st32(tS + c, *(const uint32_t(*)[32])(preg + c));
+            tc::tmem_st_wait();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&p_full[grp]);
+            if (!tc::mbar_wait(&o_full[grp], ph, a.err, abort_flag)) break;
+            tc::tc_fence_after();
+            uint32_t oreg[D];
+#pragma unroll
+            for (int c = 0; c < D; c += 32) tc::tmem_ld32(tO + c, *(uint32_t(*)[32])(oreg + c));
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&acc_empty[grp]);
+            ph ^= 1;
+            if (valid) {
+                const int slot = ent & 255;
+                const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
+                const float inv_l = 1.f / l;
+                uint4 *dst = (uint4 *)(a.part_o + prow * D);
+#pragma unroll
+                for (int c = 0; c < D; c += 8) {
+                    __half2 h0 = __floats2half2_rn(__uint_as_float(oreg[c]) * inv_l,
+                                                   __uint_as_float(oreg[c + 1]) * inv_l);
+                    __half2 h1 = __floats2half2_rn(__uint_as_float(oreg[c + 2]) * inv_l,
+                                                   __uint_as_float(oreg[c + 3]) * inv_l);
+                    __half2 h2 = __floats2half2_rn(__uint_as_float(oreg[c + 4]) * inv_l,
+                                                   __uint_as_float(oreg[c + 5]) * inv_l);
+                    __half2 h3 = __floats2half2_rn(__uint_as_float(oreg[c + 6]) * inv_l,
+                                                   __uint_as_float(oreg[c + 7]) * inv_l);
+                    uint4 u;
+                    u.x = *(uint32_t *)&h0; u.y = *(uint32_t *)&h1;
+                    u.z = *(uint32_t *)&h2; u.w = *(uint32_t *)&h3;
+                    dst[c / 8] = u;
+                }
+                a.part_lse[prow] = m * a.scale + logf(l);
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_free(tmem, 512);
+    }
+}
+
+}  // namespace
+}  // namespace msa
+
+namespace msa {
+namespace {
+
+// Phase 2: one warp per (query row, head).  The partials of the row's valid
+// kept slots are merged with weights exp(lse_i - max lse); the result is the
+// softmax over the union of the slots' keys.
+template <int D>
+__global__ void combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_o,
+                               const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
+                               float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
+                               int Hq, int G, int R, int NB, int block, int topk) {
+    constexpr int kPer = D / 32;                  // output channels per lane
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (wid >= rc * Hq) return;
+    const int64_t rl = wid / Hq;                  // row within the chunk
+    const int hq = (int)(wid % Hq);
+    const int g = hq / R, h = hq % R;
+    const int64_t r = r0 + rl;
+    const int t = (int)(r % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int32_t *row = ids + (r * G + g) * topk;
+    float m = -INFINITY, l = 0.f, acc[kPer];
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+    for (int base = 0; base < topk; base += 32) {
+        bool bad;
+        const int i = base + lane;
+        const bool ok = i < topk && slot_valid(row, i, NB, cb, &bad);
+        unsigned mask = __ballot_sync(0xffffffffu, ok);
+        while (mask) {
+            const int s = base + __ffs(mask) - 1;
+            mask &= mask - 1;
+            const int64_t prow = ((rl * G + g) * topk + s) * R + h;
+            const float li = part_lse[prow];
+            const float m_new = fmaxf(m, li);
+            const float a_old = expf(m - m_new), w = expf(li - m_new);
+            const __half *src = part_o + prow * D + lane * kPer;
+            float v[kPer];
+            if (kPer == 4) {
+                const uint2 u = *(const uint2 *)src;
+                const float2 f0 = __half22float2(*(const __half2 *)&u.x);
+                const float2 f1 = __half22float2(*(const __half2 *)&u.y);
+                v[0] = f0.x; v[1] = f0.y; v[2 % kPer] = f1.x; v[3 % kPer] = f1.y;
+            } else {
+#pragma unroll
+                for (int c = 0; c < kPer; ++c) v[c] = __half2float(src[c]);
+            }
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) acc[c] = acc[c] * a_old + w * v[c];
+            l = l * a_old + w;
+            m = m_new;
+        }
+    }
+    __nv_bfloat16 *dst = O + (r * Hq + hq) * D + lane * kPer;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) dst[c] = __float2bfloat16_rn(acc[c] * inv);
+    if (lane == 0) lse[r * Hq + hq] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+constexpr size_t kPartialBudget = (size_t)4 << 30;   // bytes of partials per chunk
+constexpr size_t kA = 256;
+size_t al(size_t x) { return (x + kA - 1) / kA * kA; }
+
+struct Plan {
+    int64_t rows_per_chunk;
+    int tpt;
+    int64_t L;
+    size_t counts, cursor, offs, toffs, entries, tiles, part_o, part_lse, total;
+};
+
+Plan make_plan(const Shape &s) {
+    Plan p;
+    p.tpt = kRows / s.R;
+    p.L = (int64_t)s.B * s.G * s.NB;
+    const size_t per_row = (size_t)s.G * s.topk * s.R * (2 * (size_t)s.d + 4);
+    int64_t rc = (int64_t)(kPartialBudget / per_row);
+    if (rc < 1) rc = 1;
+    if (rc > s.rows()) rc = s.rows();
+    p.rows_per_chunk = rc;
+    const size_t slots = (size_t)rc * s.G * s.topk;
+    size_t o = 0;
+    p.counts = o;   o += al(sizeof(int) * p.L);
+    p.cursor = o;   o += al(sizeof(int) * p.L);
+    p.offs = o;     o += al(sizeof(int) * (p.L + 1));
+    p.toffs = o;    o += al(sizeof(int) * (p.L + 1));
+    p.entries = o;  o += al(sizeof(int) * slots);
+    p.tiles = o;    o += al(sizeof(int4) * (slots + p.L));
+    p.part_o = o;   o += al(sizeof(__half) * slots * s.R * s.d);
+    p.part_lse = o; o += al(sizeof(float) * slots * s.R);
+    p.total = o;
+    return p;
+}
+
+template <int D, int BLOCK>
+cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void *V,
+                       const int32_t *ids, void *O, float *lse, uint32_t *err, char *ws,
+                       cudaStream_t st) {
+    const Plan pl = make_plan(s);
+    CUtensorMap tq, tk, tv;
+    const uint64_t dims[3] = {(uint64_t)s.d, (uint64_t)s.Hkv, (uint64_t)s.B * s.S};
+    const uint64_t strides[2] = {(uint64_t)s.d * 2, (uint64_t)s.Hkv * s.d * 2};
+    const uint32_t box[3] = {64, 1, (uint32_t)BLOCK};
+    if (!make_tmap_bf16(&tk, K, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tv, V, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    // Q as [B*T, Hq, d]: one box = the R heads of one token (R rows of 64 channels)
+    const uint64_t qdims[3] = {(uint64_t)s.d, (uint64_t)s.Hq, (uint64_t)s.B * s.T};
+    const uint64_t qstrides[2] = {(uint64_t)s.d * 2, (uint64_t)s.Hq * s.d * 2};
+    const uint32_t qbox[3] = {64, (uint32_t)s.R, 1};
+    if (!make_tmap_bf16(&tq, Q, 3, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
+    int *counts = (int *)(ws + pl.counts), *cursor = (int *)(ws + pl.cursor);
+    int *offs = (int *)(ws + pl.offs), *toffs = (int *)(ws + pl.toffs);
+    int *entries = (int *)(ws + pl.entries);
+    int4 *tiles = (int4 *)(ws + pl.tiles);
+    __half *part_o = (__half *)(ws + pl.part_o);
+    float *part_lse = (float *)(ws + pl.part_lse);
+    const size_t smem = 1024 + 2 * (size_t)kRows * D * 2 + 4 * (size_t)BLOCK * D * 2 + 256;
+    auto kern = attn_tc_kernel<D, BLOCK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int L = (int)pl.L;
+    for (int64_t r0 = 0; r0 < s.rows(); r0 += pl.rows_per_chunk) {
+        const int64_t rc = std::min<int64_t>(pl.rows_per_chunk, s.rows() - r0);
+        e = cudaMemsetAsync(counts, 0, pl.offs - pl.counts, st);   // counts and cursor
+        if (e != cudaSuccess) return e;
+        const int64_t nrow = rc * s.G;
+        const unsigned g1 = (unsigned)((nrow + 255) / 256);
+        csr_count_kernel<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB,
+                                             s.block, s.topk);
+        csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offs, toffs, L, pl.tpt);
+        csr_fill_kernel<<<g1, 256, 0, st>>>(ids, offs, cursor, entries, r0, rc, s.T, s.S, s.G,
+                                            s.NB, s.block, s.topk);
+        csr_tiles_kernel<<<(L + 255) / 256, 256, 0, st>>>(counts, offs, toffs, tiles, L, pl.tpt);
+        AttnArgs a{};
+        a.Q = (const __nv_bfloat16 *)Q;
+        a.entries = entries;
+        a.tiles = tiles;
+        a.n_tiles = toffs + L;
+        a.part_o = part_o; a.part_lse = part_lse; a.err = err; a.r0 = r0;
+        a.T = s.T; a.S = s.S; a.Hq = s.Hq; a.G = s.G; a.R = s.R; a.NB = s.NB; a.topk = s.topk;
+        a.tpt = pl.tpt;
+        a.scale = s.scale;
+        a.scale_log2 = s.scale * kLog2e;
+        kern<<<sms, kThreads, smem, st>>>(tq, tk, tv, a);
+        const int64_t warps = rc * s.Hq;
+        combine_kernel<D><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+            ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R,
+            s.NB, s.block, s.topk);
+        count_launches(6);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Shape &s) {
+    return s.dtype == MSA_BF16 && s.d == 128 && (s.block == 128 || s.block == 64) &&
+           (s.R == 1 || s.R == 2 || s.R == 4 || s.R == 8 || s.R == 16) && s.topk <= 256;
+}
+
+size_t attn_tc_workspace(const Shape &s) { return make_plan(s).total; }
+
+cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
+                           const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
+                           cudaStream_t st) {
+    if (s.block == 128)
+        return run_chunks<128, 128>(s, Q, K, V, ids, O, lse, err, (char *)ws, st);
+    return run_chunks<128, 64>(s, Q, K, V, ids, O, lse, err, (char *)ws, st);
+}
+
+}  // namespace msa

@@ -1,0 +1,293 @@
+// index_tc.cu -- index branch on the tensor cores (bf16 prefill).
+//
+// Block scores ("MiniMax Sparse Attention", Summary, second paragraph:
+// blocks are scored by max-pooling token-level index dot products):
+//   bs[b, t, g, n] = max_{j in block n, j <= p(t)} q_idx[b, t, g, :] . k_idx[b, j, :]
+//
+// The token-level scores form a GEMM: rows are the (token, group) pairs of
+// q_idx viewed as a [B*T*G, d_idx] matrix, columns are index keys.  A work
+// item is (batch entry, 128-row tile, chunk of key tiles).  Per key tile of
+// 256 keys, one elected thread issues tcgen05.mma (M=128, N=256, K=16 steps,
+// bf16 in, fp32 accumulate) into one of two TMEM accumulators; the TMA
+// producer keeps a ring of k_idx tiles in shared memory; four epilogue warps
+// read the accumulator back (each thread owns one row), apply the causal
+// mask j <= p(t) and max-pool every block's columns, so only one fp32 per
+// (row, block) reaches HBM.  With index inputs on the 1/4 grid every dot
+// product is exact in fp32, so the scores equal the fp64 definition.
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
+// owner, warps 2-9 epilogue in two groups of four, one per TMEM accumulator
+// (warp w reads TMEM lanes 32*(w%4) .. +31).
+#include <math.h>
+
+#include "tc.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kM = 128;            // rows per tile
+constexpr int kN = 256;            // keys per MMA tile
+constexpr int kThreads = 320;          // 2 + 8 warps
+constexpr int kKtChunk = 32;       // key tiles per work item
+
+struct IndexArgs {
+    float *bs;
+    uint32_t *err;
+    int B, T, S, G, NB, block, d_idx;
+    int MT;                        // row tiles per batch entry
+    int CPT;                       // chunks per row tile (max over tiles)
+    int items;
+    int fill_noncausal;            // write -inf for blocks past the tile's key range
+};
+
+struct Item {
+    int b, mt, kt0, kt1, nkt;
+    bool valid;
+};
+
+__device__ __forceinline__ Item decode_item(const IndexArgs &a, int i) {
+    Item it;
+    const int c = i % a.CPT;
+    const int rest = i / a.CPT;
+    it.mt = a.MT - 1 - (rest % a.MT);          // large causal ranges first
+    it.b = rest / a.MT;
+    const int rows = a.T * a.G;
+    const int r_hi = min(rows - 1, it.mt * kM + kM - 1);
+    const int64_t p_hi = (int64_t)a.S - a.T + r_hi / a.G;
+    it.nkt = (int)(p_hi / kN) + 1;
+    it.kt0 = c * kKtChunk;
+    it.kt1 = min(it.nkt, it.kt0 + kKtChunk);
+    it.valid = it.kt0 < it.nkt;
+    return it;
+}
+
+template <int DIDX, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                IndexArgs a) {
+    constexpr int kAtoms = DIDX / 64;                     // 128-byte swizzle atoms along d_idx
+    constexpr uint32_t kABytes = kM * DIDX * 2;
+    constexpr uint32_t kBBytes = kN * DIDX * 2;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = smem;                                   // [2][kAtoms][kM][64]
+    uint8_t *sB = smem + 2 * kABytes;                     // [STAGES][kAtoms][kN][64]
+    uint64_t *bar = (uint64_t *)(sB + STAGES * kBBytes);
+    uint64_t *a_full = bar, *a_empty = bar + 2;
+    uint64_t *b_full = bar + 4, *b_empty = bar + 4 + STAGES;
+    uint64_t *acc_full = bar + 4 + 2 * STAGES, *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = (uint32_t *)(acc_empty + 2);
+    volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&a_full[i], 1);
+            tc::mbar_init(&a_empty[i], 1);
+            tc::mbar_init(&acc_full[i], 1);
+            tc::mbar_init(&acc_empty[i], 4 * 32);   // one epilogue group
+        }
+        for (int i = 0; i < STAGES; ++i) {
+            tc::mbar_init(&b_full[i], 1);
+            tc::mbar_init(&b_empty[i], 1);
+        }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(tmem_slot, 512);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0, bphase = 0, abuf = 0, aphase = 0;
+            for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+                const Item it = decode_item(a, i);
+                if (!it.valid) continue;
+                if (!tc::mbar_wait(&a_empty[abuf], aphase ^ 1, a.err, abort_flag)) break;
+                tc::mbar_expect_tx(&a_full[abuf], kABytes);
+                const int row0 = it.b * a.T * a.G + it.mt * kM;
+                for (int at = 0; at < kAtoms; ++at)
+                    tc::tma_load_2d(sA + abuf * kABytes + at * kM * 128, &tm_q, &a_full[abuf],
+                                    at * 64, row0);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+                for (int kt = it.kt0; kt < it.kt1; ++kt) {
+                    if (!tc::mbar_wait(&b_empty[stage], bphase ^ 1, a.err, abort_flag)) break;
+                    tc::mbar_expect_tx(&b_full[stage], kBBytes);
+                    const int key0 = it.b * a.S + kt * kN;
+                    for (int at = 0; at < kAtoms; ++at)
+                        tc::tma_load_2d(sB + stage * kBBytes + at * kN * 128, &tm_k,
+                                        &b_full[stage], at * 64, key0);
+                    if (++stage == STAGES) { stage = 0; bphase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::idesc_bf16(kM, kN, 0, 0);
+            int stage = 0, bphase = 0, abuf = 0, aphase = 0, acc = 0, accphase = 0;
+            for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+                const Item it = decode_item(a, i);
+                if (!it.valid) continue;
+                if (!tc::mbar_wait(&a_full[abuf], aphase, a.err, abort_flag)) break;
+                const uint32_t a_base = tc::smem_u32(sA + abuf * kABytes);
+                for (int kt = it.kt0; kt < it.kt1; ++kt) {
+                    if (!tc::mbar_wait(&acc_empty[acc], accphase ^ 1, a.err, abort_flag)) break;
+                    if (!tc::mbar_wait(&b_full[stage], bphase, a.err, abort_flag)) break;
+                    tc::tc_fence_after();
+                    const uint32_t b_base = tc::smem_u32(sB + stage * kBBytes);
+#pragma unroll
+                    for (int ks = 0; ks < DIDX / 16; ++ks) {
+                        const uint32_t off_a = (ks / 4) * kM * 128 + (ks % 4) * 32;
+                        const uint32_t off_b = (ks / 4) * kN * 128 + (ks % 4) * 32;
+                        tc::mma_ss(tmem + acc * kN, tc::sdesc_sw128(a_base + off_a, 16, 1024),
+                                   tc::sdesc_sw128(b_base + off_b, 16, 1024), idesc, ks > 0);
+                    }
+                    tc::mma_commit(&b_empty[stage]);
+                    tc::mma_commit(&acc_full[acc]);
+                    if (++stage == STAGES) { stage = 0; bphase ^= 1; }
+                    if (++acc == 2) { acc = 0; accphase ^= 1; }
+                }
+                tc::mma_commit(&a_empty[abuf]);
+                if (++abuf == 2) { abuf = 0; aphase ^= 1; }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue
+        // Two groups of four warps; group `grp` drains accumulator buffer
+        // `grp`, i.e. every other key tile, so each group has two MMA
+        // periods per tile.  Warp w reads TMEM lanes 32*(w%4) .. +31.
+        const int grp = (warp - 2) / 4;
+        const int quad = warp % 4;
+        const int row_in_tile = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int nbpt = kN / a.block;                    // blocks per key tile (2 or 4)
+        const int cpb = a.block / 64;                     // 64-column chunks per block
+        int acc = 0, accphase = 0;
+        for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+            const Item it = decode_item(a, i);
+            if (!it.valid) continue;
+            const int r = it.mt * kM + row_in_tile;       // row within batch entry b
+            const bool row_ok = r < a.T * a.G;
+            const int t = r / a.G;
+            const int64_t p = (int64_t)a.S - a.T + t;
+            float *out = a.bs + ((int64_t)it.b * a.T * a.G + r) * a.NB;
+            for (int kt = it.kt0; kt < it.kt1; ++kt) {
+                const int my_acc = acc, my_phase = accphase;
+                if (++acc == 2) { acc = 0; accphase ^= 1; }
+                if (my_acc != grp) continue;
+                if (!tc::mbar_wait(&acc_full[my_acc], my_phase, a.err, abort_flag)) break;
+                tc::tc_fence_after();
+                const uint32_t tbase = tmem + my_acc * kN + lane_off;
+                float chunk_max[4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {                 // two halves of 128 columns
+                    uint32_t v[4][32];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) tc::tmem_ld32(tbase + h * 128 + u * 32, v[u]);
+                    tc::tmem_ld_wait();
+                    const int64_t j0 = (int64_t)kt * kN + h * 128;
+                    if (j0 + 127 <= p) {                      // no causal mask needed
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {         // 64-column chunks
+                            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+                            for (int q = 0; q < 32; q += 2) {
+                                m0 = fmaxf(m0, __uint_as_float(v[2 * c][q]));
+                                m1 = fmaxf(m1, __uint_as_float(v[2 * c][q + 1]));
+                                m2 = fmaxf(m2, __uint_as_float(v[2 * c + 1][q]));
+                                m3 = fmaxf(m3, __uint_as_float(v[2 * c + 1][q + 1]));
+                            }
+                            chunk_max[2 * h + c] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) {
+                                const int64_t j = j0 + c * 64 + q;
+                                if (j <= p) m0 = fmaxf(m0, __uint_as_float(v[2 * c][q]));
+                                if (j + 32 <= p) m1 = fmaxf(m1, __uint_as_float(v[2 * c + 1][q]));
+                            }
+                            chunk_max[2 * h + c] = fmaxf(m0, m1);
+                        }
+                    }
+                }
+                tc::tc_fence_before();
+                tc::mbar_arrive(&acc_empty[my_acc]);
+                if (row_ok) {
+                    const int n0 = kt * nbpt;
+                    if (cpb == 2) {
+                        *(float2 *)(out + n0) = make_float2(fmaxf(chunk_max[0], chunk_max[1]),
+                                                            fmaxf(chunk_max[2], chunk_max[3]));
+                    } else {
+                        *(float4 *)(out + n0) = make_float4(chunk_max[0], chunk_max[1],
+                                                            chunk_max[2], chunk_max[3]);
+                    }
+                }
+            }
+            if (a.fill_noncausal && row_ok && it.kt1 == it.nkt && grp == 0) {
+                for (int n = it.nkt * nbpt; n < a.NB; ++n) out[n] = -INFINITY;
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_free(tmem, 512);
+    }
+}
+
+template <int DIDX, int STAGES>
+cudaError_t launch_tc(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
+                      bool fill_noncausal, uint32_t *err, cudaStream_t st) {
+    CUtensorMap tq, tk;
+    const uint64_t qd[2] = {(uint64_t)s.d_idx, (uint64_t)s.B * s.T * s.G};
+    const uint64_t qs[1] = {(uint64_t)s.d_idx * 2};
+    const uint32_t qb[2] = {64, kM};
+    const uint64_t kd[2] = {(uint64_t)s.d_idx, (uint64_t)s.B * s.S};
+    const uint32_t kb[2] = {64, kN};
+    if (!make_tmap_bf16(&tq, q_idx, 2, qd, qs, qb)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tk, k_idx, 2, kd, qs, kb)) return cudaErrorInvalidValue;
+    IndexArgs a{};
+    a.bs = bs; a.err = err;
+    a.B = s.B; a.T = s.T; a.S = s.S; a.G = s.G; a.NB = s.NB; a.block = s.block; a.d_idx = s.d_idx;
+    a.MT = (s.T * s.G + kM - 1) / kM;
+    const int nkt_max = (s.S - 1) / kN + 1;
+    a.CPT = (nkt_max + kKtChunk - 1) / kKtChunk;
+    a.items = s.B * a.MT * a.CPT;
+    a.fill_noncausal = fill_noncausal ? 1 : 0;
+    const size_t smem = 1024 + 2 * (size_t)kM * DIDX * 2 + (size_t)STAGES * kN * DIDX * 2 + 256;
+    auto k = index_tc_kernel<DIDX, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = a.items < sms ? a.items : sms;
+    k<<<grid, kThreads, smem, st>>>(tq, tk, a);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool index_tc_supported(const Shape &s) {
+    return s.dtype == MSA_BF16 && (s.d_idx == 64 || s.d_idx == 128) && s.T * s.G >= kM &&
+           (s.block == 64 || s.block == 128);
+}
+
+cudaError_t launch_index_scores_tc(const Shape &s, const void *q_idx, const void *k_idx,
+                                   float *bs, bool fill_noncausal, uint32_t *err,
+                                   cudaStream_t st) {
+    if (s.d_idx == 64) return launch_tc<64, 4>(s, q_idx, k_idx, bs, fill_noncausal, err, st);
+    return launch_tc<128, 2>(s, q_idx, k_idx, bs, fill_noncausal, err, st);
+}
+
+}  // namespace msa

@@ -49,11 +49,24 @@ msa_status_t make_shape(const msa_params_t *p, Shape *s) {
 size_t block_score_bytes(const Shape &s) { return sizeof(float) * (size_t)s.index_rows() * s.NB; }
 size_t block_id_bytes(const Shape &s) { return sizeof(int32_t) * (size_t)s.index_rows() * s.topk; }
 
+// Prefill shapes go to the tensor-core KV-block-outer kernel; decode-like
+// shapes (few query tokens per sequence) to the query-outer kernel.
+bool use_attn_tc(const Shape &s) { return attn_tc_supported(s) && s.T >= 64; }
+size_t attn_scratch(const Shape &s) { return use_attn_tc(s) ? align_up(attn_tc_workspace(s)) : 0; }
+
 // Workspace layout: [error word 256 B][attention scratch]
-size_t attn_ws(const Shape &) { return kErrorBytes; }
-// msa_forward: [error word][block scores][block ids][attention scratch]
+size_t attn_ws(const Shape &s) { return kErrorBytes + attn_scratch(s); }
+// msa_forward: [error word][attention scratch][block scores][block ids]
 size_t forward_ws(const Shape &s) {
-    return kErrorBytes + align_up(block_score_bytes(s)) + align_up(block_id_bytes(s));
+    return kErrorBytes + attn_scratch(s) + align_up(block_score_bytes(s)) +
+           align_up(block_id_bytes(s));
+}
+
+cudaError_t launch_attention(const Shape &s, const void *Q, const void *K, const void *V,
+                             const int32_t *ids, void *O, float *lse, uint32_t *err,
+                             char *scratch, cudaStream_t st) {
+    if (use_attn_tc(s)) return launch_attn_tc(s, Q, K, V, ids, O, lse, err, scratch, st);
+    return launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
 }
 
 msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
@@ -93,7 +106,10 @@ msa_status_t msa_index_block_scores(const msa_params_t *params, const void *q_id
     if (rc != MSA_OK) return rc;
     if (!q_idx || !k_idx || !block_scores) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(block_scores)) return MSA_ERR_INVALID_ARG;
-    return cuda_status(launch_index_scores_simt(s, q_idx, k_idx, block_scores, (cudaStream_t)stream));
+    cudaStream_t st = (cudaStream_t)stream;
+    if (index_tc_supported(s))
+        return cuda_status(launch_index_scores_tc(s, q_idx, k_idx, block_scores, true, nullptr, st));
+    return cuda_status(launch_index_scores_simt(s, q_idx, k_idx, block_scores, st));
 }
 
 msa_status_t msa_topk_blocks(const msa_params_t *params, const float *block_scores,
@@ -121,7 +137,8 @@ msa_status_t msa_sparse_attn_fwd(const msa_params_t *params, const void *Q, cons
     cudaStream_t st = (cudaStream_t)stream;
     uint32_t *err = (uint32_t *)workspace;
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
-    if (e == cudaSuccess) e = launch_attn_simt(s, Q, K, V, block_ids, O, lse, err, st);
+    if (e == cudaSuccess)
+        e = launch_attention(s, Q, K, V, block_ids, O, lse, err, (char *)workspace + kErrorBytes, st);
     return cuda_status(e);
 }
 
@@ -142,13 +159,16 @@ msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const vo
     cudaStream_t st = (cudaStream_t)stream;
     char *ws = (char *)workspace;
     uint32_t *err = (uint32_t *)ws;
-    float *bs = (float *)(ws + kErrorBytes);
+    char *scratch = ws + kErrorBytes;
+    float *bs = (float *)(scratch + attn_scratch(s));
     int32_t *ids = block_ids ? block_ids
-                             : (int32_t *)(ws + kErrorBytes + align_up(block_score_bytes(s)));
+                             : (int32_t *)((char *)bs + align_up(block_score_bytes(s)));
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
-    if (e == cudaSuccess) e = launch_index_scores_simt(s, q_idx, k_idx, bs, st);
+    if (e == cudaSuccess)
+        e = index_tc_supported(s) ? launch_index_scores_tc(s, q_idx, k_idx, bs, false, err, st)
+                                  : launch_index_scores_simt(s, q_idx, k_idx, bs, st);
     if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
-    if (e == cudaSuccess) e = launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
+    if (e == cudaSuccess) e = launch_attention(s, Q, K, V, ids, O, lse, err, scratch, st);
     return cuda_status(e);
 }
 

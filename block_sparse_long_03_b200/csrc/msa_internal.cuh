@@ -48,6 +48,17 @@ void count_launches(int n);
 // Launchers (each returns a cudaError_t from the launch).
 cudaError_t launch_index_scores_simt(const Shape &s, const void *q_idx, const void *k_idx,
                                      float *bs, cudaStream_t st);
+// Tensor-core index scoring (bf16, d_idx in {64, 128}, at least 128 index rows).
+bool index_tc_supported(const Shape &s);
+cudaError_t launch_index_scores_tc(const Shape &s, const void *q_idx, const void *k_idx,
+                                   float *bs, bool fill_noncausal, uint32_t *err,
+                                   cudaStream_t st);
+// Tensor-core KV-block-outer sparse attention (bf16, d = 128) and its workspace.
+bool attn_tc_supported(const Shape &s);
+size_t attn_tc_workspace(const Shape &s);
+cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
+                           const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
+                           cudaStream_t st);
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st);
 cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
