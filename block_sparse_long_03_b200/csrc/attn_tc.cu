@@ -36,16 +36,31 @@ constexpr int kThreads = 320;        // warp 0 load, warp 1 MMA, warps 2-9 softm
 constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
 constexpr float kLog2e = 1.4426950408889634f;
 
+// True when the row's non-negative ids are strictly ascending (the form
+// msa_topk_blocks writes), so no id can repeat.
+__device__ __forceinline__ bool row_ascending(const int32_t *row, int topk) {
+    int prev = -1;
+    for (int i = 0; i < topk; ++i) {
+        const int n = row[i];
+        if (n < 0) continue;
+        if (n <= prev) return false;
+        prev = n;
+    }
+    return true;
+}
+
 // Validity of slot `i` of a kept-id row, shared by every phase: in range, not
 // a repeat of an earlier slot, and holding at least one causal token.
+// `ascending` (from row_ascending) skips the repeat scan.
 __device__ __forceinline__ bool slot_valid(const int32_t *row, int i, int NB, int cb,
-                                           bool *bad) {
+                                           bool ascending, bool *bad) {
     const int n = row[i];
     *bad = false;
     if (n < 0) return false;
     if (n >= NB) { *bad = true; return false; }
-    for (int k = 0; k < i; ++k)
-        if (row[k] == n) { *bad = true; return false; }
+    if (!ascending)
+        for (int k = 0; k < i; ++k)
+            if (row[k] == n) { *bad = true; return false; }
     return n <= cb;
 }
 
@@ -62,9 +77,10 @@ __global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restric
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
     const int32_t *row = ids + (r * G + g) * topk;
+    const bool asc = row_ascending(row, topk);
     for (int i = 0; i < topk; ++i) {
         bool bad;
-        if (slot_valid(row, i, NB, cb, &bad))
+        if (slot_valid(row, i, NB, cb, asc, &bad))
             atomicAdd(&counts[((int64_t)b * G + g) * NB + row[i]], 1);
         else if (bad)
             record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
@@ -113,9 +129,10 @@ __global__ void csr_fill_kernel(const int32_t *__restrict__ ids, const int *__re
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
     const int32_t *row = ids + (r * G + g) * topk;
+    const bool asc = row_ascending(row, topk);
     for (int i = 0; i < topk; ++i) {
         bool bad;
-        if (!slot_valid(row, i, NB, cb, &bad)) continue;
+        if (!slot_valid(row, i, NB, cb, asc, &bad)) continue;
         const int64_t list = ((int64_t)b * G + g) * NB + row[i];
         const int pos = atomicAdd(&cursor[list], 1);
         entries[offs[list] + pos] = (int)(((r - r0) << 8) | i);
@@ -209,7 +226,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------ loads: K/V blocks and Q rows by TMA
         // The next tile's descriptor and entries are fetched one tile ahead.
-        int kvb = -1, cur_list = -1, kv_ph[2] = {0, 0}, q_ph[2] = {0, 0};
+        int kvb = -1, cur_list = -1;
+        uint32_t kv_ph = 0, q_ph = 0;              // per-buffer phase bits
         int4 nd = load_tile(a, 0, total);
         int ne[4];
 #pragma unroll
@@ -234,7 +252,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (list != cur_list) {
                 kvb = (kvb + 1) & 1;
                 cur_list = list;
-                if (lane == 0 && tc::mbar_wait(&kv_empty[kvb], kv_ph[kvb] ^ 1, a.err, abort_flag)) {
+                if (lane == 0 &&
+                    tc::mbar_wait(&kv_empty[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag)) {
                     tc::mbar_expect_tx(&kv_full[kvb], 2 * kKBytes);
                     const int key0 = b * a.S + n * BLOCK;
 #pragma unroll
@@ -245,11 +264,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                         &kv_full[kvb], at * 64, g, key0);
                     }
                 }
-                kv_ph[kvb] ^= 1;
+                kv_ph ^= 1u << kvb;
             }
             const int qb = i & 1;
-            if (!tc::mbar_wait(&q_empty[qb], q_ph[qb] ^ 1, a.err, abort_flag)) break;
-            q_ph[qb] ^= 1;
+            if (!tc::mbar_wait(&q_empty[qb], ((q_ph >> qb) & 1) ^ 1, a.err, abort_flag)) break;
+            q_ph ^= 1u << qb;
             uint8_t *dst = sQ + qb * kQBytes;
             if (a.R >= 8) {
                 // One TMA box per token: its R heads x 64 channels, R * 128 bytes, so
@@ -296,8 +315,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
-            int kvb = -1, cur_list = -1, kv_ph[2] = {0, 0}, q_ph[2] = {0, 0};
-            int acc_ph[2] = {0, 0}, p_ph[2] = {0, 0};
+            int kvb = -1, cur_list = -1;
+            uint32_t kv_ph = 0, q_ph = 0, acc_ph = 0, p_ph = 0;   // per-buffer phase bits
             int prev_acc = -1, prev_kvb = -1, prev_list = -1;
             int next_list = load_tile(a, 0, total).x;
             for (int i = 0;; ++i) {
@@ -308,14 +327,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (list != cur_list) {
                         kvb = (kvb + 1) & 1;
                         cur_list = list;
-                        kv_ph[kvb] ^= 1;
+                        kv_ph ^= 1u << kvb;
                     }
                     const int acc = i & 1, qb = i & 1;
-                    if (!tc::mbar_wait(&acc_empty[acc], acc_ph[acc] ^ 1, a.err, abort_flag)) break;
-                    acc_ph[acc] ^= 1;
-                    if (!tc::mbar_wait(&q_full[qb], q_ph[qb], a.err, abort_flag)) break;
-                    q_ph[qb] ^= 1;
-                    if (!tc::mbar_wait(&kv_full[kvb], kv_ph[kvb] ^ 1, a.err, abort_flag)) break;
+                    if (!tc::mbar_wait(&acc_empty[acc], ((acc_ph >> acc) & 1) ^ 1, a.err, abort_flag))
+                        break;
+                    acc_ph ^= 1u << acc;
+                    if (!tc::mbar_wait(&q_full[qb], (q_ph >> qb) & 1, a.err, abort_flag)) break;
+                    q_ph ^= 1u << qb;
+                    if (!tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
+                        break;
                     tc::tc_fence_after();
                     const uint32_t qa = tc::smem_u32(sQ + qb * kQBytes);
                     const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
@@ -332,8 +353,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 if (prev_acc >= 0) {
                     // O = P V for the previous tile (P from TMEM, V from shared memory)
-                    if (!tc::mbar_wait(&p_full[prev_acc], p_ph[prev_acc], a.err, abort_flag)) break;
-                    p_ph[prev_acc] ^= 1;
+                    if (!tc::mbar_wait(&p_full[prev_acc], (p_ph >> prev_acc) & 1, a.err, abort_flag))
+                        break;
+                    p_ph ^= 1u << prev_acc;
                     tc::tc_fence_after();
                     const uint32_t va = tc::smem_u32(sV + prev_kvb * kKBytes);
 #pragma unroll
@@ -377,77 +399,99 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int64_t j_base = (int64_t)n * BLOCK;
             if (!tc::mbar_wait(&s_full[grp], ph, a.err, abort_flag)) break;
             tc::tc_fence_after();
-            uint32_t sreg[BLOCK];
-#pragma unroll
-            for (int c = 0; c < BLOCK; c += 32) tc::tmem_ld32(tS + c, *(uint32_t(*)[32])(sreg + c));
-            tc::tmem_ld_wait();
+            // Pass 1: row maximum, 64 columns at a time (keeps register use low).
             const bool masked = valid && (j_base + BLOCK - 1 > p);
-            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-            if (!masked) {
+            float m = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < BLOCK; c += 4) {
-                    m0 = fmaxf(m0, __uint_as_float(sreg[c]));
-                    m1 = fmaxf(m1, __uint_as_float(sreg[c + 1]));
-                    m2 = fmaxf(m2, __uint_as_float(sreg[c + 2]));
-                    m3 = fmaxf(m3, __uint_as_float(sreg[c + 3]));
+            for (int c0 = 0; c0 < BLOCK; c0 += 64) {
+                uint32_t v[64];
+                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v));
+                tc::tmem_ld32(tS + c0 + 32, *(uint32_t(*)[32])(v + 32));
+                tc::tmem_ld_wait();
+                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                if (!masked) {
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        m0 = fmaxf(m0, __uint_as_float(v[c]));
+                        m1 = fmaxf(m1, __uint_as_float(v[c + 1]));
+                        m2 = fmaxf(m2, __uint_as_float(v[c + 2]));
+                        m3 = fmaxf(m3, __uint_as_float(v[c + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (j_base + c0 + c <= p) m0 = fmaxf(m0, __uint_as_float(v[c]));
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BLOCK; ++c)
-                    if (j_base + c <= p) m0 = fmaxf(m0, __uint_as_float(sreg[c]));
+                m = fmaxf(m, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
             }
-            float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
             if (!valid) m = 0.f;
             const float mb = m * a.scale_log2;
+            // Pass 2: P = 2^((s - m) * scale * log2 e) as bf16 pairs into the S
+            // columns already consumed (P of 64 keys occupies 32 columns).
             float l0 = 0.f, l1 = 0.f;
-            uint32_t preg[BLOCK / 2];
 #pragma unroll
-            for (int c = 0; c < BLOCK; c += 2) {
-                float p0 = exp2f(fmaf(__uint_as_float(sreg[c]), a.scale_log2, -mb));
-                float p1 = exp2f(fmaf(__uint_as_float(sreg[c + 1]), a.scale_log2, -mb));
-                if (!valid || (masked && j_base + c > p)) p0 = 0.f;
-                if (!valid || (masked && j_base + c + 1 > p)) p1 = 0.f;
-                l0 += p0;
-                l1 += p1;
-                __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-                preg[c / 2] = *(uint32_t *)&pk;
+            for (int c0 = 0; c0 < BLOCK; c0 += 64) {
+                uint32_t v[64];
+                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v));
+                tc::tmem_ld32(tS + c0 + 32, *(uint32_t(*)[32])(v + 32));
+                tc::tmem_ld_wait();
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    float p0 = tc::ex2_approx(fmaf(__uint_as_float(v[c]), a.scale_log2, -mb));
+                    float p1 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb));
+                    if (masked) {
+                        if (j_base + c0 + c > p) p0 = 0.f;
+                        if (j_base + c0 + c + 1 > p) p1 = 0.f;
+                    }
+                    if (!valid) { p0 = 0.f; p1 = 0.f; }
+                    l0 += p0;
+                    l1 += p1;
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+                    pk[c / 2] = *(uint32_t *)&b2;
+                }
+                tc::tmem_st32(tS + c0 / 2, pk);
             }
             const float l = l0 + l1;
-#pragma unroll
-            for (int c = 0; c < BLOCK / 2; c += 32)
-                tc::tmem_st32(tS + c, *(const uint32_t(*)[32])(preg + c));
             tc::tmem_st_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(&p_full[grp]);
             if (!tc::mbar_wait(&o_full[grp], ph, a.err, abort_flag)) break;
             tc::tc_fence_after();
-            uint32_t oreg[D];
+            const int slot = ent & 255;
+            const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
+            const float inv_l = valid ? 1.f / l : 0.f;
+            uint4 *dst = (uint4 *)(a.part_o + prow * D);
 #pragma unroll
-            for (int c = 0; c < D; c += 32) tc::tmem_ld32(tO + c, *(uint32_t(*)[32])(oreg + c));
-            tc::tmem_ld_wait();
-            tc::tc_fence_before();
-            tc::mbar_arrive(&acc_empty[grp]);
+            for (int c0 = 0; c0 < D; c0 += 64) {
+                uint32_t v[64];
+                tc::tmem_ld32(tO + c0, *(uint32_t(*)[32])(v));
+                tc::tmem_ld32(tO + c0 + 32, *(uint32_t(*)[32])(v + 32));
+                tc::tmem_ld_wait();
+                if (c0 + 64 >= D) {                    // last columns read: release TMEM
+                    tc::tc_fence_before();
+                    tc::mbar_arrive(&acc_empty[grp]);
+                }
+                if (valid) {
+#pragma unroll
+                    for (int c = 0; c < 64; c += 8) {
+                        __half2 h0 = __floats2half2_rn(__uint_as_float(v[c]) * inv_l,
+                                                       __uint_as_float(v[c + 1]) * inv_l);
+                        __half2 h1 = __floats2half2_rn(__uint_as_float(v[c + 2]) * inv_l,
+                                                       __uint_as_float(v[c + 3]) * inv_l);
+                        __half2 h2 = __floats2half2_rn(__uint_as_float(v[c + 4]) * inv_l,
+                                                       __uint_as_float(v[c + 5]) * inv_l);
+                        __half2 h3 = __floats2half2_rn(__uint_as_float(v[c + 6]) * inv_l,
+                                                       __uint_as_float(v[c + 7]) * inv_l);
+                        uint4 u;
+                        u.x = *(uint32_t *)&h0; u.y = *(uint32_t *)&h1;
+                        u.z = *(uint32_t *)&h2; u.w = *(uint32_t *)&h3;
+                        dst[(c0 + c) / 8] = u;
+                    }
+                }
+            }
             ph ^= 1;
             if (valid) {
-                const int slot = ent & 255;
-                const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
-                const float inv_l = 1.f / l;
-                uint4 *dst = (uint4 *)(a.part_o + prow * D);
-#pragma unroll
-                for (int c = 0; c < D; c += 8) {
-                    __half2 h0 = __floats2half2_rn(__uint_as_float(oreg[c]) * inv_l,
-                                                   __uint_as_float(oreg[c + 1]) * inv_l);
-                    __half2 h1 = __floats2half2_rn(__uint_as_float(oreg[c + 2]) * inv_l,
-                                                   __uint_as_float(oreg[c + 3]) * inv_l);
-                    __half2 h2 = __floats2half2_rn(__uint_as_float(oreg[c + 4]) * inv_l,
-                                                   __uint_as_float(oreg[c + 5]) * inv_l);
-                    __half2 h3 = __floats2half2_rn(__uint_as_float(oreg[c + 6]) * inv_l,
-                                                   __uint_as_float(oreg[c + 7]) * inv_l);
-                    uint4 u;
-                    u.x = *(uint32_t *)&h0; u.y = *(uint32_t *)&h1;
-                    u.z = *(uint32_t *)&h2; u.w = *(uint32_t *)&h3;
-                    dst[c / 8] = u;
-                }
                 a.part_lse[prow] = m * a.scale + logf(l);
             }
         }
@@ -485,13 +529,14 @@ __global__ void combine_kernel(const int32_t *__restrict__ ids, const __half *__
     const int t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
     const int32_t *row = ids + (r * G + g) * topk;
+    const bool asc = row_ascending(row, topk);
     float m = -INFINITY, l = 0.f, acc[kPer];
 #pragma unroll
     for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
     for (int base = 0; base < topk; base += 32) {
         bool bad;
         const int i = base + lane;
-        const bool ok = i < topk && slot_valid(row, i, NB, cb, &bad);
+        const bool ok = i < topk && slot_valid(row, i, NB, cb, asc, &bad);
         unsigned mask = __ballot_sync(0xffffffffu, ok);
         while (mask) {
             const int s = base + __ffs(mask) - 1;
@@ -623,6 +668,17 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 }
 
 }  // namespace
+
+cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
+                           const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
+                           cudaStream_t st) {
+    const int64_t warps = rc * s.Hq;
+    combine_kernel<128><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+        ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
+        s.block, s.topk);
+    count_launches(1);
+    return cudaGetLastError();
+}
 
 bool attn_tc_supported(const Shape &s) {
     return s.dtype == MSA_BF16 && s.d == 128 && (s.block == 128 || s.block == 64) &&

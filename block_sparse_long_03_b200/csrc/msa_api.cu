@@ -52,7 +52,20 @@ size_t block_id_bytes(const Shape &s) { return sizeof(int32_t) * (size_t)s.index
 // Prefill shapes go to the tensor-core KV-block-outer kernel; decode-like
 // shapes (few query tokens per sequence) to the query-outer kernel.
 bool use_attn_tc(const Shape &s) { return attn_tc_supported(s) && s.T >= 64; }
-size_t attn_scratch(const Shape &s) { return use_attn_tc(s) ? align_up(attn_tc_workspace(s)) : 0; }
+bool use_attn_decode(const Shape &s) { return !use_attn_tc(s) && decode_attn_supported(s); }
+size_t attn_scratch(const Shape &s) {
+    if (use_attn_tc(s)) return align_up(attn_tc_workspace(s));
+    if (use_attn_decode(s)) return align_up(decode_attn_workspace(s));
+    return 0;
+}
+
+cudaError_t launch_index(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
+                         bool fill_noncausal, uint32_t *err, cudaStream_t st) {
+    if (index_tc_supported(s))
+        return launch_index_scores_tc(s, q_idx, k_idx, bs, fill_noncausal, err, st);
+    if (decode_index_supported(s)) return launch_decode_index(s, q_idx, k_idx, bs, st);
+    return launch_index_scores_simt(s, q_idx, k_idx, bs, st);
+}
 
 // Workspace layout: [error word 256 B][attention scratch]
 size_t attn_ws(const Shape &s) { return kErrorBytes + attn_scratch(s); }
@@ -66,6 +79,7 @@ cudaError_t launch_attention(const Shape &s, const void *Q, const void *K, const
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
                              char *scratch, cudaStream_t st) {
     if (use_attn_tc(s)) return launch_attn_tc(s, Q, K, V, ids, O, lse, err, scratch, st);
+    if (use_attn_decode(s)) return launch_decode_attn(s, Q, K, V, ids, O, lse, err, scratch, st);
     return launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
 }
 
@@ -107,9 +121,7 @@ msa_status_t msa_index_block_scores(const msa_params_t *params, const void *q_id
     if (!q_idx || !k_idx || !block_scores) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(block_scores)) return MSA_ERR_INVALID_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    if (index_tc_supported(s))
-        return cuda_status(launch_index_scores_tc(s, q_idx, k_idx, block_scores, true, nullptr, st));
-    return cuda_status(launch_index_scores_simt(s, q_idx, k_idx, block_scores, st));
+    return cuda_status(launch_index(s, q_idx, k_idx, block_scores, true, nullptr, st));
 }
 
 msa_status_t msa_topk_blocks(const msa_params_t *params, const float *block_scores,
@@ -164,9 +176,7 @@ msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const vo
     int32_t *ids = block_ids ? block_ids
                              : (int32_t *)((char *)bs + align_up(block_score_bytes(s)));
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
-    if (e == cudaSuccess)
-        e = index_tc_supported(s) ? launch_index_scores_tc(s, q_idx, k_idx, bs, false, err, st)
-                                  : launch_index_scores_simt(s, q_idx, k_idx, bs, st);
+    if (e == cudaSuccess) e = launch_index(s, q_idx, k_idx, bs, false, err, st);
     if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
     if (e == cudaSuccess) e = launch_attention(s, Q, K, V, ids, O, lse, err, scratch, st);
     return cuda_status(e);

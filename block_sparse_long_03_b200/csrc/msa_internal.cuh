@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -59,6 +60,21 @@ size_t attn_tc_workspace(const Shape &s);
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st);
+// LSE-weighted combine of per-(row, head, kept slot) partials into O and lse
+// for query rows [r0, r0 + rc) (d = 128).
+cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
+                           const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
+                           cudaStream_t st);
+// Decode path (few query tokens per sequence): HBM-streaming index scoring and
+// one-CTA-per-kept-block attention feeding the same combine.
+bool decode_index_supported(const Shape &s);
+cudaError_t launch_decode_index(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
+                                cudaStream_t st);
+bool decode_attn_supported(const Shape &s);
+size_t decode_attn_workspace(const Shape &s);
+cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
+                               const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
+                               cudaStream_t st);
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st);
 cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
