@@ -32,7 +32,7 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;           // tile rows = tokens_per_tile * R
-constexpr int kThreads = 320;        // warp 0 load, warp 1 MMA, warps 2-9 softmax/epilogue
+constexpr int kThreads = 320;        // warp 0 loads, warp 1 MMA, warps 2-9 softmax/epilogue
 constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -164,8 +164,9 @@ struct AttnArgs {
     const int *entries;         // CSR entries: (row - r0) << 8 | slot
     const int4 *tiles;          // {list, count, first entry, 0} per tile
     const int *n_tiles;         // device-side tile count
-    __half *part_o;             // [rc * G * topk * R, D] normalised partial outputs
-    float *part_lse;            // [rc * G * topk * R]
+    __half *part_o;             // normalised partial O, blocked chunks (partial_chunk)
+    float *part_lse;            // [n_prows]
+    int64_t n_prows;            // rc * G * topk * R
     uint32_t *err;
     int64_t r0;
     int T, S, Hq, G, R, NB, topk, tpt;
@@ -399,60 +400,65 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int64_t j_base = (int64_t)n * BLOCK;
             if (!tc::mbar_wait(&s_full[grp], ph, a.err, abort_flag)) break;
             tc::tc_fence_after();
-            // Pass 1: row maximum, 64 columns at a time (keeps register use low).
+            // Row maximum over the causal keys of the block (one TMEM read).
             const bool masked = valid && (j_base + BLOCK - 1 > p);
-            float m = -INFINITY;
+            uint32_t v[BLOCK];
 #pragma unroll
-            for (int c0 = 0; c0 < BLOCK; c0 += 64) {
-                uint32_t v[64];
-                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v));
-                tc::tmem_ld32(tS + c0 + 32, *(uint32_t(*)[32])(v + 32));
-                tc::tmem_ld_wait();
-                float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-                if (!masked) {
+            for (int c0 = 0; c0 < BLOCK; c0 += 32)
+                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v + c0));
+            tc::tmem_ld_wait();
+            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+            if (!masked) {
 #pragma unroll
-                    for (int c = 0; c < 64; c += 4) {
-                        m0 = fmaxf(m0, __uint_as_float(v[c]));
-                        m1 = fmaxf(m1, __uint_as_float(v[c + 1]));
-                        m2 = fmaxf(m2, __uint_as_float(v[c + 2]));
-                        m3 = fmaxf(m3, __uint_as_float(v[c + 3]));
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (j_base + c0 + c <= p) m0 = fmaxf(m0, __uint_as_float(v[c]));
+                for (int c = 0; c < BLOCK; c += 4) {
+                    m0 = fmaxf(m0, __uint_as_float(v[c]));
+                    m1 = fmaxf(m1, __uint_as_float(v[c + 1]));
+                    m2 = fmaxf(m2, __uint_as_float(v[c + 2]));
+                    m3 = fmaxf(m3, __uint_as_float(v[c + 3]));
                 }
-                m = fmaxf(m, fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)));
+            } else {
+#pragma unroll
+                for (int c = 0; c < BLOCK; ++c)
+                    if (j_base + c <= p) m0 = fmaxf(m0, __uint_as_float(v[c]));
             }
+            float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
             if (!valid) m = 0.f;
             const float mb = m * a.scale_log2;
-            // Pass 2: P = 2^((s - m) * scale * log2 e) as bf16 pairs into the S
-            // columns already consumed (P of 64 keys occupies 32 columns).
-            float l0 = 0.f, l1 = 0.f;
+            // P = 2^((s - m) * scale * log2 e) in three sweeps so that the 2^x
+            // instructions are independent: exponents in fp32 packed as half
+            // pairs (the S registers die as they are consumed), 2^x on the
+            // pairs (P is rounded to bf16 for the MMA, so a half-precision 2^x
+            // is exact enough), then the fp32 row sum and the bf16 packing in
+            // place.  P (bf16 pairs) goes to the S columns already read.
+            uint32_t pk[BLOCK / 2];
 #pragma unroll
-            for (int c0 = 0; c0 < BLOCK; c0 += 64) {
-                uint32_t v[64];
-                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v));
-                tc::tmem_ld32(tS + c0 + 32, *(uint32_t(*)[32])(v + 32));
-                tc::tmem_ld_wait();
-                uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    float p0 = tc::ex2_approx(fmaf(__uint_as_float(v[c]), a.scale_log2, -mb));
-                    float p1 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb));
-                    if (masked) {
-                        if (j_base + c0 + c > p) p0 = 0.f;
-                        if (j_base + c0 + c + 1 > p) p1 = 0.f;
-                    }
-                    if (!valid) { p0 = 0.f; p1 = 0.f; }
-                    l0 += p0;
-                    l1 += p1;
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                    pk[c / 2] = *(uint32_t *)&b2;
+            for (int c = 0; c < BLOCK; c += 2) {
+                float x0 = fmaf(__uint_as_float(v[c]), a.scale_log2, -mb);
+                float x1 = fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb);
+                if (masked) {
+                    if (j_base + c > p) x0 = -INFINITY;
+                    if (j_base + c + 1 > p) x1 = -INFINITY;
                 }
-                tc::tmem_st32(tS + c0 / 2, pk);
+                __half2 xh = __floats2half2_rn(x0, x1);
+                pk[c / 2] = *(uint32_t *)&xh;
             }
-            const float l = l0 + l1;
+#pragma unroll
+            for (int c = 0; c < BLOCK / 2; ++c) pk[c] = tc::ex2_approx_h2(pk[c]);
+            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+            for (int c = 0; c < BLOCK / 2; c += 2) {
+                const float2 e0 = __half22float2(*(const __half2 *)&pk[c]);
+                const float2 e1 = __half22float2(*(const __half2 *)&pk[c + 1]);
+                l0 += e0.x; l1 += e0.y; l2 += e1.x; l3 += e1.y;
+                __nv_bfloat162 b0 = __floats2bfloat162_rn(e0.x, e0.y);
+                __nv_bfloat162 b1 = __floats2bfloat162_rn(e1.x, e1.y);
+                pk[c] = *(uint32_t *)&b0;
+                pk[c + 1] = *(uint32_t *)&b1;
+            }
+#pragma unroll
+            for (int c = 0; c < BLOCK / 2; c += 32)
+                tc::tmem_st32(tS + c, *(const uint32_t(*)[32])(pk + c));
+            const float l = (l0 + l1) + (l2 + l3);
             tc::tmem_st_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(&p_full[grp]);
@@ -460,35 +466,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             tc::tc_fence_after();
             const int slot = ent & 255;
             const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
-            const float inv_l = valid ? 1.f / l : 0.f;
-            uint4 *dst = (uint4 *)(a.part_o + prow * D);
+            const float inv_l = 1.f / l;
+            // partial O in 32-row blocked chunk planes (partial_chunk): the rows
+            // of a warp store to consecutive addresses
+            uint4 *dst = (uint4 *)a.part_o + partial_chunk(prow, 0, D);
+            // O row to fp16 pairs in place; TMEM is released as soon as the row
+            // is in registers, before the stores.
+            uint32_t ov[D];
 #pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 64) {
-                uint32_t v[64];
-                tc::tmem_ld32(tO + c0, *(uint32_t(*)[32])(v));
-                tc::tmem_ld32(tO + c0 + 32, *(uint32_t(*)[32])(v + 32));
-                tc::tmem_ld_wait();
-                if (c0 + 64 >= D) {                    // last columns read: release TMEM
-                    tc::tc_fence_before();
-                    tc::mbar_arrive(&acc_empty[grp]);
-                }
-                if (valid) {
+            for (int c0 = 0; c0 < D; c0 += 32) tc::tmem_ld32(tO + c0, *(uint32_t(*)[32])(ov + c0));
+            tc::tmem_ld_wait();
+            tc::tc_fence_before();
+            tc::mbar_arrive(&acc_empty[grp]);               // accumulators free for tile i + 2
 #pragma unroll
-                    for (int c = 0; c < 64; c += 8) {
-                        __half2 h0 = __floats2half2_rn(__uint_as_float(v[c]) * inv_l,
-                                                       __uint_as_float(v[c + 1]) * inv_l);
-                        __half2 h1 = __floats2half2_rn(__uint_as_float(v[c + 2]) * inv_l,
-                                                       __uint_as_float(v[c + 3]) * inv_l);
-                        __half2 h2 = __floats2half2_rn(__uint_as_float(v[c + 4]) * inv_l,
-                                                       __uint_as_float(v[c + 5]) * inv_l);
-                        __half2 h3 = __floats2half2_rn(__uint_as_float(v[c + 6]) * inv_l,
-                                                       __uint_as_float(v[c + 7]) * inv_l);
-                        uint4 u;
-                        u.x = *(uint32_t *)&h0; u.y = *(uint32_t *)&h1;
-                        u.z = *(uint32_t *)&h2; u.w = *(uint32_t *)&h3;
-                        dst[(c0 + c) / 8] = u;
-                    }
-                }
+            for (int c = 0; c < D; c += 2) {
+                __half2 hv = __floats2half2_rn(__uint_as_float(ov[c]) * inv_l,
+                                               __uint_as_float(ov[c + 1]) * inv_l);
+                ov[c / 2] = *(uint32_t *)&hv;
+            }
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < D / 2; c += 4)
+                    dst[(c / 4) * 32] = make_uint4(ov[c], ov[c + 1], ov[c + 2], ov[c + 3]);
             }
             ph ^= 1;
             if (valid) {
@@ -510,63 +509,121 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 namespace msa {
 namespace {
 
-// Phase 2: one warp per (query row, head).  The partials of the row's valid
-// kept slots are merged with weights exp(lse_i - max lse); the result is the
-// softmax over the union of the slots' keys.
-template <int D>
-__global__ void combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_o,
+// Phase 2: the LSE-weighted merge of a (query row, group)'s partials over
+// its valid kept slots, for each of the group's R heads: weights
+// exp(lse_i - max lse) give the softmax over the union of the slots' keys.
+// Four warps share a (row, group), each merging a quarter of the d/8 16-byte
+// channel chunks.  Lane l owns head l % R and slots l / R, l / R + 32 / R, ...;
+// with the blocked chunk layout every load of the warp is 512 contiguous
+// bytes, and all loads of a warp are independent (issued together).
+// Needs R | 32 and topk <= 64.
+template <int D, int kMaxPer>
+__global__ void __launch_bounds__(256, kMaxPer <= 8 ? 4 : 2)
+combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_o,
                                const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
                                float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
                                int Hq, int G, int R, int NB, int block, int topk) {
-    constexpr int kPer = D / 32;                  // output channels per lane
+    constexpr int kChunksPerWarp = 4;             // kMaxPer: slots per lane, >= topk * R / 32
+    constexpr int kWarpsPerRow = D / 8 / kChunksPerWarp;
     const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
-    if (wid >= rc * Hq) return;
-    const int64_t rl = wid / Hq;                  // row within the chunk
-    const int hq = (int)(wid % Hq);
-    const int g = hq / R, h = hq % R;
+    if (wid >= rc * G * kWarpsPerRow) return;
+    const int part = (int)(wid % kWarpsPerRow);
+    const int64_t rgl = wid / kWarpsPerRow;
+    const int64_t rl = rgl / G;                   // row within the chunk
+    const int g = (int)(rgl % G);
     const int64_t r = r0 + rl;
     const int t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
     const int32_t *row = ids + (r * G + g) * topk;
-    const bool asc = row_ascending(row, topk);
-    float m = -INFINITY, l = 0.f, acc[kPer];
+    // the row's ids, slot lane and lane + 32
+    const int id0 = lane < topk ? row[lane] : -1;
+    const int id1 = lane + 32 < topk ? row[lane + 32] : -1;
+    // strictly ascending over the non-negative ids <=> every id exceeds the
+    // running maximum of the ids before it (warp prefix-max scan)
+    int pm0 = id0;
+    for (int off = 1; off < 32; off *= 2) {
+        const int o = __shfl_up_sync(0xffffffffu, pm0, off);
+        if (lane >= off) pm0 = max(pm0, o);
+    }
+    const int before0 = __shfl_up_sync(0xffffffffu, pm0, 1);
+    const int max_first = __shfl_sync(0xffffffffu, pm0, 31);
+    int pm1 = id1;
+    for (int off = 1; off < 32; off *= 2) {
+        const int o = __shfl_up_sync(0xffffffffu, pm1, off);
+        if (lane >= off) pm1 = max(pm1, o);
+    }
+    const int before1 = max(max_first, __shfl_up_sync(0xffffffffu, pm1, 1));
+    const bool bad0 = id0 >= 0 && lane > 0 && id0 <= before0;
+    const bool bad1 = id1 >= 0 && (lane > 0 ? id1 <= before1 : id1 <= max_first);
+    const bool asc = !__any_sync(0xffffffffu, bad0 || bad1);
+    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (topk + sstep - 1) / sstep;
+    const int64_t base = (rl * G + g) * topk * R;
+    float li[kMaxPer], m = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
-    for (int base = 0; base < topk; base += 32) {
-        bool bad;
-        const int i = base + lane;
-        const bool ok = i < topk && slot_valid(row, i, NB, cb, asc, &bad);
-        unsigned mask = __ballot_sync(0xffffffffu, ok);
-        while (mask) {
-            const int s = base + __ffs(mask) - 1;
-            mask &= mask - 1;
-            const int64_t prow = ((rl * G + g) * topk + s) * R + h;
-            const float li = part_lse[prow];
-            const float m_new = fmaxf(m, li);
-            const float a_old = expf(m - m_new), w = expf(li - m_new);
-            const __half *src = part_o + prow * D + lane * kPer;
-            float v[kPer];
-            if (kPer == 4) {
-                const uint2 u = *(const uint2 *)src;
-                const float2 f0 = __half22float2(*(const __half2 *)&u.x);
-                const float2 f1 = __half22float2(*(const __half2 *)&u.y);
-                v[0] = f0.x; v[1] = f0.y; v[2 % kPer] = f1.x; v[3 % kPer] = f1.y;
-            } else {
+    for (int k = 0; k < kMaxPer; ++k) {
+        const int sl = s0 + k * sstep;
+        const int idk = __shfl_sync(0xffffffffu, sl < 32 ? id0 : id1, sl & 31);
+        bool ok = k < per && sl < topk && idk >= 0 && idk < NB && idk <= cb;
+        if (ok && !asc) {                          // rare: caller ids out of order
+            for (int q = 0; q < sl; ++q) ok = ok && row[q] != idk;
+        }
+        li[k] = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+        m = fmaxf(m, li[k]);
+    }
+    for (int off = R; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float w[kMaxPer], lsum = 0.f;
 #pragma unroll
-                for (int c = 0; c < kPer; ++c) v[c] = __half2float(src[c]);
+    for (int k = 0; k < kMaxPer; ++k) {
+        w[k] = li[k] == -INFINITY ? 0.f : expf(li[k] - m);
+        lsum += w[k];
+    }
+    for (int off = R; off < 32; off *= 2) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const uint4 *src = (const uint4 *)part_o;
+    __nv_bfloat16 *dst = O + (r * Hq + (int64_t)g * R + h) * D;
+    float acc[kChunksPerWarp][8];
+#pragma unroll
+    for (int c = 0; c < kChunksPerWarp; ++c)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[c][q] = 0.f;
+    // k < per is uniform across the warp, so the loads are issued together;
+    // a slot that holds no partial (weight 0) has its data replaced by 0
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        if (k < per) {
+            const int64_t prow = base + (int64_t)(s0 + k * sstep) * R + h;
+            const bool use = w[k] > 0.f;
+#pragma unroll
+            for (int c = 0; c < kChunksPerWarp; ++c) {
+                uint4 u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
+                if (!use) u = make_uint4(0u, 0u, 0u, 0u);
+                const __half2 *hp = (const __half2 *)&u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(hp[q]);
+                    acc[c][2 * q] = fmaf(w[k], f.x, acc[c][2 * q]);
+                    acc[c][2 * q + 1] = fmaf(w[k], f.y, acc[c][2 * q + 1]);
+                }
             }
-#pragma unroll
-            for (int c = 0; c < kPer; ++c) acc[c] = acc[c] * a_old + w * v[c];
-            l = l * a_old + w;
-            m = m_new;
         }
     }
-    __nv_bfloat16 *dst = O + (r * Hq + hq) * D + lane * kPer;
-    const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-    for (int c = 0; c < kPer; ++c) dst[c] = __float2bfloat16_rn(acc[c] * inv);
-    if (lane == 0) lse[r * Hq + hq] = l > 0.f ? m + logf(l) : -INFINITY;
+    for (int c = 0; c < kChunksPerWarp; ++c) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            for (int off = R; off < 32; off *= 2)
+                acc[c][q] += __shfl_xor_sync(0xffffffffu, acc[c][q], off);
+        if (s0 == 0) {
+            __nv_bfloat162 o2[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o2[q] = __floats2bfloat162_rn(acc[c][2 * q] * inv, acc[c][2 * q + 1] * inv);
+            *(uint4 *)(dst + (part * kChunksPerWarp + c) * 8) = *(const uint4 *)o2;
+        }
+    }
+    if (part == 0 && s0 == 0) lse[r * Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
 }
 
 constexpr size_t kPartialBudget = (size_t)4 << 30;   // bytes of partials per chunk
@@ -597,7 +654,7 @@ Plan make_plan(const Shape &s) {
     p.toffs = o;    o += al(sizeof(int) * (p.L + 1));
     p.entries = o;  o += al(sizeof(int) * slots);
     p.tiles = o;    o += al(sizeof(int4) * (slots + p.L));
-    p.part_o = o;   o += al(sizeof(__half) * slots * s.R * s.d);
+    p.part_o = o;   o += al(sizeof(__half) * ((slots * s.R + 31) / 32 * 32) * s.d);
     p.part_lse = o; o += al(sizeof(float) * slots * s.R);
     p.total = o;
     return p;
@@ -651,16 +708,15 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         a.tiles = tiles;
         a.n_tiles = toffs + L;
         a.part_o = part_o; a.part_lse = part_lse; a.err = err; a.r0 = r0;
+        a.n_prows = rc * s.G * s.topk * s.R;
         a.T = s.T; a.S = s.S; a.Hq = s.Hq; a.G = s.G; a.R = s.R; a.NB = s.NB; a.topk = s.topk;
         a.tpt = pl.tpt;
         a.scale = s.scale;
         a.scale_log2 = s.scale * kLog2e;
         kern<<<sms, kThreads, smem, st>>>(tq, tk, tv, a);
-        const int64_t warps = rc * s.Hq;
-        combine_kernel<D><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
-            ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R,
-            s.NB, s.block, s.topk);
-        count_launches(6);
+        e = launch_combine(s, ids, part_o, part_lse, O, lse, r0, rc, st);
+        if (e != cudaSuccess) return e;
+        count_launches(5);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -672,17 +728,29 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st) {
-    const int64_t warps = rc * s.Hq;
-    combine_kernel<128><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
-        ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
-        s.block, s.topk);
+    const int64_t warps = rc * s.G * (128 / 32);
+    const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+    const int per = (s.topk + 32 / s.R - 1) / (32 / s.R);
+    if (per <= 8)
+        combine_kernel<128, 8><<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O, lse,
+                                                     r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
+                                                     s.block, s.topk);
+    else
+        combine_kernel<128, 16><<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O,
+                                                      lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
+                                                      s.block, s.topk);
     count_launches(1);
     return cudaGetLastError();
 }
 
+bool combine_supported(const Shape &s) {
+    return (s.R == 1 || s.R == 2 || s.R == 4 || s.R == 8 || s.R == 16 || s.R == 32) &&
+           s.topk <= 64 && (s.topk + 32 / s.R - 1) / (32 / s.R) <= 16;
+}
+
 bool attn_tc_supported(const Shape &s) {
-    return s.dtype == MSA_BF16 && s.d == 128 && (s.block == 128 || s.block == 64) &&
-           (s.R == 1 || s.R == 2 || s.R == 4 || s.R == 8 || s.R == 16) && s.topk <= 256;
+    return s.dtype == MSA_BF16 && s.d == 128 && (s.block == 128 || s.block == 64) && s.R <= 16 &&
+           combine_supported(s);
 }
 
 size_t attn_tc_workspace(const Shape &s) { return make_plan(s).total; }

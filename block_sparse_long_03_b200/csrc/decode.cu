@@ -192,7 +192,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
                     const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ ids,
                     __half *__restrict__ part_o, float *__restrict__ part_lse, uint32_t *err,
                     int T_, int S, int Hq, int Hkv, int R, int NB, int topk, float scale_log2,
-                    float scale) {
+                    float scale, int64_t n_prows) {
     constexpr int kRowBytes = D * 2;
     constexpr int kChunks = D / 8;
     extern __shared__ __align__(128) uint8_t sm[];
@@ -359,11 +359,12 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
         }
     }
     __syncthreads();
-    // write the R partial rows (D fp16 each) and their LSE
+    // write the R partial rows in the blocked chunk layout (partial_chunk)
+    // and their LSE
     const int64_t prow0 = (rg * topk + slot) * R;
     for (int c = tid; c < R * kChunks; c += kAttnThreads) {
-        const int h = c / kChunks, ch = c % kChunks;
-        *(uint4 *)(part_o + (prow0 + h) * D + ch * 8) = *(const uint4 *)(sO + h * D + ch * 8);
+        const int h = c % R, ch = c / R;
+        ((uint4 *)part_o)[partial_chunk(prow0 + h, ch, D)] = *(const uint4 *)(sO + h * D + ch * 8);
     }
     if (tid < R) {
         const int h = tid;
@@ -412,13 +413,15 @@ cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const v
     const float scale_log2 = s.scale * 1.4426950408889634f;
     k<<<(unsigned)ctas, kAttnThreads, smem, st>>>(
         (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, ids, part_o,
-        part_lse, err, s.T, s.S, s.Hq, s.Hkv, s.R, s.NB, s.topk, scale_log2, s.scale);
+        part_lse, err, s.T, s.S, s.Hq, s.Hkv, s.R, s.NB, s.topk, scale_log2, s.scale,
+        (int64_t)s.index_rows() * s.topk * s.R);
     count_launches(1);
     return cudaGetLastError();
 }
 
 size_t part_bytes_o(const Shape &s) {
-    return (((size_t)s.index_rows() * s.topk * s.R * s.d * 2) + 255) / 256 * 256;
+    const size_t rows = ((size_t)s.index_rows() * s.topk * s.R + 31) / 32 * 32;
+    return ((rows * s.d * 2) + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -436,7 +439,7 @@ cudaError_t launch_decode_index(const Shape &s, const void *q_idx, const void *k
 
 bool decode_attn_supported(const Shape &s) {
     return s.dtype == MSA_BF16 && s.d == 128 && s.R <= 8 && (s.block == 64 || s.block == 128) &&
-           s.index_rows() * s.topk < (1ll << 31);
+           s.index_rows() * s.topk < (1ll << 31) && combine_supported(s);
 }
 
 size_t decode_attn_workspace(const Shape &s) {

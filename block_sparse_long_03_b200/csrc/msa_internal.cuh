@@ -60,6 +60,17 @@ size_t attn_tc_workspace(const Shape &s);
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st);
+// Partial outputs (fp16, one row of d channels per (query row, head, kept
+// slot)) are stored in 16-byte chunks, blocked by 32 rows: the chunk c of row
+// prow is uint4 number partial_chunk(prow, c).  Consecutive rows of one chunk
+// are adjacent (coalesced stores), and all chunks of 32 rows share one
+// contiguous d/8 * 512-byte span (page-local reads).
+__host__ __device__ __forceinline__ int64_t partial_chunk(int64_t prow, int c, int d) {
+    return (prow >> 5) * (int64_t)(d / 8) * 32 + (int64_t)c * 32 + (prow & 31);
+}
+
+// Shapes the combine kernel handles: R divides 32, topk <= 64, topk * R <= 512.
+bool combine_supported(const Shape &s);
 // LSE-weighted combine of per-(row, head, kept slot) partials into O and lse
 // for query rows [r0, r0 + rc) (d = 128).
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,

@@ -83,6 +83,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// 2^x for two halves at once (PTX ex2.approx.f16x2): one special-function
+// instruction per pair.
+__device__ __forceinline__ uint32_t ex2_approx_h2(uint32_t x2) {
+    uint32_t y;
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x2));
+    return y;
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar,
