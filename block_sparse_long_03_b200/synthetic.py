@@ -68,6 +68,12 @@ WORKLOADS = {
     "chunked_prefill_1m": Workload("chunked_prefill_1m", B=1, T=4096, S=1 << 20, Hq=32, Hkv=4,
                                    d=128, d_idx=64, block=128, topk=64, dtype=torch.bfloat16,
                                    hot_blocks_per_group=32),
+    # Reduced sizes of the same shapes, small enough for profiler captures
+    # (a few GB on the device).
+    "prefill_8k": Workload("prefill_8k", B=1, T=8192, S=8192, Hq=64, Hkv=8, d=128, d_idx=64,
+                           block=128, topk=32, dtype=torch.bfloat16, hot_blocks_per_group=8),
+    "decode_4x128k": Workload("decode_4x128k", B=4, T=1, S=131072, Hq=32, Hkv=8, d=128,
+                              d_idx=64, block=64, topk=32, dtype=torch.bfloat16),
 }
 
 
