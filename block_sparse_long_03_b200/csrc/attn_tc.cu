@@ -36,55 +36,66 @@ constexpr int kThreads = 320;        // warp 0 loads, warp 1 MMA, warps 2-9 soft
 constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// True when the row's non-negative ids are strictly ascending (the form
-// msa_topk_blocks writes), so no id can repeat.
-__device__ __forceinline__ bool row_ascending(const int32_t *row, int topk) {
-    int prev = -1;
-    for (int i = 0; i < topk; ++i) {
-        const int n = row[i];
-        if (n < 0) continue;
-        if (n <= prev) return false;
-        prev = n;
+// Validity of the kept slots lane and lane + 32 of a row (topk <= 64),
+// computed by one warp: in range, holding a causal token, and not a repeat
+// (a strictly ascending row, the form msa_topk_blocks writes, cannot repeat;
+// otherwise earlier slots are scanned).  bad = an id >= NB or a repeat.
+struct SlotPair {
+    int id0, id1;
+    bool ok0, ok1, bad0, bad1;
+};
+__device__ __forceinline__ SlotPair warp_slots(const int32_t *row, int topk, int NB, int cb,
+                                               int lane) {
+    SlotPair r;
+    r.id0 = lane < topk ? row[lane] : -1;
+    r.id1 = lane + 32 < topk ? row[lane + 32] : -1;
+    int pm0 = r.id0;
+    for (int off = 1; off < 32; off *= 2) {
+        const int o = __shfl_up_sync(0xffffffffu, pm0, off);
+        if (lane >= off) pm0 = max(pm0, o);
     }
-    return true;
-}
-
-// Validity of slot `i` of a kept-id row, shared by every phase: in range, not
-// a repeat of an earlier slot, and holding at least one causal token.
-// `ascending` (from row_ascending) skips the repeat scan.
-__device__ __forceinline__ bool slot_valid(const int32_t *row, int i, int NB, int cb,
-                                           bool ascending, bool *bad) {
-    const int n = row[i];
-    *bad = false;
-    if (n < 0) return false;
-    if (n >= NB) { *bad = true; return false; }
-    if (!ascending)
-        for (int k = 0; k < i; ++k)
-            if (row[k] == n) { *bad = true; return false; }
-    return n <= cb;
+    const int before0 = __shfl_up_sync(0xffffffffu, pm0, 1);
+    const int max_first = __shfl_sync(0xffffffffu, pm0, 31);
+    int pm1 = r.id1;
+    for (int off = 1; off < 32; off *= 2) {
+        const int o = __shfl_up_sync(0xffffffffu, pm1, off);
+        if (lane >= off) pm1 = max(pm1, o);
+    }
+    const int before1 = max(max_first, __shfl_up_sync(0xffffffffu, pm1, 1));
+    const bool dis0 = r.id0 >= 0 && lane > 0 && r.id0 <= before0;
+    const bool dis1 = r.id1 >= 0 && (lane > 0 ? r.id1 <= before1 : r.id1 <= max_first);
+    const bool asc = !__any_sync(0xffffffffu, dis0 || dis1);
+    bool rep0 = false, rep1 = false;
+    if (!asc) {
+        for (int q = 0; q < lane && r.id0 >= 0; ++q) rep0 |= row[q] == r.id0;
+        for (int q = 0; q < lane + 32 && r.id1 >= 0; ++q) rep1 |= row[q] == r.id1;
+    }
+    r.bad0 = r.id0 >= NB || (r.id0 >= 0 && rep0);
+    r.bad1 = r.id1 >= NB || (r.id1 >= 0 && rep1);
+    r.ok0 = r.id0 >= 0 && !r.bad0 && r.id0 <= cb;
+    r.ok1 = r.id1 >= 0 && !r.bad1 && r.id1 <= cb;
+    return r;
 }
 
 // ---------------------------------------------------------------- CSR build
 
-// counts[(b*G + g)*NB + n] += 1 for every valid kept slot of the chunk's rows.
+// counts[(b*G + g)*NB + n] += 1 for every valid kept slot of the chunk's rows;
+// one warp per (row, group), one lane per slot.
 __global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restrict__ counts,
                                  uint32_t *err, int64_t r0, int64_t rc, int T_, int S, int G,
                                  int NB, int block, int topk) {
-    const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
     const int64_t r = r0 + x / G;                 // b * T + t
     const int g = (int)(x % G);
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
-    const int32_t *row = ids + (r * G + g) * topk;
-    const bool asc = row_ascending(row, topk);
-    for (int i = 0; i < topk; ++i) {
-        bool bad;
-        if (slot_valid(row, i, NB, cb, asc, &bad))
-            atomicAdd(&counts[((int64_t)b * G + g) * NB + row[i]], 1);
-        else if (bad)
-            record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
-    }
+    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    int *base = counts + ((int64_t)b * G + g) * NB;
+    if (sp.ok0) atomicAdd(base + sp.id0, 1);
+    if (sp.ok1) atomicAdd(base + sp.id1, 1);
+    if (sp.bad0 || sp.bad1) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
 }
 
 // Single-CTA exclusive scans: offs = scan(counts), tile_offs = scan(ceil(counts / tpt)).
@@ -118,24 +129,28 @@ __global__ void csr_scan_kernel(const int *__restrict__ counts, int *__restrict_
     if (tid == nt - 1) { offs[L] = s_a[nt - 1]; tile_offs[L] = s_b[nt - 1]; }
 }
 
-// entries[offs[list] + k] = (row - r0) << 8 | slot, for every valid kept slot.
+// entries[offs[list] + k] = (row - r0) << 8 | slot, for every valid kept slot;
+// one warp per (row, group), one lane per slot.
 __global__ void csr_fill_kernel(const int32_t *__restrict__ ids, const int *__restrict__ offs,
                                 int *__restrict__ cursor, int *__restrict__ entries, int64_t r0,
                                 int64_t rc, int T_, int S, int G, int NB, int block, int topk) {
-    const int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
     const int64_t r = r0 + x / G;
     const int g = (int)(x % G);
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
-    const int32_t *row = ids + (r * G + g) * topk;
-    const bool asc = row_ascending(row, topk);
-    for (int i = 0; i < topk; ++i) {
-        bool bad;
-        if (!slot_valid(row, i, NB, cb, asc, &bad)) continue;
-        const int64_t list = ((int64_t)b * G + g) * NB + row[i];
-        const int pos = atomicAdd(&cursor[list], 1);
-        entries[offs[list] + pos] = (int)(((r - r0) << 8) | i);
+    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const int64_t lbase = ((int64_t)b * G + g) * NB;
+    const int tag = (int)((r - r0) << 8);
+    if (sp.ok0) {
+        const int64_t list = lbase + sp.id0;
+        entries[offs[list] + atomicAdd(&cursor[list], 1)] = tag | lane;
+    }
+    if (sp.ok1) {
+        const int64_t list = lbase + sp.id1;
+        entries[offs[list] + atomicAdd(&cursor[list], 1)] = tag | (lane + 32);
     }
 }
 
@@ -535,28 +550,7 @@ combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_
     const int64_t r = r0 + rl;
     const int t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
-    const int32_t *row = ids + (r * G + g) * topk;
-    // the row's ids, slot lane and lane + 32
-    const int id0 = lane < topk ? row[lane] : -1;
-    const int id1 = lane + 32 < topk ? row[lane + 32] : -1;
-    // strictly ascending over the non-negative ids <=> every id exceeds the
-    // running maximum of the ids before it (warp prefix-max scan)
-    int pm0 = id0;
-    for (int off = 1; off < 32; off *= 2) {
-        const int o = __shfl_up_sync(0xffffffffu, pm0, off);
-        if (lane >= off) pm0 = max(pm0, o);
-    }
-    const int before0 = __shfl_up_sync(0xffffffffu, pm0, 1);
-    const int max_first = __shfl_sync(0xffffffffu, pm0, 31);
-    int pm1 = id1;
-    for (int off = 1; off < 32; off *= 2) {
-        const int o = __shfl_up_sync(0xffffffffu, pm1, off);
-        if (lane >= off) pm1 = max(pm1, o);
-    }
-    const int before1 = max(max_first, __shfl_up_sync(0xffffffffu, pm1, 1));
-    const bool bad0 = id0 >= 0 && lane > 0 && id0 <= before0;
-    const bool bad1 = id1 >= 0 && (lane > 0 ? id1 <= before1 : id1 <= max_first);
-    const bool asc = !__any_sync(0xffffffffu, bad0 || bad1);
+    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
     const int h = lane % R, s0 = lane / R, sstep = 32 / R;
     const int per = (topk + sstep - 1) / sstep;
     const int64_t base = (rl * G + g) * topk * R;
@@ -564,11 +558,8 @@ combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_
 #pragma unroll
     for (int k = 0; k < kMaxPer; ++k) {
         const int sl = s0 + k * sstep;
-        const int idk = __shfl_sync(0xffffffffu, sl < 32 ? id0 : id1, sl & 31);
-        bool ok = k < per && sl < topk && idk >= 0 && idk < NB && idk <= cb;
-        if (ok && !asc) {                          // rare: caller ids out of order
-            for (int q = 0; q < sl; ++q) ok = ok && row[q] != idk;
-        }
+        const bool okk = __shfl_sync(0xffffffffu, sl < 32 ? sp.ok0 : sp.ok1, sl & 31);
+        const bool ok = k < per && sl < topk && okk;
         li[k] = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
         m = fmaxf(m, li[k]);
     }
@@ -694,8 +685,8 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         const int64_t rc = std::min<int64_t>(pl.rows_per_chunk, s.rows() - r0);
         e = cudaMemsetAsync(counts, 0, pl.offs - pl.counts, st);   // counts and cursor
         if (e != cudaSuccess) return e;
-        const int64_t nrow = rc * s.G;
-        const unsigned g1 = (unsigned)((nrow + 255) / 256);
+        const int64_t nrow = rc * s.G;                      // one warp each
+        const unsigned g1 = (unsigned)((nrow * 32 + 255) / 256);
         csr_count_kernel<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB,
                                              s.block, s.topk);
         csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offs, toffs, L, pl.tpt);
