@@ -163,11 +163,23 @@ def _barrier(ws):
 
 
 def _max_over_ranks(x: float, ws: int) -> float:
+    """The slowest rank's value (timing metadata only; no data-path exchange)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Every rank works on its own independent problem (weak scaling)."""
+    return 1000 * rank
+
+
+def aggregate_tokens_per_s(tokens_per_rank: int, ms_max: float, ws: int) -> float:
+    """Whole-job throughput: the tokens of all ranks over the slowest rank's time."""
+    return ws * tokens_per_rank / (ms_max / 1e3)
 
 
 class Problem:
@@ -262,7 +274,7 @@ def e2e_prefill(prob: Problem, steps: int, warmup: int, ws: int) -> dict:
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = host_O.numel() * host_O.element_size() + host_lse.numel() * host_lse.element_size()
     del dev_in
-    return {"value": ws * w.B * w.T / (ms / 1e3), "unit": "tokens/s",
+    return {"value": aggregate_tokens_per_s(w.B * w.T, ms, ws), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": ms}
 
 
@@ -340,14 +352,14 @@ def run_ours(args, rank: int, ws: int):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     pk = peaks()
-    prob = Problem(args.workload, seed=rank)
+    prob = Problem(args.workload, seed=rank_seed(rank))
     w = prob.w
     launches0 = msa.msa_kernel_launches()
     with ClockSampler(local) as clk:
         ms = time_steps(prob.step, args.steps, args.warmup, ws)
     timed_launches = msa.msa_kernel_launches() - launches0
     per_step = timed_launches / float(args.steps + args.warmup)
-    value = ws * w.B * w.T / (ms / 1e3)
+    value = aggregate_tokens_per_s(w.B * w.T, ms, ws)
     stages = prob.stage_times_ms(max(2, args.steps))
     attn_fl, idx_fl = attention_flops(w), index_flops(w)
     dominant = max(stages, key=stages.get)
@@ -368,7 +380,7 @@ def run_ours(args, rank: int, ws: int):
 
     decode = None
     if not args.no_decode:
-        dp = Problem(DECODE, seed=100 + rank)
+        dp = Problem(DECODE, seed=rank_seed(rank) + 1)
         with ClockSampler(local) as dclk:
             dms = time_steps(dp.step, max(args.steps, 10), args.warmup, ws)
         dst = dp.stage_times_ms(max(args.steps, 10))

@@ -8,14 +8,15 @@ in ``include/msa.h``); this package is its Python binding.
 from .binding import (EXPORTS, MSA_BF16, MSA_F32, MSA_OK, MSA_WS_FORWARD, MSA_WS_SPARSE_ATTN,
                       MsaError, Params, alloc_workspace, forward, index_block_scores,
                       make_params, msa_forward, msa_get_device_error, msa_index_block_scores,
-                      msa_kernel_launches,
+                      msa_kernel_launches, msa_selftest_wait_timeout,
                       msa_sparse_attn_fwd, msa_topk_blocks, msa_workspace_size, params_from,
                       sparse_attn_fwd, status_string, topk_blocks)
 
 __all__ = [
     "EXPORTS", "MSA_BF16", "MSA_F32", "MSA_OK", "MSA_WS_FORWARD", "MSA_WS_SPARSE_ATTN",
     "MsaError", "Params", "alloc_workspace", "forward", "index_block_scores", "make_params",
-    "msa_forward", "msa_get_device_error", "msa_index_block_scores", "msa_kernel_launches", "msa_sparse_attn_fwd",
+    "msa_forward", "msa_get_device_error", "msa_index_block_scores", "msa_kernel_launches",
+    "msa_selftest_wait_timeout", "msa_sparse_attn_fwd",
     "msa_topk_blocks", "msa_workspace_size", "params_from", "sparse_attn_fwd", "status_string",
     "topk_blocks",
 ]

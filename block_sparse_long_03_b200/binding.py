@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
-           "msa_kernel_launches", "msa_forward_noalloc")
+           "msa_kernel_launches", "msa_forward_noalloc", "msa_selftest_wait_timeout")
 
 
 class MsaError(RuntimeError):
@@ -59,6 +59,8 @@ def _load():
     lib.msa_get_device_error.argtypes = [vp, vp]
     lib.msa_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.msa_forward_noalloc.restype = st
+    lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
+    lib.msa_selftest_wait_timeout.restype = st
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = ctypes.c_uint64
     for name in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd",
@@ -141,6 +143,12 @@ def msa_forward(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, worksp
 def msa_get_device_error(workspace, stream=None) -> int:
     """The status recorded on the device by the last call that used `workspace`."""
     return int(lib.msa_get_device_error(_ptr(workspace), _stream(stream)))
+
+
+def msa_selftest_wait_timeout(workspace, limit_us: int, stream=None):
+    """Run the device wait-timeout check (see include/msa.h)."""
+    _check(lib.msa_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us),
+                                         _stream(stream)), "msa_selftest_wait_timeout")
 
 
 def msa_kernel_launches() -> int:

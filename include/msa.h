@@ -198,6 +198,18 @@ MSA_EXPORT msa_status_t msa_forward_noalloc(const msa_params_t *params, const vo
                                             float *lse, void *stream);
 
 /*
+ * Diagnostics: a check of the device failure path.  Launches one CTA that
+ * takes the library's bounded mbarrier wait on a barrier nothing completes,
+ * with a limit of limit_us microseconds (1 .. 1,000,000).  When the wait
+ * gives up the kernel records MSA_ERR_DEVICE_TIMEOUT in the error word of
+ * `workspace` (at least 256 bytes, 256-byte aligned), releases its tensor
+ * memory and returns; read the status with msa_get_device_error.  Every wait
+ * of the library's kernels ends this way (limit 2 s) instead of hanging.
+ */
+MSA_EXPORT msa_status_t msa_selftest_wait_timeout(void *workspace, size_t workspace_bytes,
+                                                  uint32_t limit_us, void *stream);
+
+/*
  * Diagnostics: the number of CUDA kernels this library has launched in this
  * process since it was loaded (all devices, all calls).  Lets a caller count
  * the kernels a region of work issued.

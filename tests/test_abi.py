@@ -20,7 +20,7 @@ def test_header_declares_the_calls():
     names = declared_symbols()
     for want in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd", "msa_forward",
                  "msa_workspace_size", "msa_status_string", "msa_get_device_error",
-                 "msa_kernel_launches"):
+                 "msa_kernel_launches", "msa_selftest_wait_timeout"):
         assert want in names
 
 

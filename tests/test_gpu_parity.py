@@ -42,12 +42,28 @@ def _case(name):
                         block=64, topk=1, dtype=bf),
         "fp32_gqa8": W("fp32_gqa8", B=1, T=384, S=512, Hq=16, Hkv=2, d=128, d_idx=64,
                        block=128, topk=3, dtype=torch.float32),
+        # tensor-core prefill path across group sizes, index widths and batching
+        "bf16_prefill_R16": W("bf16_prefill_R16", B=1, T=1024, S=1024, Hq=32, Hkv=2, d=128,
+                              d_idx=64, block=128, topk=4, dtype=bf, hot_blocks_per_group=1),
+        "bf16_prefill_R1_didx128": W("bf16_prefill_R1_didx128", B=1, T=512, S=512, Hq=4, Hkv=4,
+                                     d=128, d_idx=128, block=64, topk=5, dtype=bf),
+        "bf16_prefill_B2_chunk": W("bf16_prefill_B2_chunk", B=2, T=300, S=1024, Hq=8, Hkv=4,
+                                   d=128, d_idx=64, block=128, topk=3, dtype=bf),
+        # decode path: block 128, several query tokens, 64 kept blocks (two slot passes)
+        "bf16_decode_block128": W("bf16_decode_block128", B=3, T=1, S=4096, Hq=16, Hkv=2, d=128,
+                                  d_idx=64, block=128, topk=6, dtype=bf),
+        "bf16_decode_T4": W("bf16_decode_T4", B=2, T=4, S=2048, Hq=8, Hkv=2, d=128, d_idx=64,
+                            block=64, topk=4, dtype=bf),
+        "bf16_decode_topk64": W("bf16_decode_topk64", B=2, T=1, S=8192, Hq=32, Hkv=4, d=128,
+                                d_idx=64, block=64, topk=64, dtype=bf),
     }
     return cases[name]
 
 
 CASES = ["tiny_fp32_prefill", "bf16_prefill_2x1024", "bf16_chunk_ragged", "bf16_decode_small",
-         "bf16_d64_mha", "bf16_dense_limit", "bf16_topk1", "fp32_gqa8"]
+         "bf16_d64_mha", "bf16_dense_limit", "bf16_topk1", "fp32_gqa8", "bf16_prefill_R16",
+         "bf16_prefill_R1_didx128", "bf16_prefill_B2_chunk", "bf16_decode_block128",
+         "bf16_decode_T4", "bf16_decode_topk64"]
 
 
 def _inputs(w, seed=0):
