@@ -32,7 +32,7 @@ namespace msa {
 namespace {
 
 constexpr int kRows = 128;           // tile rows = tokens_per_tile * R
-constexpr int kThreads = 320;        // warp 0 loads, warp 1 MMA, warps 2-9 softmax/epilogue
+constexpr int kThreads = 512;        // four warpgroups: loads + MMA, two softmax, epilogue
 constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -98,42 +98,43 @@ __global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restric
     if (sp.bad0 || sp.bad1) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
 }
 
-// Single-CTA exclusive scans: offs = scan(counts), tile_offs = scan(ceil(counts / tpt)).
-// offs[L] and tile_offs[L] hold the totals.
-__global__ void csr_scan_kernel(const int *__restrict__ counts, int *__restrict__ offs,
-                                int *__restrict__ tile_offs, int L, int tpt) {
-    __shared__ int s_a[1024], s_b[1024];
+// Single-CTA exclusive scan: tile_offs = scan(ceil(counts / tpt)); tile_offs[L]
+// holds the number of tiles.
+__global__ void csr_scan_kernel(const int *__restrict__ counts, int *__restrict__ tile_offs, int L,
+                                int tpt) {
+    __shared__ int s_b[1024];
     const int tid = threadIdx.x, nt = blockDim.x;
     const int per = (L + nt - 1) / nt;
     const int lo = min(L, tid * per), hi = min(L, lo + per);
-    int a = 0, b = 0;
-    for (int i = lo; i < hi; ++i) { a += counts[i]; b += (counts[i] + tpt - 1) / tpt; }
-    s_a[tid] = a;
+    int b = 0;
+    for (int i = lo; i < hi; ++i) b += (counts[i] + tpt - 1) / tpt;
     s_b[tid] = b;
     __syncthreads();
     for (int off = 1; off < nt; off *= 2) {       // inclusive Hillis-Steele scan
-        const int va = tid >= off ? s_a[tid - off] : 0;
         const int vb = tid >= off ? s_b[tid - off] : 0;
         __syncthreads();
-        s_a[tid] += va;
         s_b[tid] += vb;
         __syncthreads();
     }
-    int ea = s_a[tid] - a, eb = s_b[tid] - b;      // exclusive
+    int eb = s_b[tid] - b;                         // exclusive
     for (int i = lo; i < hi; ++i) {
-        offs[i] = ea;
         tile_offs[i] = eb;
-        ea += counts[i];
         eb += (counts[i] + tpt - 1) / tpt;
     }
-    if (tid == nt - 1) { offs[L] = s_a[nt - 1]; tile_offs[L] = s_b[nt - 1]; }
+    if (tid == nt - 1) tile_offs[L] = s_b[nt - 1];
 }
 
-// entries[offs[list] + k] = (row - r0) << 8 | slot, for every valid kept slot;
-// one warp per (row, group), one lane per slot.
-__global__ void csr_fill_kernel(const int32_t *__restrict__ ids, const int *__restrict__ offs,
-                                int *__restrict__ cursor, int *__restrict__ entries, int64_t r0,
-                                int64_t rc, int T_, int S, int G, int NB, int block, int topk) {
+// Tile records: record k of a chunk is rec_ints(tpt) ints, {list, tokens in
+// the tile, 0, 0, entry[0 .. tpt)} with entry = (row - r0) << 8 | slot, so a
+// tile's description is one contiguous read with no dependent load.
+__host__ __device__ constexpr int rec_ints(int tpt) { return 4 + tpt; }
+
+// Every valid kept slot of the chunk's rows into its list's next free record
+// entry; one warp per (row, group), one lane per slot.
+__global__ void csr_fill_kernel(const int32_t *__restrict__ ids,
+                                const int *__restrict__ tile_offs, int *__restrict__ cursor,
+                                int *__restrict__ recs, int64_t r0, int64_t rc, int T_, int S,
+                                int G, int NB, int block, int topk, int tpt) {
     const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
@@ -146,26 +147,28 @@ __global__ void csr_fill_kernel(const int32_t *__restrict__ ids, const int *__re
     const int tag = (int)((r - r0) << 8);
     if (sp.ok0) {
         const int64_t list = lbase + sp.id0;
-        entries[offs[list] + atomicAdd(&cursor[list], 1)] = tag | lane;
+        const int pos = atomicAdd(&cursor[list], 1);
+        recs[(int64_t)(tile_offs[list] + pos / tpt) * rec_ints(tpt) + 4 + pos % tpt] = tag | lane;
     }
     if (sp.ok1) {
         const int64_t list = lbase + sp.id1;
-        entries[offs[list] + atomicAdd(&cursor[list], 1)] = tag | (lane + 32);
+        const int pos = atomicAdd(&cursor[list], 1);
+        recs[(int64_t)(tile_offs[list] + pos / tpt) * rec_ints(tpt) + 4 + pos % tpt] =
+            tag | (lane + 32);
     }
 }
 
-// tiles[tile_offs[list] + c] = {list, tokens in the tile, index of its first
-// entry, 0} for every tile of every list.
-__global__ void csr_tiles_kernel(const int *__restrict__ counts, const int *__restrict__ offs,
-                                 const int *__restrict__ tile_offs, int4 *__restrict__ tiles,
-                                 int L, int tpt) {
+// Record headers {list, tokens in the tile, 0, 0} for every tile of every list.
+__global__ void csr_tiles_kernel(const int *__restrict__ counts, const int *__restrict__ tile_offs,
+                                 int *__restrict__ recs, int L, int tpt) {
     const int list = blockIdx.x * blockDim.x + threadIdx.x;
     if (list >= L) return;
     const int cnt = counts[list];
     const int nt = (cnt + tpt - 1) / tpt;
     const int base = tile_offs[list];
     for (int c = 0; c < nt; ++c)
-        tiles[base + c] = make_int4(list, min(tpt, cnt - c * tpt), offs[list] + c * tpt, 0);
+        *(int4 *)(recs + (int64_t)(base + c) * rec_ints(tpt)) =
+            make_int4(list, min(tpt, cnt - c * tpt), 0, 0);
 }
 
 }  // namespace
@@ -176,8 +179,7 @@ namespace {
 
 struct AttnArgs {
     const __nv_bfloat16 *Q;     // [B, T, Hq, D]
-    const int *entries;         // CSR entries: (row - r0) << 8 | slot
-    const int4 *tiles;          // {list, count, first entry, 0} per tile
+    const int *recs;            // tile records (rec_ints(tpt) ints each)
     const int *n_tiles;         // device-side tile count
     __half *part_o;             // normalised partial O, blocked chunks (partial_chunk)
     float *part_lse;            // [n_prows]
@@ -192,43 +194,71 @@ __device__ __forceinline__ int run_tile(int i) {
     return (i / kRun) * (gridDim.x * kRun) + blockIdx.x * kRun + (i % kRun);
 }
 
-__device__ __forceinline__ int4 load_tile(const AttnArgs &a, int i, int total) {
+// Header {list, count} of a CTA's i-th tile ({-1, 0} past the end) and entry
+// k (< tpt) of its record (0 past the end); independent loads.
+__device__ __forceinline__ int2 load_head(const AttnArgs &a, int i, int total) {
     const int tile = run_tile(i);
-    return tile < total ? a.tiles[tile] : make_int4(-1, 0, 0, 0);
+    return tile < total ? __ldg((const int2 *)(a.recs + (int64_t)tile * rec_ints(a.tpt)))
+                        : make_int2(-1, 0);
 }
+__device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int k) {
+    const int tile = run_tile(i);
+    return tile < total && k < a.tpt ? __ldg(a.recs + (int64_t)tile * rec_ints(a.tpt) + 4 + k) : 0;
+}
+
+// Warp roles (four warpgroups, 512 threads):
+//   warpgroup 0     warp 1 issues the MMAs; warps 0, 2 and 3 gather the Q
+//                   rows (cp.async) and warp 0 loads the K/V blocks (TMA);
+//   warpgroups 1-2  softmax, tiles 0, 2, 4, ... and 1, 3, 5, ...;
+//   warpgroup 3     epilogue of every tile: O from TMEM to an fp16 partial.
+// TMEM: three S/P buffers (S: BLOCK fp32 columns; P: bf16 pairs in the first
+// BLOCK/2 of them; the row max m and row sum l in the last two columns) at
+// columns 0, 128, 256 and one O accumulator at 384.  The epilogue divides O
+// by l, converts and stores it with the LSE, so no global store is issued by
+// the softmax warps; an S/P buffer is free again once PV has read P and the
+// epilogue has read m and l.
+constexpr int kRegsLoad = 88, kRegsSoftmax = 136, kRegsEpilogue = 152;
+static_assert(kRegsLoad + 2 * kRegsSoftmax + kRegsEpilogue <= 4 * (65536 / kThreads),
+              "warpgroup register budgets exceed the launch's registers");
 
 template <int D, int BLOCK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, AttnArgs a) {
     constexpr int kAtoms = D / 64;
+    constexpr int kQBuf = 3;                      // Q tiles in flight = S/P buffers
     constexpr uint32_t kQBytes = kRows * D * 2;
     constexpr uint32_t kKBytes = BLOCK * D * 2;
-    constexpr uint32_t kAccCols = 256;            // S (BLOCK) + O (D) per accumulator set
-    static_assert(BLOCK + D <= (int)kAccCols, "TMEM budget");
+    constexpr uint32_t kSCols = 128, kOCol = 384;
+    static_assert(BLOCK <= (int)kSCols && D <= 128, "TMEM budget");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = smem;                           // [2][kAtoms][128][64]
-    uint8_t *sK = sQ + 2 * kQBytes;               // [2][kAtoms][BLOCK][64]
+    uint8_t *sQ = smem;                           // [3][kAtoms][128][64]
+    uint8_t *sK = sQ + kQBuf * kQBytes;           // [2][kAtoms][BLOCK][64]
     uint8_t *sV = sK + 2 * kKBytes;               // [2][kAtoms][BLOCK][64]
     uint64_t *bar = (uint64_t *)(sV + 2 * kKBytes);
-    uint64_t *q_full = bar, *q_empty = bar + 2, *kv_full = bar + 4, *kv_empty = bar + 6;
-    uint64_t *s_full = bar + 8, *p_full = bar + 10, *o_full = bar + 12, *acc_empty = bar + 14;
-    uint32_t *tmem_slot = (uint32_t *)(bar + 16);
+    uint64_t *q_full = bar, *q_empty = bar + 3;   // [3] each
+    uint64_t *kv_full = bar + 6, *kv_empty = bar + 8;        // [2] each
+    uint64_t *s_full = bar + 10, *p_full = bar + 13, *s_free = bar + 16;   // [3] each
+    uint64_t *o_full = bar + 19, *o_empty = bar + 20;
+    uint32_t *tmem_slot = (uint32_t *)(bar + 21);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 32);
+        for (int i = 0; i < kQBuf; ++i) {
+            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 96);   // TMA: one; cp.async: per thread
             tc::mbar_init(&q_empty[i], 1);
-            tc::mbar_init(&kv_full[i], 1);
-            tc::mbar_init(&kv_empty[i], 1);
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_full[i], 128);
-            tc::mbar_init(&o_full[i], 1);
-            tc::mbar_init(&acc_empty[i], 128);
+            tc::mbar_init(&s_free[i], 1 + 128);    // PV commit + epilogue threads
         }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&kv_full[i], 1);
+            tc::mbar_init(&kv_empty[i], 1);
+        }
+        tc::mbar_init(o_full, 1);
+        tc::mbar_init(o_empty, 128);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -238,274 +268,346 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int total = *a.n_tiles;
+    const int wg = warp / 4;
 
-    if (warp == 0) {
-        // ------------------------------------------------ loads: K/V blocks and Q rows by TMA
-        // The next tile's descriptor and entries are fetched one tile ahead.
-        int kvb = -1, cur_list = -1;
-        uint32_t kv_ph = 0, q_ph = 0;              // per-buffer phase bits
-        int4 nd = load_tile(a, 0, total);
-        int ne[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int tt = lane + 32 * k;
-            ne[k] = tt < nd.y ? a.entries[nd.z + tt] : 0;
-        }
-        for (int i = 0;; ++i) {
-            const int4 d = nd;
-            int e[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) e[k] = ne[k];
-            if (d.x < 0 || *abort_flag) break;
-            nd = load_tile(a, i + 1, total);
+    // Each role sets its warpgroup's register budget first.
+    if (wg == 0) {
+        tc::regs_dec<kRegsLoad>();
+        if (warp == 0 || (warp >= 2 && a.R < 8)) {
+            // ------------------------------------------------ loads
+            // K/V blocks by TMA (warp 0, lane 0) whenever the list changes, and
+            // the tile's Q rows gathered by warps 0, 2 and 3 with 16-byte
+            // cp.async copies straight into the 128-byte-swizzled K-major
+            // layout the MMA reads.  Each warp instruction copies two whole
+            // 256-byte rows; lane l always copies 16-byte chunk l % 16.  A
+            // thread's copies arrive on q_full when they complete
+            // (cp.async.mbarrier.arrive.noinc), so no warp waits for its own
+            // copies and loads run up to three tiles ahead.
+            const int gw = warp == 0 ? 0 : warp - 1;   // gather warp 0..2
+            const int cc = lane % 16;
+            const uint32_t q_swz = (uint32_t)(cc / 8) * (kRows * 128);
+            const int lr = __ffs(a.R) - 1;             // log2 R
+            int kvb = -1, cur_list = -1;
+            uint32_t kv_ph = 0;                        // per K/V buffer phase bits
+            // Records of the next two tiles in flight: lane l holds entries
+            // l, l + 32, l + 64, l + 96 of a record.
+            int2 h1 = load_head(a, 0, total), h2 = load_head(a, 1, total);
+            int e1[4], e2[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int tt = lane + 32 * k;
-                ne[k] = tt < nd.y ? a.entries[nd.z + tt] : 0;
+                e1[k] = load_ent(a, 0, total, lane + 32 * k);
+                e2[k] = load_ent(a, 1, total, lane + 32 * k);
             }
-            const int list = d.x, count = d.y;
-            const int n = list % a.NB, g = (list / a.NB) % a.G, b = list / (a.NB * a.G);
-            if (list != cur_list) {
-                kvb = (kvb + 1) & 1;
-                cur_list = list;
-                if (lane == 0 &&
-                    tc::mbar_wait(&kv_empty[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag)) {
-                    tc::mbar_expect_tx(&kv_full[kvb], 2 * kKBytes);
-                    const int key0 = b * a.S + n * BLOCK;
+            for (int i = 0;; ++i) {
+                const int2 d = h1;
+                int e[4];
 #pragma unroll
-                    for (int at = 0; at < kAtoms; ++at) {
-                        tc::tma_load_3d(sK + kvb * kKBytes + at * BLOCK * 128, &tm_k,
-                                        &kv_full[kvb], at * 64, g, key0);
-                        tc::tma_load_3d(sV + kvb * kKBytes + at * BLOCK * 128, &tm_v,
-                                        &kv_full[kvb], at * 64, g, key0);
-                    }
-                }
-                kv_ph ^= 1u << kvb;
-            }
-            const int qb = i & 1;
-            if (!tc::mbar_wait(&q_empty[qb], ((q_ph >> qb) & 1) ^ 1, a.err, abort_flag)) break;
-            q_ph ^= 1u << qb;
-            uint8_t *dst = sQ + qb * kQBytes;
-            if (a.R >= 8) {
-                // One TMA box per token: its R heads x 64 channels, R * 128 bytes, so
-                // every box starts on a 1024-byte swizzle-atom boundary.
-                if (lane == 0) tc::mbar_expect_tx(&q_full[qb], (uint32_t)count * a.R * D * 2);
-                __syncwarp();
+                for (int k = 0; k < 4; ++k) e[k] = e1[k];
+                if (d.x < 0) break;
+                h1 = h2;
+                h2 = load_head(a, i + 2, total);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int tt = lane + 32 * k;
-                    if (tt < count) {
-                        const int grow = (int)(a.r0 + (e[k] >> 8));
+                    e1[k] = e2[k];
+                    e2[k] = load_ent(a, i + 2, total, lane + 32 * k);
+                }
+                const int list = d.x, count = d.y;
+                const int n = list % a.NB, g = (list / a.NB) % a.G, b = list / (a.NB * a.G);
+                if (list != cur_list) {
+                    kvb = (kvb + 1) & 1;
+                    cur_list = list;
+                    if (warp == 0 && lane == 0 &&
+                        tc::mbar_wait(&kv_empty[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag)) {
+                        tc::mbar_expect_tx(&kv_full[kvb], 2 * kKBytes);
+                        const int key0 = b * a.S + n * BLOCK;
+#pragma unroll
+                        for (int at = 0; at < kAtoms; ++at) {
+                            tc::tma_load_3d(sK + kvb * kKBytes + at * BLOCK * 128, &tm_k,
+                                            &kv_full[kvb], at * 64, g, key0);
+                            tc::tma_load_3d(sV + kvb * kKBytes + at * BLOCK * 128, &tm_v,
+                                            &kv_full[kvb], at * 64, g, key0);
+                        }
+                    }
+                    kv_ph ^= 1u << kvb;
+                }
+                const int qb = i % kQBuf;
+                if (!tc::mbar_wait(&q_empty[qb], ((i / kQBuf) & 1) ^ 1, a.err, abort_flag)) break;
+                if (a.R >= 8) {
+                    // 8 or more heads per token: one TMA box per token and 64-channel
+                    // atom (R * 128 bytes, whole swizzle atoms); lane k < count holds
+                    // token k's entry.
+                    if (lane == 0)
+                        tc::mbar_expect_tx(&q_full[qb], (uint32_t)count * a.R * D * 2);
+                    __syncwarp();
+                    if (lane < count) {
+                        const int grow = (int)(a.r0 + (e[0] >> 8));
 #pragma unroll
                         for (int at = 0; at < kAtoms; ++at)
-                            tc::tma_load_3d(dst + at * kRows * 128 + tt * a.R * 128, &tm_q,
-                                            &q_full[qb], at * 64, g * a.R, grow);
+                            tc::tma_load_3d(sQ + qb * kQBytes + at * kRows * 128 + lane * a.R * 128,
+                                            &tm_q, &q_full[qb], at * 64, g * a.R, grow);
+                    }
+                    continue;
+                }
+                const uint32_t dst = tc::smem_u32(sQ + qb * kQBytes) + q_swz;
+                const int rows = count << lr;
+                const int64_t head0 = (int64_t)g * a.R;
+                // row pair q = rows 2q, 2q + 1 (lanes 0-15 / 16-31); both rows'
+                // tokens sit in the same 32-token block, so one register holds
+                // their entries and a shuffle hands each lane its token's entry
+                for (int q = gw; 2 * q < rows; q += 3) {
+                    const int r = 2 * q + lane / 16;
+                    const int tk = r >> lr, hh = r & (a.R - 1);
+                    const int kk = (2 * q) >> (lr + 5);
+                    const int ev = kk == 0 ? e[0] : kk == 1 ? e[1] : kk == 2 ? e[2] : e[3];
+                    const int ent = __shfl_sync(0xffffffffu, ev, tk & 31);
+                    if (r < rows) {
+                        const __nv_bfloat16 *src =
+                            a.Q + ((a.r0 + (ent >> 8)) * a.Hq + head0 + hh) * D + cc * 8;
+                        const uint32_t sa = dst + r * 128 + (((cc % 8) ^ (r % 8)) * 16);
+                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
+                                     "l"(src)
+                                     : "memory");
                     }
                 }
-            } else {
-                // Fewer than 8 heads per token: a token's rows do not fill a swizzle
-                // atom, so the rows are gathered with 16-byte cp.async copies into
-                // the 128-byte-swizzled layout directly.
-                constexpr int kChunksPerRow = D / 8;
-                const int nchunks = count * a.R * kChunksPerRow;
-                for (int c = lane; c < nchunks; c += 32) {
-                    const int r = c / kChunksPerRow, cc = c % kChunksPerRow;
-                    const int tk = r / a.R, hh = r % a.R;
-                    const int eval = a.entries[d.z + tk];
-                    const int64_t grow = a.r0 + (eval >> 8);
-                    const __nv_bfloat16 *src =
-                        a.Q + (grow * a.Hq + (int64_t)g * a.R + hh) * D + cc * 8;
-                    const uint32_t sa = tc::smem_u32(dst + (cc / 8) * (kRows * 128) + r * 128 +
-                                                     (((cc % 8) ^ (r % 8)) * 16));
-                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(src)
-                                 : "memory");
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];"
+                             ::"r"(tc::smem_u32(&q_full[qb])) : "memory");
+            }
+            // the last copies must land before the CTA can retire
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        } else if (warp == 1) {
+            // ------------------------------------------------ MMA issuer
+            // Iteration t issues S(t) = Q K^T and PV(t - 2): O = P V.  S(t) goes
+            // first, so the S of a softmax group's next tile is already computed
+            // when the group finishes its current one.  The one exception: when
+            // S(t) starts a list whose K/V buffer is released by PV(t - 2) (tile
+            // t - 2 was the last of its list), PV(t - 2) must be issued first or
+            // the load of that buffer would wait on an MMA never issued.
+            if (lane == 0) {
+                constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
+                constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
+                int kvb = -1, cur_list = -1;
+                uint32_t kv_ph = 0;
+                // K/V buffer and list of tiles t - 1 and t - 2 (-1: none)
+                int kvb1 = -1, kvb2 = -1, list1 = -1, list2 = -1;
+                int next_list = load_head(a, 0, total).x, next_list2 = load_head(a, 1, total).x;
+                for (int t = 0;; ++t) {
+                    const int list = next_list;
+                    const bool have = list >= 0 && !*abort_flag;
+                    if (have) {
+                        next_list = next_list2;
+                        next_list2 = load_head(a, t + 2, total).x;
+                    }
+                    const bool new_list = have && list != cur_list;
+                    const bool pv_first = !have || (new_list && list2 >= 0 && list1 != list2);
+                    auto issue_pv = [&]() -> bool {
+                        if (kvb2 < 0) return true;       // no tile t - 2
+                        const int tp = t - 2, bp = tp % kQBuf;
+                        if (!tc::mbar_wait(&p_full[bp], (tp / kQBuf) & 1, a.err, abort_flag))
+                            return false;
+                        if (tp >= 1 && !tc::mbar_wait(o_empty, (tp - 1) & 1, a.err, abort_flag))
+                            return false;
+                        tc::tc_fence_after();
+                        const uint32_t va = tc::smem_u32(sV + kvb2 * kKBytes);
+    #pragma unroll
+                        for (int ks = 0; ks < BLOCK / 16; ++ks) {
+                            const uint64_t bd = tc::sdesc_sw128(va + ks * 2048, BLOCK * 128, 1024);
+                            tc::mma_ts(tmem + kOCol, tmem + bp * kSCols + ks * 8, bd, idesc_o, ks > 0);
+                        }
+                        tc::mma_commit(o_full);
+                        tc::mma_commit(&s_free[bp]);
+                        if (list1 != list2) tc::mma_commit(&kv_empty[kvb2]);
+                        return true;
+                    };
+                    auto issue_s = [&]() -> bool {
+                        if (new_list) {
+                            kvb = (kvb + 1) & 1;
+                            cur_list = list;
+                            kv_ph ^= 1u << kvb;
+                        }
+                        const int bs = t % kQBuf;
+                        if (t >= kQBuf &&
+                            !tc::mbar_wait(&s_free[bs], ((t / kQBuf) - 1) & 1, a.err, abort_flag))
+                            return false;
+                        if (!tc::mbar_wait(&q_full[bs], (t / kQBuf) & 1, a.err, abort_flag))
+                            return false;
+                        if (!tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
+                            return false;
+                        tc::tc_fence_after();
+                        const uint32_t qa = tc::smem_u32(sQ + bs * kQBytes);
+                        const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
+    #pragma unroll
+                        for (int ks = 0; ks < D / 16; ++ks) {
+                            const uint64_t ad =
+                                tc::sdesc_sw128(qa + (ks / 4) * kRows * 128 + (ks % 4) * 32, 16, 1024);
+                            const uint64_t bd =
+                                tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
+                            tc::mma_ss(tmem + bs * kSCols, ad, bd, idesc_s, ks > 0);
+                        }
+                        tc::mma_commit(&q_empty[bs]);
+                        tc::mma_commit(&s_full[bs]);
+                        return true;
+                    };
+                    bool ok = true;
+                    if (pv_first) ok = issue_pv();
+                    if (ok && have) ok = issue_s();
+                    if (ok && !pv_first) ok = issue_pv();
+                    if (!ok) break;
+                    // shift the (t - 1, t - 2) history
+                    kvb2 = kvb1; list2 = list1;
+                    kvb1 = have ? kvb : -1; list1 = have ? list : -1;
+                    if (!have && kvb2 < 0) break;      // every PV issued
                 }
-                asm volatile("cp.async.commit_group;" ::: "memory");
-                asm volatile("cp.async.wait_group 0;" ::: "memory");
-                tc::fence_proxy_async();
-                tc::mbar_arrive(&q_full[qb]);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
-            constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
-            int kvb = -1, cur_list = -1;
-            uint32_t kv_ph = 0, q_ph = 0, acc_ph = 0, p_ph = 0;   // per-buffer phase bits
-            int prev_acc = -1, prev_kvb = -1, prev_list = -1;
-            int next_list = load_tile(a, 0, total).x;
-            for (int i = 0;; ++i) {
-                const int list = next_list;
-                const bool have = list >= 0 && !*abort_flag;
-                if (have) {
-                    next_list = load_tile(a, i + 1, total).x;
-                    if (list != cur_list) {
-                        kvb = (kvb + 1) & 1;
-                        cur_list = list;
-                        kv_ph ^= 1u << kvb;
-                    }
-                    const int acc = i & 1, qb = i & 1;
-                    if (!tc::mbar_wait(&acc_empty[acc], ((acc_ph >> acc) & 1) ^ 1, a.err, abort_flag))
-                        break;
-                    acc_ph ^= 1u << acc;
-                    if (!tc::mbar_wait(&q_full[qb], (q_ph >> qb) & 1, a.err, abort_flag)) break;
-                    q_ph ^= 1u << qb;
-                    if (!tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
-                        break;
-                    tc::tc_fence_after();
-                    const uint32_t qa = tc::smem_u32(sQ + qb * kQBytes);
-                    const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
-#pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks) {
-                        const uint64_t ad =
-                            tc::sdesc_sw128(qa + (ks / 4) * kRows * 128 + (ks % 4) * 32, 16, 1024);
-                        const uint64_t bd =
-                            tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
-                        tc::mma_ss(tmem + acc * kAccCols, ad, bd, idesc_s, ks > 0);
-                    }
-                    tc::mma_commit(&q_empty[qb]);
-                    tc::mma_commit(&s_full[acc]);
-                }
-                if (prev_acc >= 0) {
-                    // O = P V for the previous tile (P from TMEM, V from shared memory)
-                    if (!tc::mbar_wait(&p_full[prev_acc], (p_ph >> prev_acc) & 1, a.err, abort_flag))
-                        break;
-                    p_ph ^= 1u << prev_acc;
-                    tc::tc_fence_after();
-                    const uint32_t va = tc::smem_u32(sV + prev_kvb * kKBytes);
-#pragma unroll
-                    for (int ks = 0; ks < BLOCK / 16; ++ks) {
-                        const uint64_t bd = tc::sdesc_sw128(va + ks * 2048, BLOCK * 128, 1024);
-                        tc::mma_ts(tmem + prev_acc * kAccCols + BLOCK,
-                                   tmem + prev_acc * kAccCols + ks * 8, bd, idesc_o, ks > 0);
-                    }
-                    tc::mma_commit(&o_full[prev_acc]);
-                    if (list != prev_list) tc::mma_commit(&kv_empty[prev_kvb]);
-                }
-                if (!have) break;
-                prev_acc = i & 1;
-                prev_kvb = kvb;
-                prev_list = list;
-            }
-        }
-    } else {
-        // ------------------------------------------------ softmax + epilogue (two groups)
-        const int grp = (warp - 2) / 4;
+    } else if (wg == 1 || wg == 2) {
+        tc::regs_inc<kRegsSoftmax>();
+        // ------------------------------------------------ softmax (two groups)
+        // Group g takes tiles g, g + 2, ...; S/P buffer t % 3.  Row maximum,
+        // P = 2^((s - m) * scale * log2 e) on the special-function unit packed
+        // to bf16 into TMEM for the PV product, and m and the fp32 row sum l
+        // into the buffer's last two columns for the epilogue.
+        const int grp = wg - 1;
         const int quad = warp % 4;
         const int row = quad * 32 + lane;
         const int tt = row / a.R, h = row % a.R;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const uint32_t tS = tmem + grp * kAccCols + lane_off;
-        const uint32_t tO = tS + BLOCK;
-        int ph = 0;
-        int4 nd = load_tile(a, grp, total);
-        int nent = tt < nd.y ? a.entries[nd.z + tt] : 0;
+        // records of this group's next two tiles in flight
+        int2 nh = load_head(a, grp, total), nh2 = load_head(a, grp + 2, total);
+        int nent = load_ent(a, grp, total, tt), nent2 = load_ent(a, grp + 2, total, tt);
         for (int i = grp;; i += 2) {
-            const int4 d = nd;
+            const int2 d = nh;
             const int ent = nent;
-            if (d.x < 0 || *abort_flag) break;
-            nd = load_tile(a, i + 2, total);
-            nent = tt < nd.y ? a.entries[nd.z + tt] : 0;
+            if (d.x < 0) break;
+            nh = nh2;
+            nent = nent2;
+            nh2 = load_head(a, i + 4, total);
+            nent2 = load_ent(a, i + 4, total, tt);
             const int list = d.x;
-            const int n = list % a.NB, g = (list / a.NB) % a.G;
+            const int n = list % a.NB;
             const bool valid = tt < d.y;
-            const int t = (int)((a.r0 + (ent >> 8)) % a.T);
-            const int64_t p = (int64_t)a.S - a.T + t;
-            const int64_t j_base = (int64_t)n * BLOCK;
-            if (!tc::mbar_wait(&s_full[grp], ph, a.err, abort_flag)) break;
+            const int rl = ent >> 8;                           // row within the chunk
+            const int p = a.S - a.T + (int)((a.r0 + rl) % a.T);   // query position
+            const int j_base = n * BLOCK;
+            const int bsel = i % kQBuf;
+            const uint32_t tS = tmem + bsel * kSCols + lane_off;
+            if (!tc::mbar_wait(&s_full[bsel], (i / kQBuf) & 1, a.err, abort_flag)) break;
             tc::tc_fence_after();
-            // Row maximum over the causal keys of the block (one TMEM read).
             const bool masked = valid && (j_base + BLOCK - 1 > p);
-            uint32_t v[BLOCK];
-#pragma unroll
-            for (int c0 = 0; c0 < BLOCK; c0 += 32)
-                tc::tmem_ld32(tS + c0, *(uint32_t(*)[32])(v + c0));
-            tc::tmem_ld_wait();
+            // S is read from TMEM twice, 64 columns at a time (a TMEM read is
+            // cheap; holding a whole 128-column row would cost 64 registers).
+            // Causal mask (only in a token's own block): keys past the query
+            // position read as -inf.
+            // Pass 1: row maximum.
             float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-            if (!masked) {
 #pragma unroll
-                for (int c = 0; c < BLOCK; c += 4) {
+            for (int h0 = 0; h0 < BLOCK; h0 += 64) {
+                uint32_t v[64];
+                tc::tmem_ld32(tS + h0, *(uint32_t(*)[32])(v));
+                tc::tmem_ld32(tS + h0 + 32, *(uint32_t(*)[32])(v + 32));
+                tc::tmem_ld_wait();
+                if (masked) {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (j_base + h0 + c > p) v[c] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
                     m0 = fmaxf(m0, __uint_as_float(v[c]));
                     m1 = fmaxf(m1, __uint_as_float(v[c + 1]));
                     m2 = fmaxf(m2, __uint_as_float(v[c + 2]));
                     m3 = fmaxf(m3, __uint_as_float(v[c + 3]));
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < BLOCK; ++c)
-                    if (j_base + c <= p) m0 = fmaxf(m0, __uint_as_float(v[c]));
             }
             float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
             if (!valid) m = 0.f;
             const float mb = m * a.scale_log2;
-            // P = 2^((s - m) * scale * log2 e) in three sweeps so that the 2^x
-            // instructions are independent: exponents in fp32 packed as half
-            // pairs (the S registers die as they are consumed), 2^x on the
-            // pairs (P is rounded to bf16 for the MMA, so a half-precision 2^x
-            // is exact enough), then the fp32 row sum and the bf16 packing in
-            // place.  P (bf16 pairs) goes to the S columns already read.
-            uint32_t pk[BLOCK / 2];
-#pragma unroll
-            for (int c = 0; c < BLOCK; c += 2) {
-                float x0 = fmaf(__uint_as_float(v[c]), a.scale_log2, -mb);
-                float x1 = fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb);
-                if (masked) {
-                    if (j_base + c > p) x0 = -INFINITY;
-                    if (j_base + c + 1 > p) x1 = -INFINITY;
-                }
-                __half2 xh = __floats2half2_rn(x0, x1);
-                pk[c / 2] = *(uint32_t *)&xh;
-            }
-#pragma unroll
-            for (int c = 0; c < BLOCK / 2; ++c) pk[c] = tc::ex2_approx_h2(pk[c]);
+            // Pass 2: 2^x, packed to bf16 pairs and written over the S columns
+            // already read, with four partial row sums.  Rows past the tile's
+            // tokens hold no query and are never stored.
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-            for (int c = 0; c < BLOCK / 2; c += 2) {
-                const float2 e0 = __half22float2(*(const __half2 *)&pk[c]);
-                const float2 e1 = __half22float2(*(const __half2 *)&pk[c + 1]);
-                l0 += e0.x; l1 += e0.y; l2 += e1.x; l3 += e1.y;
-                __nv_bfloat162 b0 = __floats2bfloat162_rn(e0.x, e0.y);
-                __nv_bfloat162 b1 = __floats2bfloat162_rn(e1.x, e1.y);
-                pk[c] = *(uint32_t *)&b0;
-                pk[c + 1] = *(uint32_t *)&b1;
-            }
+            for (int h0 = 0; h0 < BLOCK; h0 += 64) {
+                uint32_t v[64];
+                tc::tmem_ld32(tS + h0, *(uint32_t(*)[32])(v));
+                tc::tmem_ld32(tS + h0 + 32, *(uint32_t(*)[32])(v + 32));
+                tc::tmem_ld_wait();
+                if (masked) {
 #pragma unroll
-            for (int c = 0; c < BLOCK / 2; c += 32)
-                tc::tmem_st32(tS + c, *(const uint32_t(*)[32])(pk + c));
+                    for (int c = 0; c < 64; ++c)
+                        if (j_base + h0 + c > p) v[c] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c += 4) {
+                    const float e0 = tc::ex2_approx(fmaf(__uint_as_float(v[c]), a.scale_log2, -mb));
+                    const float e1 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb));
+                    const float e2 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 2]), a.scale_log2, -mb));
+                    const float e3 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 3]), a.scale_log2, -mb));
+                    l0 += e0; l1 += e1; l2 += e2; l3 += e3;
+                    __nv_bfloat162 b0 = __floats2bfloat162_rn(e0, e1);
+                    __nv_bfloat162 b1 = __floats2bfloat162_rn(e2, e3);
+                    v[c / 2] = *(uint32_t *)&b0;
+                    v[c / 2 + 1] = *(uint32_t *)&b1;
+                }
+                tc::tmem_st32(tS + h0 / 2, *(const uint32_t(*)[32])(v));
+            }
             const float l = (l0 + l1) + (l2 + l3);
+            tc::tmem_st1(tS + (kSCols - 2), __float_as_uint(m));
+            tc::tmem_st1(tS + (kSCols - 1), __float_as_uint(l));
             tc::tmem_st_wait();
             tc::tc_fence_before();
-            tc::mbar_arrive(&p_full[grp]);
-            if (!tc::mbar_wait(&o_full[grp], ph, a.err, abort_flag)) break;
-            tc::tc_fence_after();
-            const int slot = ent & 255;
+            tc::mbar_arrive(&p_full[bsel]);
+        }
+    } else {
+        tc::regs_inc<kRegsEpilogue>();
+        // ------------------------------------------------ epilogue
+        // Every tile in order: wait for its PV product, read the O row, m and l
+        // from TMEM (which frees the accumulator for the next PV and, with PV
+        // done, the tile's S/P buffer), then O / l to fp16, stored in 32-row
+        // blocked chunk planes (partial_chunk) so that the rows of a warp store
+        // to consecutive addresses, and LSE = m * scale + ln l.
+        const int quad = warp % 4;
+        const int row = quad * 32 + lane;
+        const int tt = row / a.R, h = row % a.R;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const uint32_t tO = tmem + kOCol + lane_off;
+        int2 nh = load_head(a, 0, total), nh2 = load_head(a, 1, total);
+        int nent = load_ent(a, 0, total, tt), nent2 = load_ent(a, 1, total, tt);
+        for (int i = 0;; ++i) {
+            const int2 d = nh;
+            const int ent = nent;
+            if (d.x < 0) break;
+            nh = nh2;
+            nent = nent2;
+            nh2 = load_head(a, i + 2, total);
+            nent2 = load_ent(a, i + 2, total, tt);
+            const bool valid = tt < d.y;
+            const int g = (d.x / a.NB) % a.G, slot = ent & 255;
             const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
-            const float inv_l = 1.f / l;
-            // partial O in 32-row blocked chunk planes (partial_chunk): the rows
-            // of a warp store to consecutive addresses
             uint4 *dst = (uint4 *)a.part_o + partial_chunk(prow, 0, D);
-            // O row to fp16 pairs in place; TMEM is released as soon as the row
-            // is in registers, before the stores.
+            if (!tc::mbar_wait(o_full, i & 1, a.err, abort_flag)) break;
+            tc::tc_fence_after();
             uint32_t ov[D];
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) tc::tmem_ld32(tO + c0, *(uint32_t(*)[32])(ov + c0));
+            const int bsel = i % kQBuf;
+            const uint32_t tS = tmem + bsel * kSCols + lane_off;
+            const float m = __uint_as_float(tc::tmem_ld1(tS + (kSCols - 2)));
+            const float l = __uint_as_float(tc::tmem_ld1(tS + (kSCols - 1)));
             tc::tmem_ld_wait();
             tc::tc_fence_before();
-            tc::mbar_arrive(&acc_empty[grp]);               // accumulators free for tile i + 2
+            tc::mbar_arrive(o_empty);
+            tc::mbar_arrive(&s_free[bsel]);
+            const float inv = 1.f / l;
 #pragma unroll
             for (int c = 0; c < D; c += 2) {
-                __half2 hv = __floats2half2_rn(__uint_as_float(ov[c]) * inv_l,
-                                               __uint_as_float(ov[c + 1]) * inv_l);
+                __half2 hv = __floats2half2_rn(__uint_as_float(ov[c]) * inv,
+                                               __uint_as_float(ov[c + 1]) * inv);
                 ov[c / 2] = *(uint32_t *)&hv;
             }
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < D / 2; c += 4)
                     dst[(c / 4) * 32] = make_uint4(ov[c], ov[c + 1], ov[c + 2], ov[c + 3]);
-            }
-            ph ^= 1;
-            if (valid) {
                 a.part_lse[prow] = m * a.scale + logf(l);
             }
         }
@@ -625,7 +727,7 @@ struct Plan {
     int64_t rows_per_chunk;
     int tpt;
     int64_t L;
-    size_t counts, cursor, offs, toffs, entries, tiles, part_o, part_lse, total;
+    size_t counts, cursor, toffs, recs, part_o, part_lse, total;
 };
 
 Plan make_plan(const Shape &s) {
@@ -641,10 +743,9 @@ Plan make_plan(const Shape &s) {
     size_t o = 0;
     p.counts = o;   o += al(sizeof(int) * p.L);
     p.cursor = o;   o += al(sizeof(int) * p.L);
-    p.offs = o;     o += al(sizeof(int) * (p.L + 1));
     p.toffs = o;    o += al(sizeof(int) * (p.L + 1));
-    p.entries = o;  o += al(sizeof(int) * slots);
-    p.tiles = o;    o += al(sizeof(int4) * (slots + p.L));
+    // at most ceil(slots / tpt) full tiles plus one partial tile per list
+    p.recs = o;     o += al(sizeof(int) * rec_ints(p.tpt) * ((slots + p.tpt - 1) / p.tpt + p.L));
     p.part_o = o;   o += al(sizeof(__half) * ((slots * s.R + 31) / 32 * 32) * s.d);
     p.part_lse = o; o += al(sizeof(float) * slots * s.R);
     p.total = o;
@@ -668,12 +769,11 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
     const uint32_t qbox[3] = {64, (uint32_t)s.R, 1};
     if (!make_tmap_bf16(&tq, Q, 3, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
     int *counts = (int *)(ws + pl.counts), *cursor = (int *)(ws + pl.cursor);
-    int *offs = (int *)(ws + pl.offs), *toffs = (int *)(ws + pl.toffs);
-    int *entries = (int *)(ws + pl.entries);
-    int4 *tiles = (int4 *)(ws + pl.tiles);
+    int *toffs = (int *)(ws + pl.toffs);
+    int *recs = (int *)(ws + pl.recs);
     __half *part_o = (__half *)(ws + pl.part_o);
     float *part_lse = (float *)(ws + pl.part_lse);
-    const size_t smem = 1024 + 2 * (size_t)kRows * D * 2 + 4 * (size_t)BLOCK * D * 2 + 256;
+    const size_t smem = 1024 + 3 * (size_t)kRows * D * 2 + 4 * (size_t)BLOCK * D * 2 + 256;
     auto kern = attn_tc_kernel<D, BLOCK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -683,20 +783,19 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
     const int L = (int)pl.L;
     for (int64_t r0 = 0; r0 < s.rows(); r0 += pl.rows_per_chunk) {
         const int64_t rc = std::min<int64_t>(pl.rows_per_chunk, s.rows() - r0);
-        e = cudaMemsetAsync(counts, 0, pl.offs - pl.counts, st);   // counts and cursor
+        e = cudaMemsetAsync(counts, 0, pl.toffs - pl.counts, st);   // counts and cursor
         if (e != cudaSuccess) return e;
         const int64_t nrow = rc * s.G;                      // one warp each
         const unsigned g1 = (unsigned)((nrow * 32 + 255) / 256);
         csr_count_kernel<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB,
                                              s.block, s.topk);
-        csr_scan_kernel<<<1, 1024, 0, st>>>(counts, offs, toffs, L, pl.tpt);
-        csr_fill_kernel<<<g1, 256, 0, st>>>(ids, offs, cursor, entries, r0, rc, s.T, s.S, s.G,
-                                            s.NB, s.block, s.topk);
-        csr_tiles_kernel<<<(L + 255) / 256, 256, 0, st>>>(counts, offs, toffs, tiles, L, pl.tpt);
+        csr_scan_kernel<<<1, 1024, 0, st>>>(counts, toffs, L, pl.tpt);
+        csr_fill_kernel<<<g1, 256, 0, st>>>(ids, toffs, cursor, recs, r0, rc, s.T, s.S, s.G,
+                                            s.NB, s.block, s.topk, pl.tpt);
+        csr_tiles_kernel<<<(L + 255) / 256, 256, 0, st>>>(counts, toffs, recs, L, pl.tpt);
         AttnArgs a{};
         a.Q = (const __nv_bfloat16 *)Q;
-        a.entries = entries;
-        a.tiles = tiles;
+        a.recs = recs;
         a.n_tiles = toffs + L;
         a.part_o = part_o; a.part_lse = part_lse; a.err = err; a.r0 = r0;
         a.n_prows = rc * s.G * s.topk * s.R;
