@@ -187,6 +187,7 @@ struct AttnArgs {
     uint32_t *err;
     int64_t r0;
     int T, S, Hq, G, R, NB, topk, tpt;
+    int q_box4;                 // Q tensor map is 4-D: one box = both channel atoms
     float scale, scale_log2;
 };
 
@@ -229,29 +230,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     constexpr int kQBuf = 3;                      // Q tiles in flight = S/P buffers
     constexpr uint32_t kQBytes = kRows * D * 2;
     constexpr uint32_t kKBytes = BLOCK * D * 2;
+    // A Q tile is 16 groups of 8 rows; a group holds its kAtoms 64-channel
+    // swizzle atoms (8 rows x 128 bytes each) back to back, so 8 heads of a
+    // token are one contiguous 2-KB TMA box.
+    constexpr uint32_t kGroupBytes = 8 * D * 2;
     constexpr uint32_t kSCols = 128, kOCol = 384;
     static_assert(BLOCK <= (int)kSCols && D <= 128, "TMEM budget");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = smem;                           // [3][kAtoms][128][64]
+    uint8_t *sQ = smem;                           // [3][16 row groups][kAtoms][8][64]
     uint8_t *sK = sQ + kQBuf * kQBytes;           // [2][kAtoms][BLOCK][64]
     uint8_t *sV = sK + 2 * kKBytes;               // [2][kAtoms][BLOCK][64]
     uint64_t *bar = (uint64_t *)(sV + 2 * kKBytes);
-    uint64_t *q_full = bar, *q_empty = bar + 3;   // [3] each
-    uint64_t *kv_full = bar + 6, *kv_empty = bar + 8;        // [2] each
-    uint64_t *s_full = bar + 10, *p_full = bar + 13, *s_free = bar + 16;   // [3] each
-    uint64_t *o_full = bar + 19, *o_empty = bar + 20;
-    uint32_t *tmem_slot = (uint32_t *)(bar + 21);
+    // A Q buffer is free again when the S product that read it completes
+    // (s_full); an S/P buffer when the epilogue has read m and l, after PV.
+    uint64_t *q_full = bar;                       // [3]
+    uint64_t *kv_full = bar + 3, *kv_empty = bar + 5;        // [2] each
+    uint64_t *s_full = bar + 7, *p_full = bar + 10, *s_free = bar + 13;   // [3] each
+    uint64_t *o_full = bar + 16, *o_empty = bar + 17;
+    uint32_t *tmem_slot = (uint32_t *)(bar + 18);
     volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQBuf; ++i) {
             tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 96);   // TMA: one; cp.async: per thread
-            tc::mbar_init(&q_empty[i], 1);
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_full[i], 128);
-            tc::mbar_init(&s_free[i], 1 + 128);    // PV commit + epilogue threads
+            tc::mbar_init(&s_free[i], 128);        // epilogue threads, after PV
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&kv_full[i], 1);
@@ -285,8 +291,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // copies and loads run up to three tiles ahead.
             const int gw = warp == 0 ? 0 : warp - 1;   // gather warp 0..2
             const int cc = lane % 16;
-            const uint32_t q_swz = (uint32_t)(cc / 8) * (kRows * 128);
+            const uint32_t q_swz = (uint32_t)(cc / 8) * 1024;
             const int lr = __ffs(a.R) - 1;             // log2 R
+            // A token's Q rows are read once per kept block: keep them in L2
+            // ahead of the partials streaming out.
+            const uint64_t q_pol = tc::policy_evict_last();
             int kvb = -1, cur_list = -1;
             uint32_t kv_ph = 0;                        // per K/V buffer phase bits
             // Records of the next two tiles in flight: lane l holds entries
@@ -331,20 +340,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     kv_ph ^= 1u << kvb;
                 }
                 const int qb = i % kQBuf;
-                if (!tc::mbar_wait(&q_empty[qb], ((i / kQBuf) & 1) ^ 1, a.err, abort_flag)) break;
+                if (!tc::mbar_wait(&s_full[qb], ((i / kQBuf) & 1) ^ 1, a.err, abort_flag)) break;
                 if (a.R >= 8) {
-                    // 8 or more heads per token: one TMA box per token and 64-channel
-                    // atom (R * 128 bytes, whole swizzle atoms); lane k < count holds
-                    // token k's entry.
+                    // 8 or more heads per token: the token's heads in groups of 8
+                    // rows, one TMA box per group holding both 64-channel atoms
+                    // (or one box per atom); lane k < count holds token k's entry.
                     if (lane == 0)
                         tc::mbar_expect_tx(&q_full[qb], (uint32_t)count * a.R * D * 2);
                     __syncwarp();
                     if (lane < count) {
                         const int grow = (int)(a.r0 + (e[0] >> 8));
+                        for (int j = 0; j < a.R / 8; ++j) {
+                            uint8_t *grp8 = sQ + qb * kQBytes + (lane * (a.R / 8) + j) * kGroupBytes;
+                            if (a.q_box4) {
+                                tc::tma_load_4d_hint(grp8, &tm_q, &q_full[qb], 0, g * a.R + j * 8, 0,
+                                                     grow, q_pol);
+                            } else {
 #pragma unroll
-                        for (int at = 0; at < kAtoms; ++at)
-                            tc::tma_load_3d(sQ + qb * kQBytes + at * kRows * 128 + lane * a.R * 128,
-                                            &tm_q, &q_full[qb], at * 64, g * a.R, grow);
+                                for (int at = 0; at < kAtoms; ++at)
+                                    tc::tma_load_3d_hint(grp8 + at * 1024, &tm_q, &q_full[qb],
+                                                         at * 64, g * a.R + j * 8, grow, q_pol);
+                            }
+                        }
                     }
                     continue;
                 }
@@ -363,9 +380,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (r < rows) {
                         const __nv_bfloat16 *src =
                             a.Q + ((a.r0 + (ent >> 8)) * a.Hq + head0 + hh) * D + cc * 8;
-                        const uint32_t sa = dst + r * 128 + (((cc % 8) ^ (r % 8)) * 16);
-                        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa),
-                                     "l"(src)
+                        const uint32_t sa = dst + (r / 8) * kGroupBytes + (r % 8) * 128 +
+                                            (((cc % 8) ^ (r % 8)) * 16);
+                        asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;"
+                                     ::"r"(sa), "l"(src), "l"(q_pol)
                                      : "memory");
                     }
                 }
@@ -392,7 +410,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 int next_list = load_head(a, 0, total).x, next_list2 = load_head(a, 1, total).x;
                 for (int t = 0;; ++t) {
                     const int list = next_list;
-                    const bool have = list >= 0 && !*abort_flag;
+                    const bool have = list >= 0;
                     if (have) {
                         next_list = next_list2;
                         next_list2 = load_head(a, t + 2, total).x;
@@ -414,7 +432,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             tc::mma_ts(tmem + kOCol, tmem + bp * kSCols + ks * 8, bd, idesc_o, ks > 0);
                         }
                         tc::mma_commit(o_full);
-                        tc::mma_commit(&s_free[bp]);
                         if (list1 != list2) tc::mma_commit(&kv_empty[kvb2]);
                         return true;
                     };
@@ -430,7 +447,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             return false;
                         if (!tc::mbar_wait(&q_full[bs], (t / kQBuf) & 1, a.err, abort_flag))
                             return false;
-                        if (!tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
+                        if (new_list &&
+                            !tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
                             return false;
                         tc::tc_fence_after();
                         const uint32_t qa = tc::smem_u32(sQ + bs * kQBytes);
@@ -438,12 +456,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     #pragma unroll
                         for (int ks = 0; ks < D / 16; ++ks) {
                             const uint64_t ad =
-                                tc::sdesc_sw128(qa + (ks / 4) * kRows * 128 + (ks % 4) * 32, 16, 1024);
+                                tc::sdesc_sw128(qa + (ks / 4) * 1024 + (ks % 4) * 32, 16, kGroupBytes);
                             const uint64_t bd =
                                 tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
                             tc::mma_ss(tmem + bs * kSCols, ad, bd, idesc_s, ks > 0);
                         }
-                        tc::mma_commit(&q_empty[bs]);
                         tc::mma_commit(&s_full[bs]);
                         return true;
                     };
@@ -570,6 +587,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int tt = row / a.R, h = row % a.R;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t tO = tmem + kOCol + lane_off;
+        // partials are read back only by the combine: first out of L2
+        const uint64_t st_pol = tc::policy_evict_first();
         int2 nh = load_head(a, 0, total), nh2 = load_head(a, 1, total);
         int nent = load_ent(a, 0, total, tt), nent2 = load_ent(a, 1, total, tt);
         for (int i = 0;; ++i) {
@@ -607,8 +626,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (valid) {
 #pragma unroll
                 for (int c = 0; c < D / 2; c += 4)
-                    dst[(c / 4) * 32] = make_uint4(ov[c], ov[c + 1], ov[c + 2], ov[c + 3]);
-                a.part_lse[prow] = m * a.scale + logf(l);
+                    tc::st_global_v4_hint(dst + (c / 4) * 32,
+                                          make_uint4(ov[c], ov[c + 1], ov[c + 2], ov[c + 3]), st_pol);
+                tc::st_global_f32_hint(a.part_lse + prow, m * a.scale + logf(l), st_pol);
             }
         }
     }
@@ -763,11 +783,23 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
     const uint32_t box[3] = {64, 1, (uint32_t)BLOCK};
     if (!make_tmap_bf16(&tk, K, 3, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16(&tv, V, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    // Q as [B*T, Hq, d]: one box = the R heads of one token (R rows of 64 channels)
-    const uint64_t qdims[3] = {(uint64_t)s.d, (uint64_t)s.Hq, (uint64_t)s.B * s.T};
-    const uint64_t qstrides[2] = {(uint64_t)s.d * 2, (uint64_t)s.Hq * s.d * 2};
-    const uint32_t qbox[3] = {64, (uint32_t)s.R, 1};
-    if (!make_tmap_bf16(&tq, Q, 3, qdims, qstrides, qbox)) return cudaErrorInvalidValue;
+    // Q as [B*T][atom][Hq][64] (atoms of 64 channels, stride 128 bytes): one box =
+    // 8 heads of one token, both atoms, atom-major in shared memory.  Where the
+    // encoder rejects that stride order, Q as [B*T][Hq][d] with one box per atom.
+    int q_box4 = 1;
+    {
+        const uint64_t qdims[4] = {64, (uint64_t)s.Hq, (uint64_t)s.d / 64, (uint64_t)s.B * s.T};
+        const uint64_t qstrides[3] = {(uint64_t)s.d * 2, 128, (uint64_t)s.Hq * s.d * 2};
+        const uint32_t qbox[4] = {64, 8, (uint32_t)s.d / 64, 1};
+        if (!make_tmap_bf16(&tq, Q, 4, qdims, qstrides, qbox)) {
+            q_box4 = 0;
+            const uint64_t qdims3[3] = {(uint64_t)s.d, (uint64_t)s.Hq, (uint64_t)s.B * s.T};
+            const uint64_t qstrides3[2] = {(uint64_t)s.d * 2, (uint64_t)s.Hq * s.d * 2};
+            const uint32_t qbox3[3] = {64, 8, 1};
+            if (s.R >= 8 && !make_tmap_bf16(&tq, Q, 3, qdims3, qstrides3, qbox3))
+                return cudaErrorInvalidValue;
+        }
+    }
     int *counts = (int *)(ws + pl.counts), *cursor = (int *)(ws + pl.cursor);
     int *toffs = (int *)(ws + pl.toffs);
     int *recs = (int *)(ws + pl.recs);
@@ -801,6 +833,7 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         a.n_prows = rc * s.G * s.topk * s.R;
         a.T = s.T; a.S = s.S; a.Hq = s.Hq; a.G = s.G; a.R = s.R; a.NB = s.NB; a.topk = s.topk;
         a.tpt = pl.tpt;
+        a.q_box4 = q_box4;
         a.scale = s.scale;
         a.scale_log2 = s.scale * kLog2e;
         kern<<<sms, kThreads, smem, st>>>(tq, tk, tv, a);
