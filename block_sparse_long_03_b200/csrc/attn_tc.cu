@@ -208,8 +208,10 @@ __device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int
 }
 
 // Warp roles (four warpgroups, 512 threads):
-//   warpgroup 0     warp 1 issues the MMAs; warps 0, 2 and 3 gather the Q
-//                   rows (cp.async) and warp 0 loads the K/V blocks (TMA);
+//   warpgroup 0     warp 0 loads the K/V blocks and Q rows (TMA; for fewer
+//                   than 8 heads per token, warps 0 and 3 gather Q with
+//                   cp.async), warp 1 issues the S products, warp 2 the PV
+//                   products;
 //   warpgroups 1-2  softmax, tiles 0, 2, 4, ... and 1, 3, 5, ...;
 //   warpgroup 3     epilogue of every tile: O from TMEM to an fp16 partial.
 // TMEM: three S/P buffers (S: BLOCK fp32 columns; P: bf16 pairs in the first
@@ -254,7 +256,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQBuf; ++i) {
-            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 96);   // TMA: one; cp.async: per thread
+            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 64);   // TMA: one; cp.async: per thread
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_full[i], 128);
             tc::mbar_init(&s_free[i], 128);        // epilogue threads, after PV
@@ -279,17 +281,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // Each role sets its warpgroup's register budget first.
     if (wg == 0) {
         tc::regs_dec<kRegsLoad>();
-        if (warp == 0 || (warp >= 2 && a.R < 8)) {
+        if (warp == 0 || (warp == 3 && a.R < 8)) {
             // ------------------------------------------------ loads
             // K/V blocks by TMA (warp 0, lane 0) whenever the list changes, and
-            // the tile's Q rows gathered by warps 0, 2 and 3 with 16-byte
+            // the tile's Q rows gathered by warps 0 and 3 with 16-byte
             // cp.async copies straight into the 128-byte-swizzled K-major
             // layout the MMA reads.  Each warp instruction copies two whole
             // 256-byte rows; lane l always copies 16-byte chunk l % 16.  A
             // thread's copies arrive on q_full when they complete
             // (cp.async.mbarrier.arrive.noinc), so no warp waits for its own
             // copies and loads run up to three tiles ahead.
-            const int gw = warp == 0 ? 0 : warp - 1;   // gather warp 0..2
+            const int gw = warp == 0 ? 0 : 1;          // gather warp 0..1
             const int cc = lane % 16;
             const uint32_t q_swz = (uint32_t)(cc / 8) * 1024;
             const int lr = __ffs(a.R) - 1;             // log2 R
@@ -371,7 +373,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // row pair q = rows 2q, 2q + 1 (lanes 0-15 / 16-31); both rows'
                 // tokens sit in the same 32-token block, so one register holds
                 // their entries and a shuffle hands each lane its token's entry
-                for (int q = gw; 2 * q < rows; q += 3) {
+                for (int q = gw; 2 * q < rows; q += 2) {
                     const int r = 2 * q + lane / 16;
                     const int tk = r >> lr, hh = r & (a.R - 1);
                     const int kk = (2 * q) >> (lr + 5);
@@ -392,88 +394,76 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // the last copies must land before the CTA can retire
             asm volatile("cp.async.wait_all;" ::: "memory");
-        } else if (warp == 1) {
-            // ------------------------------------------------ MMA issuer
-            // Iteration t issues S(t) = Q K^T and PV(t - 2): O = P V.  S(t) goes
-            // first, so the S of a softmax group's next tile is already computed
-            // when the group finishes its current one.  The one exception: when
-            // S(t) starts a list whose K/V buffer is released by PV(t - 2) (tile
-            // t - 2 was the last of its list), PV(t - 2) must be issued first or
-            // the load of that buffer would wait on an MMA never issued.
-            if (lane == 0) {
-                constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
-                constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
-                int kvb = -1, cur_list = -1;
-                uint32_t kv_ph = 0;
-                // K/V buffer and list of tiles t - 1 and t - 2 (-1: none)
-                int kvb1 = -1, kvb2 = -1, list1 = -1, list2 = -1;
-                int next_list = load_head(a, 0, total).x, next_list2 = load_head(a, 1, total).x;
-                for (int t = 0;; ++t) {
-                    const int list = next_list;
-                    const bool have = list >= 0;
-                    if (have) {
-                        next_list = next_list2;
-                        next_list2 = load_head(a, t + 2, total).x;
-                    }
-                    const bool new_list = have && list != cur_list;
-                    const bool pv_first = !have || (new_list && list2 >= 0 && list1 != list2);
-                    auto issue_pv = [&]() -> bool {
-                        if (kvb2 < 0) return true;       // no tile t - 2
-                        const int tp = t - 2, bp = tp % kQBuf;
-                        if (!tc::mbar_wait(&p_full[bp], (tp / kQBuf) & 1, a.err, abort_flag))
-                            return false;
-                        if (tp >= 1 && !tc::mbar_wait(o_empty, (tp - 1) & 1, a.err, abort_flag))
-                            return false;
-                        tc::tc_fence_after();
-                        const uint32_t va = tc::smem_u32(sV + kvb2 * kKBytes);
-    #pragma unroll
-                        for (int ks = 0; ks < BLOCK / 16; ++ks) {
-                            const uint64_t bd = tc::sdesc_sw128(va + ks * 2048, BLOCK * 128, 1024);
-                            tc::mma_ts(tmem + kOCol, tmem + bp * kSCols + ks * 8, bd, idesc_o, ks > 0);
-                        }
-                        tc::mma_commit(o_full);
-                        if (list1 != list2) tc::mma_commit(&kv_empty[kvb2]);
-                        return true;
-                    };
-                    auto issue_s = [&]() -> bool {
-                        if (new_list) {
-                            kvb = (kvb + 1) & 1;
-                            cur_list = list;
-                            kv_ph ^= 1u << kvb;
-                        }
-                        const int bs = t % kQBuf;
-                        if (t >= kQBuf &&
-                            !tc::mbar_wait(&s_free[bs], ((t / kQBuf) - 1) & 1, a.err, abort_flag))
-                            return false;
-                        if (!tc::mbar_wait(&q_full[bs], (t / kQBuf) & 1, a.err, abort_flag))
-                            return false;
-                        if (new_list &&
-                            !tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
-                            return false;
-                        tc::tc_fence_after();
-                        const uint32_t qa = tc::smem_u32(sQ + bs * kQBytes);
-                        const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
-    #pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks) {
-                            const uint64_t ad =
-                                tc::sdesc_sw128(qa + (ks / 4) * 1024 + (ks % 4) * 32, 16, kGroupBytes);
-                            const uint64_t bd =
-                                tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
-                            tc::mma_ss(tmem + bs * kSCols, ad, bd, idesc_s, ks > 0);
-                        }
-                        tc::mma_commit(&s_full[bs]);
-                        return true;
-                    };
-                    bool ok = true;
-                    if (pv_first) ok = issue_pv();
-                    if (ok && have) ok = issue_s();
-                    if (ok && !pv_first) ok = issue_pv();
-                    if (!ok) break;
-                    // shift the (t - 1, t - 2) history
-                    kvb2 = kvb1; list2 = list1;
-                    kvb1 = have ? kvb : -1; list1 = have ? list : -1;
-                    if (!have && kvb2 < 0) break;      // every PV issued
+        } else if (warp == 1 && lane == 0) {
+            // ------------------------------------------------ S issuer: S(t) = Q K^T
+            // into S/P buffer t % 3, once Q(t) has landed, the buffer is free
+            // (the epilogue has read tile t - 3's row sums, after its PV) and,
+            // at a list change, the list's K/V block has landed.
+            constexpr uint32_t idesc_s = tc::idesc_bf16(kRows, BLOCK, 0, 0);
+            int kvb = -1, cur_list = -1;
+            uint32_t kv_ph = 0;
+            int next_list = load_head(a, 0, total).x, next_list2 = load_head(a, 1, total).x;
+            for (int t = 0;; ++t) {
+                const int list = next_list;
+                if (list < 0) break;
+                next_list = next_list2;
+                next_list2 = load_head(a, t + 2, total).x;
+                const bool new_list = list != cur_list;
+                if (new_list) {
+                    kvb = (kvb + 1) & 1;
+                    cur_list = list;
+                    kv_ph ^= 1u << kvb;
                 }
+                const int bs = t % kQBuf;
+                if (t >= kQBuf &&
+                    !tc::mbar_wait(&s_free[bs], ((t / kQBuf) - 1) & 1, a.err, abort_flag))
+                    break;
+                if (!tc::mbar_wait(&q_full[bs], (t / kQBuf) & 1, a.err, abort_flag)) break;
+                if (new_list &&
+                    !tc::mbar_wait(&kv_full[kvb], ((kv_ph >> kvb) & 1) ^ 1, a.err, abort_flag))
+                    break;
+                tc::tc_fence_after();
+                const uint32_t qa = tc::smem_u32(sQ + bs * kQBytes);
+                const uint32_t ka = tc::smem_u32(sK + kvb * kKBytes);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t ad =
+                        tc::sdesc_sw128(qa + (ks / 4) * 1024 + (ks % 4) * 32, 16, kGroupBytes);
+                    const uint64_t bd =
+                        tc::sdesc_sw128(ka + (ks / 4) * BLOCK * 128 + (ks % 4) * 32, 16, 1024);
+                    tc::mma_ss(tmem + bs * kSCols, ad, bd, idesc_s, ks > 0);
+                }
+                tc::mma_commit(&s_full[bs]);
+            }
+        } else if (warp == 2 && lane == 0) {
+            // ------------------------------------------------ PV issuer: O = P V
+            // once P(t) is in TMEM and the epilogue has read O(t - 1).  After a
+            // list's last tile its K/V buffer is released to the loads.  The two
+            // issuers are independent, so neither waits behind the other.
+            constexpr uint32_t idesc_o = tc::idesc_bf16(kRows, D, 0, 1);
+            int kvb = -1, cur_list = -1;
+            int next_list = load_head(a, 0, total).x, next_list2 = load_head(a, 1, total).x;
+            for (int t = 0;; ++t) {
+                const int list = next_list;
+                if (list < 0) break;
+                next_list = next_list2;
+                next_list2 = load_head(a, t + 2, total).x;
+                if (list != cur_list) {
+                    kvb = (kvb + 1) & 1;
+                    cur_list = list;
+                }
+                const int bp = t % kQBuf;
+                if (!tc::mbar_wait(&p_full[bp], (t / kQBuf) & 1, a.err, abort_flag)) break;
+                if (t >= 1 && !tc::mbar_wait(o_empty, (t - 1) & 1, a.err, abort_flag)) break;
+                tc::tc_fence_after();
+                const uint32_t va = tc::smem_u32(sV + kvb * kKBytes);
+#pragma unroll
+                for (int ks = 0; ks < BLOCK / 16; ++ks) {
+                    const uint64_t bd = tc::sdesc_sw128(va + ks * 2048, BLOCK * 128, 1024);
+                    tc::mma_ts(tmem + kOCol, tmem + bp * kSCols + ks * 8, bd, idesc_o, ks > 0);
+                }
+                tc::mma_commit(o_full);
+                if (next_list != list) tc::mma_commit(&kv_empty[kvb]);
             }
         }
     } else if (wg == 1 || wg == 2) {
@@ -485,8 +475,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // into the buffer's last two columns for the epilogue.
         const int grp = wg - 1;
         const int quad = warp % 4;
-        const int row = quad * 32 + lane;
-        const int tt = row / a.R, h = row % a.R;
+        const int tt = (quad * 32 + lane) / a.R;      // the row's token in the tile
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         // records of this group's next two tiles in flight
         int2 nh = load_head(a, grp, total), nh2 = load_head(a, grp + 2, total);
