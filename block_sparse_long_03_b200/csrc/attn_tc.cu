@@ -215,7 +215,7 @@ __device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int
 //   warpgroups 1-2  softmax, tiles 0, 2, 4, ... and 1, 3, 5, ...;
 //   warpgroup 3     epilogue of every tile: O from TMEM to an fp16 partial.
 // TMEM: three S/P buffers (S: BLOCK fp32 columns; P: bf16 pairs in the first
-// BLOCK/2 of them; the row max m and row sum l in the last two columns) at
+// BLOCK/2 of them; partial row, row max m and row sum l in the last three) at
 // columns 0, 128, 256 and one O accumulator at 384.  The epilogue divides O
 // by l, converts and stores it with the LSE, so no global store is issued by
 // the softmax warps; an S/P buffer is free again once PV has read P and the
@@ -471,11 +471,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ------------------------------------------------ softmax (two groups)
         // Group g takes tiles g, g + 2, ...; S/P buffer t % 3.  Row maximum,
         // P = 2^((s - m) * scale * log2 e) on the special-function unit packed
-        // to bf16 into TMEM for the PV product, and m and the fp32 row sum l
-        // into the buffer's last two columns for the epilogue.
+        // to bf16 into TMEM for the PV product, and the partial's row, m and
+        // the fp32 row sum l into the buffer's last columns for the epilogue.
         const int grp = wg - 1;
         const int quad = warp % 4;
         const int tt = (quad * 32 + lane) / a.R;      // the row's token in the tile
+        const int h = (quad * 32 + lane) % a.R;       // and its head in the group
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         // records of this group's next two tiles in flight
         int2 nh = load_head(a, grp, total), nh2 = load_head(a, grp + 2, total);
@@ -494,6 +495,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int rl = ent >> 8;                           // row within the chunk
             const int p = a.S - a.T + (int)((a.r0 + rl) % a.T);   // query position
             const int j_base = n * BLOCK;
+            // the partial's row in the chunk (-1: no query)
+            const int prow =
+                valid ? ((rl * a.G + (list / a.NB) % a.G) * a.topk + (ent & 255)) * a.R + h : -1;
             const int bsel = i % kQBuf;
             const uint32_t tS = tmem + bsel * kSCols + lane_off;
             if (!tc::mbar_wait(&s_full[bsel], (i / kQBuf) & 1, a.err, abort_flag)) break;
@@ -557,8 +561,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 tc::tmem_st32(tS + h0 / 2, *(const uint32_t(*)[32])(v));
             }
             const float l = (l0 + l1) + (l2 + l3);
-            tc::tmem_st1(tS + (kSCols - 2), __float_as_uint(m));
-            tc::tmem_st1(tS + (kSCols - 1), __float_as_uint(l));
+            // the partial's row, m and l for the epilogue
+            tc::tmem_st4(tS + (kSCols - 4), 0u, (uint32_t)prow, __float_as_uint(m),
+                         __float_as_uint(l));
             tc::tmem_st_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(&p_full[bsel]);
@@ -566,45 +571,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
         tc::regs_inc<kRegsEpilogue>();
         // ------------------------------------------------ epilogue
-        // Every tile in order: wait for its PV product, read the O row, m and l
-        // from TMEM (which frees the accumulator for the next PV and, with PV
-        // done, the tile's S/P buffer), then O / l to fp16, stored in 32-row
-        // blocked chunk planes (partial_chunk) so that the rows of a warp store
-        // to consecutive addresses, and LSE = m * scale + ln l.
+        // Every tile in order: wait for its PV product, read the O row and the
+        // softmax's partial row, m and l from TMEM (which frees the accumulator
+        // for the next PV and, with PV done, the tile's S/P buffer), then O / l
+        // to fp16, stored in 32-row blocked chunk planes (partial_chunk) so that
+        // the rows of a warp store to consecutive addresses, and
+        // LSE = m * scale + ln l.  No tile metadata is read from memory.
         const int quad = warp % 4;
-        const int row = quad * 32 + lane;
-        const int tt = row / a.R, h = row % a.R;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const uint32_t tO = tmem + kOCol + lane_off;
         // partials are read back only by the combine: first out of L2
         const uint64_t st_pol = tc::policy_evict_first();
-        int2 nh = load_head(a, 0, total), nh2 = load_head(a, 1, total);
-        int nent = load_ent(a, 0, total, tt), nent2 = load_ent(a, 1, total, tt);
-        for (int i = 0;; ++i) {
-            const int2 d = nh;
-            const int ent = nent;
-            if (d.x < 0) break;
-            nh = nh2;
-            nent = nent2;
-            nh2 = load_head(a, i + 2, total);
-            nent2 = load_ent(a, i + 2, total, tt);
-            const bool valid = tt < d.y;
-            const int g = (d.x / a.NB) % a.G, slot = ent & 255;
-            const int64_t prow = ((((int64_t)(ent >> 8)) * a.G + g) * a.topk + slot) * a.R + h;
-            uint4 *dst = (uint4 *)a.part_o + partial_chunk(prow, 0, D);
+        for (int i = 0; run_tile(i) < total; ++i) {
             if (!tc::mbar_wait(o_full, i & 1, a.err, abort_flag)) break;
             tc::tc_fence_after();
             uint32_t ov[D];
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) tc::tmem_ld32(tO + c0, *(uint32_t(*)[32])(ov + c0));
             const int bsel = i % kQBuf;
-            const uint32_t tS = tmem + bsel * kSCols + lane_off;
-            const float m = __uint_as_float(tc::tmem_ld1(tS + (kSCols - 2)));
-            const float l = __uint_as_float(tc::tmem_ld1(tS + (kSCols - 1)));
+            uint32_t meta[4];                         // -, partial row, m, l
+            tc::tmem_ld4(tmem + bsel * kSCols + lane_off + (kSCols - 4), meta);
             tc::tmem_ld_wait();
             tc::tc_fence_before();
             tc::mbar_arrive(o_empty);
             tc::mbar_arrive(&s_free[bsel]);
+            const int prow = (int)meta[1];
+            const float m = __uint_as_float(meta[2]), l = __uint_as_float(meta[3]);
             const float inv = 1.f / l;
 #pragma unroll
             for (int c = 0; c < D; c += 2) {
@@ -612,7 +604,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                __uint_as_float(ov[c + 1]) * inv);
                 ov[c / 2] = *(uint32_t *)&hv;
             }
-            if (valid) {
+            if (prow >= 0) {
+                uint4 *dst = (uint4 *)a.part_o + partial_chunk(prow, 0, D);
 #pragma unroll
                 for (int c = 0; c < D / 2; c += 4)
                     tc::st_global_v4_hint(dst + (c / 4) * 32,
