@@ -222,12 +222,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tc::mbar_arrive(&acc_empty[my_acc]);
                 if (row_ok) {
                     const int n0 = kt * nbpt;
+                    float bm[4];
                     if (cpb == 2) {
-                        *(float2 *)(out + n0) = make_float2(fmaxf(chunk_max[0], chunk_max[1]),
-                                                            fmaxf(chunk_max[2], chunk_max[3]));
+                        bm[0] = fmaxf(chunk_max[0], chunk_max[1]);
+                        bm[1] = fmaxf(chunk_max[2], chunk_max[3]);
                     } else {
-                        *(float4 *)(out + n0) = make_float4(chunk_max[0], chunk_max[1],
-                                                            chunk_max[2], chunk_max[3]);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) bm[q] = chunk_max[q];
+                    }
+                    if (a.NB % nbpt == 0) {        // rows start vector-aligned, tile in range
+                        if (cpb == 2) *(float2 *)(out + n0) = make_float2(bm[0], bm[1]);
+                        else *(float4 *)(out + n0) = make_float4(bm[0], bm[1], bm[2], bm[3]);
+                    } else {                       // S not a multiple of the key tile
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            if (q < nbpt && n0 + q < a.NB) out[n0 + q] = bm[q];
                     }
                 }
             }

@@ -56,6 +56,9 @@ def _case(name):
                             block=64, topk=4, dtype=bf),
         "bf16_decode_topk64": W("bf16_decode_topk64", B=2, T=1, S=8192, Hq=32, Hkv=4, d=128,
                                 d_idx=64, block=64, topk=64, dtype=bf),
+        # an odd number of 64-key blocks: the last 128-key index tile holds one block
+        "bf16_prefill_odd_blocks": W("bf16_prefill_odd_blocks", B=2, T=700, S=1088, Hq=8, Hkv=2,
+                                     d=128, d_idx=64, block=64, topk=5, dtype=bf),
     }
     return cases[name]
 
@@ -63,7 +66,7 @@ def _case(name):
 CASES = ["tiny_fp32_prefill", "bf16_prefill_2x1024", "bf16_chunk_ragged", "bf16_decode_small",
          "bf16_d64_mha", "bf16_dense_limit", "bf16_topk1", "fp32_gqa8", "bf16_prefill_R16",
          "bf16_prefill_R1_didx128", "bf16_prefill_B2_chunk", "bf16_decode_block128",
-         "bf16_decode_T4", "bf16_decode_topk64"]
+         "bf16_decode_T4", "bf16_decode_topk64", "bf16_prefill_odd_blocks"]
 
 
 def _inputs(w, seed=0):
