@@ -370,6 +370,9 @@ def run_ours(args, rank: int, ws: int):
         dominant = "sparse_attn_fwd"
     roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"], "traffic": None,
+            "traffic_note": ("the timed call is one launch per row chunk of each of the CSR, "
+                             "attention and combine kernels; per-kernel DRAM bytes are in the "
+                             "ncu summaries under profiles/"),
             "peak_source": pk["source"] + " bf16 burst (of " + pk["source"] + ")",
             "stage_ms": stages,
             "attention_tflops": attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12,
