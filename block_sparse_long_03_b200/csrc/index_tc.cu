@@ -15,9 +15,11 @@
 // (row, block) reaches HBM.  With index inputs on the 1/4 grid every dot
 // product is exact in fp32, so the scores equal the fp64 definition.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM
-// owner, warps 2-9 epilogue in two groups of four, one per TMEM accumulator
-// (warp w reads TMEM lanes 32*(w%4) .. +31).
+// Warp roles (352 threads): warp 0 TMA producer, warps 1 and 10 MMA issuers
+// (even and odd key tiles, each with its own waits, so one issuer's barrier
+// round trips overlap the other's tensor-core work; warp 1 owns TMEM), warps
+// 2-9 epilogue in two groups of four, one per TMEM accumulator (warp w reads
+// TMEM lanes 32*(w%4) .. +31).
 #include <math.h>
 
 #include "tc.cuh"
@@ -27,7 +29,7 @@ namespace {
 
 constexpr int kM = 128;            // rows per tile
 constexpr int kN = 256;            // keys per MMA tile
-constexpr int kThreads = 320;          // 2 + 8 warps
+constexpr int kThreads = 352;          // 3 + 8 warps
 constexpr int kKtChunk = 32;       // key tiles per work item
 
 struct IndexArgs {
@@ -65,6 +67,7 @@ template <int DIDX, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 IndexArgs a) {
+    static_assert(STAGES % 2 == 0, "each MMA issuer owns the ring stages of its parity");
     constexpr int kAtoms = DIDX / 64;                     // 128-byte swizzle atoms along d_idx
     constexpr uint32_t kABytes = kM * DIDX * 2;
     constexpr uint32_t kBBytes = kN * DIDX * 2;
@@ -83,7 +86,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&a_full[i], 1);
-            tc::mbar_init(&a_empty[i], 1);
+            tc::mbar_init(&a_empty[i], 2);          // both MMA issuers
             tc::mbar_init(&acc_full[i], 1);
             tc::mbar_init(&acc_empty[i], 4 * 32);   // one epilogue group
         }
@@ -125,19 +128,30 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 10) {
+        // ------------------------------------------------ MMA issuers
+        // Key tiles are numbered across the CTA's items; issuer `par` takes
+        // the tiles of its parity, which use accumulator buffer `par` and the
+        // ring stages of that parity (STAGES is even).
         if (lane == 0) {
+            const int par = warp == 1 ? 0 : 1;
             constexpr uint32_t idesc = tc::idesc_bf16(kM, kN, 0, 0);
-            int stage = 0, bphase = 0, abuf = 0, aphase = 0, acc = 0, accphase = 0;
-            for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+            int j = 0, abuf = 0, aphase = 0;
+            bool ok = true;
+            for (int i = blockIdx.x; i < a.items && ok; i += gridDim.x) {
                 const Item it = decode_item(a, i);
                 if (!it.valid) continue;
                 if (!tc::mbar_wait(&a_full[abuf], aphase, a.err, abort_flag)) break;
                 const uint32_t a_base = tc::smem_u32(sA + abuf * kABytes);
                 for (int kt = it.kt0; kt < it.kt1; ++kt) {
-                    if (!tc::mbar_wait(&acc_empty[acc], accphase ^ 1, a.err, abort_flag)) break;
-                    if (!tc::mbar_wait(&b_full[stage], bphase, a.err, abort_flag)) break;
+                    const int jj = j++;
+                    if ((jj & 1) != par) continue;
+                    const int stage = jj % STAGES, acc = jj & 1;
+                    if (!tc::mbar_wait(&acc_empty[acc], ((jj >> 1) & 1) ^ 1, a.err, abort_flag) ||
+                        !tc::mbar_wait(&b_full[stage], (jj / STAGES) & 1, a.err, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc::tc_fence_after();
                     const uint32_t b_base = tc::smem_u32(sB + stage * kBBytes);
 #pragma unroll
@@ -149,9 +163,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     tc::mma_commit(&b_empty[stage]);
                     tc::mma_commit(&acc_full[acc]);
-                    if (++stage == STAGES) { stage = 0; bphase ^= 1; }
-                    if (++acc == 2) { acc = 0; accphase ^= 1; }
                 }
+                if (!ok) break;
                 tc::mma_commit(&a_empty[abuf]);
                 if (++abuf == 2) { abuf = 0; aphase ^= 1; }
             }
