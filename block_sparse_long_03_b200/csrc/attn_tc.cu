@@ -521,11 +521,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         if (j_base + h0 + c > p) v[c] = __float_as_uint(-INFINITY);
                 }
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    m0 = fmaxf(m0, __uint_as_float(v[c]));
-                    m1 = fmaxf(m1, __uint_as_float(v[c + 1]));
-                    m2 = fmaxf(m2, __uint_as_float(v[c + 2]));
-                    m3 = fmaxf(m3, __uint_as_float(v[c + 3]));
+                for (int c = 0; c < 64; c += 8) {
+                    m0 = tc::fmax3(m0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+                    m1 = tc::fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+                    m2 = tc::fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
+                    m3 = tc::fmax3(m3, __uint_as_float(v[c + 6]), __uint_as_float(v[c + 7]));
                 }
             }
             float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));

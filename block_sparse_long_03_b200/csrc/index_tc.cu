@@ -203,19 +203,23 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int u = 0; u < 4; ++u) tc::tmem_ld32(tbase + h * 128 + u * 32, v[u]);
                     tc::tmem_ld_wait();
+                    if (h == 1) {                             // all columns in registers
+                        tc::tc_fence_before();
+                        tc::mbar_arrive(&acc_empty[my_acc]);
+                    }
                     const int64_t j0 = (int64_t)kt * kN + h * 128;
                     if (j0 + 127 <= p) {                      // no causal mask needed
 #pragma unroll
                         for (int c = 0; c < 2; ++c) {         // 64-column chunks
-                            float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+                            float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
                             for (int q = 0; q < 32; q += 2) {
-                                m0 = fmaxf(m0, __uint_as_float(v[2 * c][q]));
-                                m1 = fmaxf(m1, __uint_as_float(v[2 * c][q + 1]));
-                                m2 = fmaxf(m2, __uint_as_float(v[2 * c + 1][q]));
-                                m3 = fmaxf(m3, __uint_as_float(v[2 * c + 1][q + 1]));
+                                m0 = tc::fmax3(m0, __uint_as_float(v[2 * c][q]),
+                                               __uint_as_float(v[2 * c][q + 1]));
+                                m1 = tc::fmax3(m1, __uint_as_float(v[2 * c + 1][q]),
+                                               __uint_as_float(v[2 * c + 1][q + 1]));
                             }
-                            chunk_max[2 * h + c] = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+                            chunk_max[2 * h + c] = fmaxf(m0, m1);
                         }
                     } else {
 #pragma unroll
@@ -231,8 +235,6 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         }
                     }
                 }
-                tc::tc_fence_before();
-                tc::mbar_arrive(&acc_empty[my_acc]);
                 if (row_ok) {
                     const int n0 = kt * nbpt;
                     float bm[4];
