@@ -88,7 +88,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::mbar_init(&a_full[i], 1);
             tc::mbar_init(&a_empty[i], 2);          // both MMA issuers
             tc::mbar_init(&acc_full[i], 1);
-            tc::mbar_init(&acc_empty[i], 4 * 32);   // one epilogue group
+            tc::mbar_init(&acc_empty[i], 8 * 32);   // both epilogue groups
         }
         for (int i = 0; i < STAGES; ++i) {
             tc::mbar_init(&b_full[i], 1);
@@ -171,15 +171,16 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ------------------------------------------------ epilogue
-        // Two groups of four warps; group `grp` drains accumulator buffer
-        // `grp`, i.e. every other key tile, so each group has two MMA
-        // periods per tile.  Warp w reads TMEM lanes 32*(w%4) .. +31.
+        // Two groups of four warps; on every key tile group `grp` takes
+        // columns [128 grp, 128 grp + 128) (whole blocks), so a thread reads
+        // 128 columns in one TMEM round trip and the accumulator is released
+        // after one read per group.  Warp w reads TMEM lanes 32*(w%4) .. +31.
         const int grp = (warp - 2) / 4;
         const int quad = warp % 4;
         const int row_in_tile = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int nbpt = kN / a.block;                    // blocks per key tile (2 or 4)
-        const int cpb = a.block / 64;                     // 64-column chunks per block
+        const int nbph = nbpt / 2;                        // blocks per half tile (1 or 2)
         int acc = 0, accphase = 0;
         for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
             const Item it = decode_item(a, i);
@@ -192,66 +193,52 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int kt = it.kt0; kt < it.kt1; ++kt) {
                 const int my_acc = acc, my_phase = accphase;
                 if (++acc == 2) { acc = 0; accphase ^= 1; }
-                if (my_acc != grp) continue;
                 if (!tc::mbar_wait(&acc_full[my_acc], my_phase, a.err, abort_flag)) break;
                 tc::tc_fence_after();
-                const uint32_t tbase = tmem + my_acc * kN + lane_off;
-                float chunk_max[4];
+                uint32_t v[4][32];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {                 // two halves of 128 columns
-                    uint32_t v[4][32];
+                for (int u = 0; u < 4; ++u)
+                    tc::tmem_ld32(tmem + my_acc * kN + grp * 128 + lane_off + u * 32, v[u]);
+                tc::tmem_ld_wait();
+                tc::tc_fence_before();
+                tc::mbar_arrive(&acc_empty[my_acc]);
+                const int64_t j0 = (int64_t)kt * kN + grp * 128;
+                float cm[2];                                  // per 64-column chunk
+                if (j0 + 127 <= p) {                          // no causal mask needed
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) tc::tmem_ld32(tbase + h * 128 + u * 32, v[u]);
-                    tc::tmem_ld_wait();
-                    if (h == 1) {                             // all columns in registers
-                        tc::tc_fence_before();
-                        tc::mbar_arrive(&acc_empty[my_acc]);
+                    for (int c = 0; c < 2; ++c) {
+                        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+                        for (int q = 0; q < 32; q += 2) {
+                            m0 = tc::fmax3(m0, __uint_as_float(v[2 * c][q]),
+                                           __uint_as_float(v[2 * c][q + 1]));
+                            m1 = tc::fmax3(m1, __uint_as_float(v[2 * c + 1][q]),
+                                           __uint_as_float(v[2 * c + 1][q + 1]));
+                        }
+                        cm[c] = fmaxf(m0, m1);
                     }
-                    const int64_t j0 = (int64_t)kt * kN + h * 128;
-                    if (j0 + 127 <= p) {                      // no causal mask needed
+                } else {
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {         // 64-column chunks
-                            float m0 = -INFINITY, m1 = -INFINITY;
+                    for (int c = 0; c < 2; ++c) {
+                        float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-                            for (int q = 0; q < 32; q += 2) {
-                                m0 = tc::fmax3(m0, __uint_as_float(v[2 * c][q]),
-                                               __uint_as_float(v[2 * c][q + 1]));
-                                m1 = tc::fmax3(m1, __uint_as_float(v[2 * c + 1][q]),
-                                               __uint_as_float(v[2 * c + 1][q + 1]));
-                            }
-                            chunk_max[2 * h + c] = fmaxf(m0, m1);
+                        for (int q = 0; q < 32; ++q) {
+                            const int64_t j = j0 + c * 64 + q;
+                            if (j <= p) m0 = fmaxf(m0, __uint_as_float(v[2 * c][q]));
+                            if (j + 32 <= p) m1 = fmaxf(m1, __uint_as_float(v[2 * c + 1][q]));
                         }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) {
-                                const int64_t j = j0 + c * 64 + q;
-                                if (j <= p) m0 = fmaxf(m0, __uint_as_float(v[2 * c][q]));
-                                if (j + 32 <= p) m1 = fmaxf(m1, __uint_as_float(v[2 * c + 1][q]));
-                            }
-                            chunk_max[2 * h + c] = fmaxf(m0, m1);
-                        }
+                        cm[c] = fmaxf(m0, m1);
                     }
                 }
                 if (row_ok) {
-                    const int n0 = kt * nbpt;
-                    float bm[4];
-                    if (cpb == 2) {
-                        bm[0] = fmaxf(chunk_max[0], chunk_max[1]);
-                        bm[1] = fmaxf(chunk_max[2], chunk_max[3]);
+                    const int n0 = kt * nbpt + grp * nbph;    // first block of this half
+                    if (nbph == 1) {
+                        if (n0 < a.NB) out[n0] = fmaxf(cm[0], cm[1]);
+                    } else if ((a.NB & 1) == 0 && n0 + 1 < a.NB) {
+                        *(float2 *)(out + n0) = make_float2(cm[0], cm[1]);
                     } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) bm[q] = chunk_max[q];
-                    }
-                    if (a.NB % nbpt == 0) {        // rows start vector-aligned, tile in range
-                        if (cpb == 2) *(float2 *)(out + n0) = make_float2(bm[0], bm[1]);
-                        else *(float4 *)(out + n0) = make_float4(bm[0], bm[1], bm[2], bm[3]);
-                    } else {                       // S not a multiple of the key tile
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (q < nbpt && n0 + q < a.NB) out[n0 + q] = bm[q];
+                        if (n0 < a.NB) out[n0] = cm[0];
+                        if (n0 + 1 < a.NB) out[n0 + 1] = cm[1];
                     }
                 }
             }
