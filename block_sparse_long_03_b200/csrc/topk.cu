@@ -11,8 +11,11 @@
 // order-preserving uint32 -- nothing is exponentiated.
 //
 // One warp per row.  The candidates' ordered keys are staged in shared
-// memory, then a 4-pass radix select (8 bits per pass, warp-private
-// histogram) finds the M-th largest score u*.  Every candidate above u* is
+// memory, then a radix select (8 bits per pass, warp-private histogram)
+// finds the M-th largest score u*.  Leading bits shared by every candidate
+// need no pass, and lanes holding the same digit add to the histogram once
+// (one atomic per distinct digit per warp step), since neighbouring scores
+// often share their high bits.  Every candidate above u* is
 // kept, and of the candidates equal to u* the lowest ids are kept until M is
 // reached.  A final pass in ascending id order emits the kept ids with
 // ballots, so the output is ascending without a sort; cb is appended last
@@ -51,17 +54,41 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
         return;
     }
     const float *row = bs + r * NB;
-    for (int n = lane; n < cb; n += 32) keys[n] = ordered_key(row[n]);
+    uint32_t all_and = 0xffffffffu, all_or = 0u;
+    for (int n = lane; n < cb; n += 32) {
+        const uint32_t v = ordered_key(row[n]);
+        keys[n] = v;
+        all_and &= v;
+        all_or |= v;
+    }
+    all_and = __reduce_and_sync(0xffffffffu, all_and);
+    all_or = __reduce_or_sync(0xffffffffu, all_or);
     __syncwarp();
 
+    // bits above the highest differing bit are the same in every key
+    const uint32_t diff = all_and ^ all_or;
+    const int top = diff ? 31 - __clz(diff) : -1;  // highest differing bit
     uint32_t prefix = 0, mask = 0;
+    int first_shift = 24;
+    while (first_shift > 0 && first_shift > top) first_shift -= 8;
+    if (first_shift + 8 <= 31) {
+        mask = 0xffffffffu << (first_shift + 8);
+        prefix = all_and & mask;
+    }
     int remaining = M;                // how many still to take at or below prefix
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = first_shift; shift >= 0; shift -= 8) {
         for (int i = lane; i < 256; i += 32) hist[i] = 0;
         __syncwarp();
-        for (int n = lane; n < cb; n += 32) {
-            const uint32_t v = keys[n];
-            if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1u);
+        for (int base = 0; base < cb; base += 32) {
+            const int n = base + lane;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool in = n < cb && (v & mask) == prefix;
+            const unsigned act = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                const uint32_t d = (v >> shift) & 255u;
+                const unsigned same = __match_any_sync(act, d);
+                if (lane == __ffs(same) - 1) atomicAdd(&hist[d], (uint32_t)__popc(same));
+            }
         }
         __syncwarp();
         // lane L owns digits [8L, 8L + 8); suffix sums over digits, high to low
@@ -115,10 +142,154 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
     if (lane == 0) out[M] = cb;
 }
 
+// Rows with many candidates (NB > kWarpRowMaxNB): one CTA of kCtaThreads
+// threads per row runs the same selection, the histogram and the ordered
+// emission shared by its warps.
+constexpr int kWarpRowMaxNB = 2048;
+constexpr int kCtaThreads = 256;
+
+__global__ void __launch_bounds__(kCtaThreads)
+topk_cta_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int T_, int S, int G,
+                int NB, int block, int topk) {
+    extern __shared__ uint32_t sm[];
+    constexpr int kWarps = kCtaThreads / 32;
+    uint32_t *keys = sm;                          // [NB]
+    uint32_t *hist = keys + NB;                   // [256]
+    uint32_t *red = hist + 256;                   // [2 * kWarps] reductions / warp counts
+    int *sel = (int *)(red + 2 * kWarps);         // [3]: digit, gt_count, (spare)
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int64_t r = blockIdx.x;
+    const int t = (int)((r / G) % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int M = topk - 1;
+    int32_t *out = ids + r * topk;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    if (M == 0) {
+        if (tid == 0) out[0] = cb;
+        return;
+    }
+    if (cb <= M) {
+        for (int i = tid; i < topk; i += kCtaThreads) out[i] = (i <= cb) ? i : -1;
+        return;
+    }
+    const float *row = bs + r * NB;
+    uint32_t all_and = 0xffffffffu, all_or = 0u;
+    for (int n = tid; n < cb; n += kCtaThreads) {
+        const uint32_t v = ordered_key(row[n]);
+        keys[n] = v;
+        all_and &= v;
+        all_or |= v;
+    }
+    all_and = __reduce_and_sync(0xffffffffu, all_and);
+    all_or = __reduce_or_sync(0xffffffffu, all_or);
+    if (lane == 0) { red[warp] = all_and; red[kWarps + warp] = all_or; }
+    __syncthreads();
+    all_and = 0xffffffffu; all_or = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) { all_and &= red[w]; all_or |= red[kWarps + w]; }
+    const uint32_t diff = all_and ^ all_or;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t prefix = 0, mask = 0;
+    int first_shift = 24;
+    while (first_shift > 0 && first_shift > top) first_shift -= 8;
+    if (first_shift + 8 <= 31) {
+        mask = 0xffffffffu << (first_shift + 8);
+        prefix = all_and & mask;
+    }
+    int remaining = M;
+    for (int shift = first_shift; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kCtaThreads) hist[i] = 0;
+        __syncthreads();
+        for (int base = 0; base < cb; base += kCtaThreads) {
+            const int n = base + tid;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool in = n < cb && (v & mask) == prefix;
+            const unsigned act = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                const uint32_t d = (v >> shift) & 255u;
+                const unsigned same = __match_any_sync(act, d);
+                if (lane == __ffs(same) - 1) atomicAdd(&hist[d], (uint32_t)__popc(same));
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t c[8], lane_sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c[i] = hist[lane * 8 + i]; lane_sum += c[i]; }
+            uint32_t incl = lane_sum;
+#pragma unroll
+            for (int off = 1; off < 32; off *= 2) {
+                const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += o;
+            }
+            const uint32_t above = incl - lane_sum;
+            int found = -1;
+            uint32_t gt_count = 0;
+            if (above < (uint32_t)remaining && above + lane_sum >= (uint32_t)remaining) {
+                uint32_t acc = above;
+                for (int i = 7; i >= 0; --i) {
+                    if (acc + c[i] >= (uint32_t)remaining) { found = lane * 8 + i; gt_count = acc; break; }
+                    acc += c[i];
+                }
+            }
+            if (found >= 0) { sel[0] = found; sel[1] = (int)gt_count; }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sel[0] << shift;
+        mask |= 255u << shift;
+        remaining -= sel[1];
+        __syncthreads();                              // sel and hist are reused
+    }
+    // ordered emission: per chunk of kCtaThreads ids, ranks from the warps'
+    // ballot counts
+    int ties_seen = 0, written = 0;
+    for (int base = 0; base < cb; base += kCtaThreads) {
+        const int n = base + tid;
+        const uint32_t v = (n < cb) ? keys[n] : 0u;
+        const bool eq = (n < cb) && v == prefix;
+        const unsigned eq_b = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) red[warp] = __popc(eq_b);
+        __syncthreads();
+        int eq_before = ties_seen, eq_total = ties_seen;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            eq_before += w < warp ? (int)red[w] : 0;
+            eq_total += (int)red[w];
+        }
+        const int tie_rank = eq_before + __popc(eq_b & lt_mask);
+        const bool take = (n < cb) && (v > prefix || (eq && tie_rank < remaining));
+        const unsigned tk_b = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) red[kWarps + warp] = __popc(tk_b);
+        __syncthreads();
+        int tk_before = written, tk_total = written;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            tk_before += w < warp ? (int)red[kWarps + w] : 0;
+            tk_total += (int)red[kWarps + w];
+        }
+        const int pos = tk_before + __popc(tk_b & lt_mask);
+        if (take && pos < M) out[pos] = n;
+        ties_seen = eq_total;
+        written = tk_total;
+        __syncthreads();                              // red is reused
+    }
+    if (tid == 0) out[M] = cb;
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st) {
     const int64_t nrows = s.index_rows();
+    if (s.NB > kWarpRowMaxNB) {
+        const size_t smem = sizeof(uint32_t) * ((size_t)s.NB + 256 + 2 * (kCtaThreads / 32) + 4);
+        if (smem > 220 * 1024) return cudaErrorInvalidConfiguration;
+        cudaFuncSetAttribute(topk_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        topk_cta_kernel<<<(unsigned)nrows, kCtaThreads, smem, st>>>(bs, ids, s.T, s.S, s.G, s.NB,
+                                                                     s.block, s.topk);
+        count_launches(1);
+        return cudaGetLastError();
+    }
     const size_t per_warp = sizeof(uint32_t) * ((size_t)s.NB + 256);
     int warps = 8;
     while (warps > 1 && per_warp * warps > 200 * 1024) warps /= 2;
