@@ -6,20 +6,22 @@
 //
 // The token-level scores form a GEMM: rows are the (token, group) pairs of
 // q_idx viewed as a [B*T*G, d_idx] matrix, columns are index keys.  A work
-// item is (batch entry, 128-row tile, chunk of key tiles).  Per key tile of
-// 256 keys, one elected thread issues tcgen05.mma (M=128, N=256, K=16 steps,
-// bf16 in, fp32 accumulate) into one of two TMEM accumulators; the TMA
-// producer keeps a ring of k_idx tiles in shared memory; four epilogue warps
-// read the accumulator back (each thread owns one row), apply the causal
-// mask j <= p(t) and max-pool every block's columns, so only one fp32 per
-// (row, block) reaches HBM.  With index inputs on the 1/4 grid every dot
-// product is exact in fp32, so the scores equal the fp64 definition.
+// item is (batch entry, 256-row tile, chunk of key tiles).  Key tiles of 128
+// keys stream through a TMA ring in shared memory; each is multiplied with
+// the item's two 128-row A tiles (tcgen05.mma M=128, N=128, K=16 steps, bf16
+// in, fp32 accumulate), so a key tile is read from L2 once per 256 rows.  The
+// two products of a key tile go to one of two TMEM accumulator buffers
+// (2 x 128 columns each).  Epilogue warp group g reads the 128 columns of A
+// tile g (each thread one row, one TMEM round trip), applies the causal mask
+// j <= p(t) and max-pools every block's columns, so only one fp32 per (row,
+// block) reaches HBM.  With index inputs on the 1/4 grid every dot product is
+// exact in fp32, so the scores equal the fp64 definition.
 //
 // Warp roles (352 threads): warp 0 TMA producer, warps 1 and 10 MMA issuers
 // (even and odd key tiles, each with its own waits, so one issuer's barrier
 // round trips overlap the other's tensor-core work; warp 1 owns TMEM), warps
-// 2-9 epilogue in two groups of four, one per TMEM accumulator (warp w reads
-// TMEM lanes 32*(w%4) .. +31).
+// 2-9 epilogue in two groups of four (warp w reads TMEM lanes 32*(w%4) ..
+// +31).
 #include <math.h>
 
 #include "tc.cuh"
@@ -27,16 +29,17 @@
 namespace msa {
 namespace {
 
-constexpr int kM = 128;            // rows per tile
-constexpr int kN = 256;            // keys per MMA tile
+constexpr int kM = 128;            // rows per A tile (one MMA)
+constexpr int kRowsPerItem = 2 * kM;   // two A tiles share every key tile
+constexpr int kN = 128;            // keys per key tile
 constexpr int kThreads = 352;          // 3 + 8 warps
-constexpr int kKtChunk = 32;       // key tiles per work item
+constexpr int kKtChunk = 64;       // key tiles per work item
 
 struct IndexArgs {
     float *bs;
     uint32_t *err;
     int B, T, S, G, NB, block, d_idx;
-    int MT;                        // row tiles per batch entry
+    int MT;                        // 256-row tiles per batch entry
     int CPT;                       // chunks per row tile (max over tiles)
     int items;
     int fill_noncausal;            // write -inf for blocks past the tile's key range
@@ -54,7 +57,7 @@ __device__ __forceinline__ Item decode_item(const IndexArgs &a, int i) {
     it.mt = a.MT - 1 - (rest % a.MT);          // large causal ranges first
     it.b = rest / a.MT;
     const int rows = a.T * a.G;
-    const int r_hi = min(rows - 1, it.mt * kM + kM - 1);
+    const int r_hi = min(rows - 1, it.mt * kRowsPerItem + kRowsPerItem - 1);
     const int64_t p_hi = (int64_t)a.S - a.T + r_hi / a.G;
     it.nkt = (int)(p_hi / kN) + 1;
     it.kt0 = c * kKtChunk;
@@ -73,8 +76,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr uint32_t kBBytes = kN * DIDX * 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t *sA = smem;                                   // [2][kAtoms][kM][64]
-    uint8_t *sB = smem + 2 * kABytes;                     // [STAGES][kAtoms][kN][64]
+    uint8_t *sA = smem;                                   // [2 buffers][2 tiles][kAtoms][kM][64]
+    uint8_t *sB = smem + 4 * kABytes;                     // [STAGES][kAtoms][kN][64]
     uint64_t *bar = (uint64_t *)(sB + STAGES * kBBytes);
     uint64_t *a_full = bar, *a_empty = bar + 2;
     uint64_t *b_full = bar + 4, *b_empty = bar + 4 + STAGES;
@@ -88,7 +91,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc::mbar_init(&a_full[i], 1);
             tc::mbar_init(&a_empty[i], 2);          // both MMA issuers
             tc::mbar_init(&acc_full[i], 1);
-            tc::mbar_init(&acc_empty[i], 8 * 32);   // both epilogue groups
+            tc::mbar_init(&acc_empty[i], 8);        // one arrival per epilogue warp
         }
         for (int i = 0; i < STAGES; ++i) {
             tc::mbar_init(&b_full[i], 1);
@@ -111,11 +114,12 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const Item it = decode_item(a, i);
                 if (!it.valid) continue;
                 if (!tc::mbar_wait(&a_empty[abuf], aphase ^ 1, a.err, abort_flag)) break;
-                tc::mbar_expect_tx(&a_full[abuf], kABytes);
-                const int row0 = it.b * a.T * a.G + it.mt * kM;
-                for (int at = 0; at < kAtoms; ++at)
-                    tc::tma_load_2d(sA + abuf * kABytes + at * kM * 128, &tm_q, &a_full[abuf],
-                                    at * 64, row0);
+                tc::mbar_expect_tx(&a_full[abuf], 2 * kABytes);
+                const int row0 = it.b * a.T * a.G + it.mt * kRowsPerItem;
+                for (int half = 0; half < 2; ++half)
+                    for (int at = 0; at < kAtoms; ++at)
+                        tc::tma_load_2d(sA + (abuf * 2 + half) * kABytes + at * kM * 128, &tm_q,
+                                        &a_full[abuf], at * 64, row0 + half * kM);
                 if (++abuf == 2) { abuf = 0; aphase ^= 1; }
                 for (int kt = it.kt0; kt < it.kt1; ++kt) {
                     if (!tc::mbar_wait(&b_empty[stage], bphase ^ 1, a.err, abort_flag)) break;
@@ -142,7 +146,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const Item it = decode_item(a, i);
                 if (!it.valid) continue;
                 if (!tc::mbar_wait(&a_full[abuf], aphase, a.err, abort_flag)) break;
-                const uint32_t a_base = tc::smem_u32(sA + abuf * kABytes);
+                const uint32_t a_base = tc::smem_u32(sA + abuf * 2 * kABytes);
                 for (int kt = it.kt0; kt < it.kt1; ++kt) {
                     const int jj = j++;
                     if ((jj & 1) != par) continue;
@@ -155,11 +159,15 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     tc::tc_fence_after();
                     const uint32_t b_base = tc::smem_u32(sB + stage * kBBytes);
 #pragma unroll
-                    for (int ks = 0; ks < DIDX / 16; ++ks) {
-                        const uint32_t off_a = (ks / 4) * kM * 128 + (ks % 4) * 32;
-                        const uint32_t off_b = (ks / 4) * kN * 128 + (ks % 4) * 32;
-                        tc::mma_ss(tmem + acc * kN, tc::sdesc_sw128(a_base + off_a, 16, 1024),
-                                   tc::sdesc_sw128(b_base + off_b, 16, 1024), idesc, ks > 0);
+                    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                        for (int ks = 0; ks < DIDX / 16; ++ks) {
+                            const uint32_t off_a = half * kABytes + (ks / 4) * kM * 128 + (ks % 4) * 32;
+                            const uint32_t off_b = (ks / 4) * kN * 128 + (ks % 4) * 32;
+                            tc::mma_ss(tmem + acc * 2 * kN + half * kN,
+                                       tc::sdesc_sw128(a_base + off_a, 16, 1024),
+                                       tc::sdesc_sw128(b_base + off_b, 16, 1024), idesc, ks > 0);
+                        }
                     }
                     tc::mma_commit(&b_empty[stage]);
                     tc::mma_commit(&acc_full[acc]);
@@ -171,24 +179,21 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else {
         // ------------------------------------------------ epilogue
-        // Two groups of four warps; on every key tile group `grp` takes
-        // columns [128 grp, 128 grp + 128) (whole blocks), so a thread reads
-        // 128 columns in one TMEM round trip and the accumulator is released
-        // after one read per group.  Warp w reads TMEM lanes 32*(w%4) .. +31.
+        // Two groups of four warps; on every key tile group `grp` reads the
+        // 128 columns of A tile `grp` (one row per thread, one TMEM round
+        // trip) and the accumulator buffer is released after one read per
+        // group.  Warp w reads TMEM lanes 32*(w%4) .. +31.
         const int grp = (warp - 2) / 4;
         const int quad = warp % 4;
-        const int row_in_tile = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int nbpt = kN / a.block;                    // blocks per key tile (2 or 4)
-        const int nbph = nbpt / 2;                        // blocks per half tile (1 or 2)
+        const int nbpt = kN / a.block;                    // blocks per key tile (1 or 2)
         int acc = 0, accphase = 0;
         for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
             const Item it = decode_item(a, i);
             if (!it.valid) continue;
-            const int r = it.mt * kM + row_in_tile;       // row within batch entry b
+            const int r = it.mt * kRowsPerItem + grp * kM + quad * 32 + lane;
             const bool row_ok = r < a.T * a.G;
-            const int t = r / a.G;
-            const int64_t p = (int64_t)a.S - a.T + t;
+            const int64_t p = (int64_t)a.S - a.T + r / a.G;
             float *out = a.bs + ((int64_t)it.b * a.T * a.G + r) * a.NB;
             for (int kt = it.kt0; kt < it.kt1; ++kt) {
                 const int my_acc = acc, my_phase = accphase;
@@ -198,13 +203,14 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint32_t v[4][32];
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    tc::tmem_ld32(tmem + my_acc * kN + grp * 128 + lane_off + u * 32, v[u]);
+                    tc::tmem_ld32(tmem + my_acc * 2 * kN + grp * kN + lane_off + u * 32, v[u]);
                 tc::tmem_ld_wait();
                 tc::tc_fence_before();
-                tc::mbar_arrive(&acc_empty[my_acc]);
-                const int64_t j0 = (int64_t)kt * kN + grp * 128;
+                __syncwarp();                             // every lane's read is done
+                if (lane == 0) tc::mbar_arrive(&acc_empty[my_acc]);
+                const int64_t j0 = (int64_t)kt * kN;
                 float cm[2];                                  // per 64-column chunk
-                if (j0 + 127 <= p) {                          // no causal mask needed
+                if (j0 + kN - 1 <= p) {                       // no causal mask needed
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         float m0 = -INFINITY, m1 = -INFINITY;
@@ -231,18 +237,17 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
                 if (row_ok) {
-                    const int n0 = kt * nbpt + grp * nbph;    // first block of this half
-                    if (nbph == 1) {
-                        if (n0 < a.NB) out[n0] = fmaxf(cm[0], cm[1]);
-                    } else if ((a.NB & 1) == 0 && n0 + 1 < a.NB) {
-                        *(float2 *)(out + n0) = make_float2(cm[0], cm[1]);
-                    } else {
-                        if (n0 < a.NB) out[n0] = cm[0];
-                        if (n0 + 1 < a.NB) out[n0 + 1] = cm[1];
+                    if (nbpt == 1) {
+                        out[kt] = fmaxf(cm[0], cm[1]);
+                    } else if ((a.NB & 1) == 0) {             // rows start 8-byte aligned
+                        *(float2 *)(out + 2 * kt) = make_float2(cm[0], cm[1]);
+                    } else {                                  // an odd number of 64-key blocks
+                        out[2 * kt] = cm[0];
+                        if (2 * kt + 1 < a.NB) out[2 * kt + 1] = cm[1];
                     }
                 }
             }
-            if (a.fill_noncausal && row_ok && it.kt1 == it.nkt && grp == 0) {
+            if (a.fill_noncausal && row_ok && it.kt1 == it.nkt) {
                 for (int n = it.nkt * nbpt; n < a.NB; ++n) out[n] = -INFINITY;
             }
         }
@@ -269,12 +274,12 @@ cudaError_t launch_tc(const Shape &s, const void *q_idx, const void *k_idx, floa
     IndexArgs a{};
     a.bs = bs; a.err = err;
     a.B = s.B; a.T = s.T; a.S = s.S; a.G = s.G; a.NB = s.NB; a.block = s.block; a.d_idx = s.d_idx;
-    a.MT = (s.T * s.G + kM - 1) / kM;
+    a.MT = (s.T * s.G + kRowsPerItem - 1) / kRowsPerItem;
     const int nkt_max = (s.S - 1) / kN + 1;
     a.CPT = (nkt_max + kKtChunk - 1) / kKtChunk;
     a.items = s.B * a.MT * a.CPT;
     a.fill_noncausal = fill_noncausal ? 1 : 0;
-    const size_t smem = 1024 + 2 * (size_t)kM * DIDX * 2 + (size_t)STAGES * kN * DIDX * 2 + 256;
+    const size_t smem = 1024 + 4 * (size_t)kM * DIDX * 2 + (size_t)STAGES * kN * DIDX * 2 + 256;
     auto k = index_tc_kernel<DIDX, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -297,7 +302,7 @@ bool index_tc_supported(const Shape &s) {
 cudaError_t launch_index_scores_tc(const Shape &s, const void *q_idx, const void *k_idx,
                                    float *bs, bool fill_noncausal, uint32_t *err,
                                    cudaStream_t st) {
-    if (s.d_idx == 64) return launch_tc<64, 4>(s, q_idx, k_idx, bs, fill_noncausal, err, st);
+    if (s.d_idx == 64) return launch_tc<64, 8>(s, q_idx, k_idx, bs, fill_noncausal, err, st);
     return launch_tc<128, 2>(s, q_idx, k_idx, bs, fill_noncausal, err, st);
 }
 
