@@ -55,19 +55,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Non-blocking probe of a phase (acquire on success).  Issued ahead of a
-// blocking instruction (an MMA issue), its result is ready by the time it is
-// read, so a wait on an already-completed phase costs no round trip.
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
 // Wait for the phase of `bar` with the given parity to complete, for at most
 // kWaitLimitNs.  On expiry the wait records MSA_ERR_DEVICE_TIMEOUT in the
 // error word, raises the CTA's abort flag and returns false; callers then
