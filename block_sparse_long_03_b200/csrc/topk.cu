@@ -11,11 +11,8 @@
 // order-preserving uint32 -- nothing is exponentiated.
 //
 // One warp per row.  The candidates' ordered keys are staged in shared
-// memory, then a radix select (8 bits per pass, warp-private histogram)
-// finds the M-th largest score u*.  Leading bits shared by every candidate
-// need no pass, and lanes holding the same digit add to the histogram once
-// (one atomic per distinct digit per warp step), since neighbouring scores
-// often share their high bits.  Every candidate above u* is
+// memory, then a 4-pass radix select (8 bits per pass, warp-private
+// histogram) finds the M-th largest score u*.  Every candidate above u* is
 // kept, and of the candidates equal to u* the lowest ids are kept until M is
 // reached.  A final pass in ascending id order emits the kept ids with
 // ballots, so the output is ascending without a sort; cb is appended last
@@ -54,41 +51,17 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
         return;
     }
     const float *row = bs + r * NB;
-    uint32_t all_and = 0xffffffffu, all_or = 0u;
-    for (int n = lane; n < cb; n += 32) {
-        const uint32_t v = ordered_key(row[n]);
-        keys[n] = v;
-        all_and &= v;
-        all_or |= v;
-    }
-    all_and = __reduce_and_sync(0xffffffffu, all_and);
-    all_or = __reduce_or_sync(0xffffffffu, all_or);
+    for (int n = lane; n < cb; n += 32) keys[n] = ordered_key(row[n]);
     __syncwarp();
 
-    // bits above the highest differing bit are the same in every key
-    const uint32_t diff = all_and ^ all_or;
-    const int top = diff ? 31 - __clz(diff) : -1;  // highest differing bit
     uint32_t prefix = 0, mask = 0;
-    int first_shift = 24;
-    while (first_shift > 0 && first_shift > top) first_shift -= 8;
-    if (first_shift + 8 <= 31) {
-        mask = 0xffffffffu << (first_shift + 8);
-        prefix = all_and & mask;
-    }
     int remaining = M;                // how many still to take at or below prefix
-    for (int shift = first_shift; shift >= 0; shift -= 8) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = lane; i < 256; i += 32) hist[i] = 0;
         __syncwarp();
-        for (int base = 0; base < cb; base += 32) {
-            const int n = base + lane;
-            const uint32_t v = n < cb ? keys[n] : 0u;
-            const bool in = n < cb && (v & mask) == prefix;
-            const unsigned act = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const uint32_t d = (v >> shift) & 255u;
-                const unsigned same = __match_any_sync(act, d);
-                if (lane == __ffs(same) - 1) atomicAdd(&hist[d], (uint32_t)__popc(same));
-            }
+        for (int n = lane; n < cb; n += 32) {
+            const uint32_t v = keys[n];
+            if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1u);
         }
         __syncwarp();
         // lane L owns digits [8L, 8L + 8); suffix sums over digits, high to low
@@ -144,7 +117,8 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
 
 // Rows with many candidates (NB > kWarpRowMaxNB): one CTA of kCtaThreads
 // threads per row runs the same selection, the histogram and the ordered
-// emission shared by its warps.
+// emission shared by its warps; leading bits shared by every candidate need
+// no radix pass.
 constexpr int kWarpRowMaxNB = 2048;
 constexpr int kCtaThreads = 256;
 
@@ -204,12 +178,7 @@ topk_cta_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int T_,
             const int n = base + tid;
             const uint32_t v = n < cb ? keys[n] : 0u;
             const bool in = n < cb && (v & mask) == prefix;
-            const unsigned act = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const uint32_t d = (v >> shift) & 255u;
-                const unsigned same = __match_any_sync(act, d);
-                if (lane == __ffs(same) - 1) atomicAdd(&hist[d], (uint32_t)__popc(same));
-            }
+            if (in) atomicAdd(&hist[(v >> shift) & 255u], 1u);
         }
         __syncthreads();
         if (warp == 0) {
