@@ -66,6 +66,13 @@ __device__ __forceinline__ Item decode_item(const IndexArgs &a, int i) {
     return it;
 }
 
+// The k-th item of this CTA.  Items come roughly in decreasing size (long
+// causal ranges first); alternate rounds run the CTAs in reverse order
+// ("snake" order) so every CTA gets a similar share of large and small items.
+__device__ __forceinline__ int cta_item(int k) {
+    return k * gridDim.x + ((k & 1) ? gridDim.x - 1 - blockIdx.x : blockIdx.x);
+}
+
 template <int DIDX, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -110,7 +117,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int stage = 0, bphase = 0, abuf = 0, aphase = 0;
-            for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+            for (int k = 0, i = cta_item(0); i < a.items && !*abort_flag; i = cta_item(++k)) {
                 const Item it = decode_item(a, i);
                 if (!it.valid) continue;
                 if (!tc::mbar_wait(&a_empty[abuf], aphase ^ 1, a.err, abort_flag)) break;
@@ -142,7 +149,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t idesc = tc::idesc_bf16(kM, kN, 0, 0);
             int j = 0, abuf = 0, aphase = 0;
             bool ok = true;
-            for (int i = blockIdx.x; i < a.items && ok; i += gridDim.x) {
+            for (int k = 0, i = cta_item(0); i < a.items && ok; i = cta_item(++k)) {
                 const Item it = decode_item(a, i);
                 if (!it.valid) continue;
                 if (!tc::mbar_wait(&a_full[abuf], aphase, a.err, abort_flag)) break;
@@ -188,7 +195,7 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
         const int nbpt = kN / a.block;                    // blocks per key tile (1 or 2)
         int acc = 0, accphase = 0;
-        for (int i = blockIdx.x; i < a.items && !*abort_flag; i += gridDim.x) {
+        for (int k = 0, i = cta_item(0); i < a.items && !*abort_flag; i = cta_item(++k)) {
             const Item it = decode_item(a, i);
             if (!it.valid) continue;
             const int r = it.mt * kRowsPerItem + grp * kM + quad * 32 + lane;
