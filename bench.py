@@ -63,6 +63,19 @@ def index_flops(w) -> float:
     return float(w.B * w.G * 2 * w.d_idx * (p + 1).sum())
 
 
+def partial_floor_bytes(w) -> float:
+    """HBM bytes the KV-block-outer schedule of the sparse attention call must
+    move whatever the kernels do: each (query, group, kept slot, head) partial
+    (d fp16 values + an fp32 LSE) written once and read once by the combine,
+    plus Q, K, V read once and O, LSE written once."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    p = w.S - w.T + np.arange(w.T, dtype=np.int64)
+    slots = w.B * w.G * np.minimum(w.topk, p // w.block + 1).sum()
+    partials = slots * (w.Hq // w.Hkv) * (w.d * 2 + 4) * 2
+    io = w.B * w.T * w.Hq * (2 * w.d * e + 4) + 2 * w.B * w.S * w.G * w.d * e
+    return float(partials + io)
+
+
 def decode_bytes(w) -> float:
     """HBM bytes a decode step must move: all index keys, the kept K/V
     blocks, the index queries, Q, O, LSE, block scores and ids."""
@@ -376,6 +389,12 @@ def run_ours(args, rank: int, ws: int):
             "peak_source": pk["source"] + " bf16 burst (of " + pk["source"] + ")",
             "stage_ms": stages,
             "attention_tflops": attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12,
+            # the schedule's own floor: partials through HBM at the measured bandwidth
+            "partial_traffic_floor": {
+                "hbm_bytes": partial_floor_bytes(w),
+                "ms_at_measured_hbm": partial_floor_bytes(w) / (pk["hbm_gbs"] * 1e9) * 1e3,
+                "frac": (partial_floor_bytes(w) / (pk["hbm_gbs"] * 1e9) * 1e3)
+                        / stages["sparse_attn_fwd"]},
             "index_tflops": idx_fl / (stages["index_block_scores"] / 1e3) / 1e12}
     e2e = None if args.no_e2e else e2e_prefill(prob, max(1, min(args.steps, 3)), 1, ws)
     prob.free()
