@@ -18,14 +18,15 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_OK = 0
 MSA_F32, MSA_BF16 = 0, 1
-MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD = 0, 1
+MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD, MSA_WS_FORWARD_HOST = 0, 1, 2
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
                 4: "MSA_ERR_DEVICE_TIMEOUT", 5: "MSA_ERR_WORKSPACE", 6: "MSA_ERR_BAD_BLOCK_IDS"}
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
-           "msa_kernel_launches", "msa_forward_noalloc", "msa_selftest_wait_timeout")
+           "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
+           "msa_selftest_wait_timeout")
 
 
 class MsaError(RuntimeError):
@@ -59,6 +60,8 @@ def _load():
     lib.msa_get_device_error.argtypes = [vp, vp]
     lib.msa_forward_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.msa_forward_noalloc.restype = st
+    lib.msa_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_forward_host.restype = st
     lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.msa_selftest_wait_timeout.restype = st
     lib.msa_kernel_launches.argtypes = []
@@ -138,6 +141,19 @@ def msa_forward(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, worksp
     _check(lib.msa_forward(ctypes.byref(params), _ptr(q_idx), _ptr(k_idx), _ptr(Q), _ptr(K),
                            _ptr(V), _ptr(block_ids), _ptr(O), _ptr(lse), _ptr(workspace),
                            workspace.numel(), _stream(stream)), "msa_forward")
+
+
+def msa_forward_host(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, device_buffer,
+                     stream=None):
+    """msa_forward on page-locked host tensors (``pin_memory()``); the copies to
+    and from ``device_buffer`` (a CUDA uint8 tensor of at least
+    ``msa_workspace_size(params, MSA_WS_FORWARD_HOST)`` bytes) run inside the
+    call, overlapped with the kernels.  O, lse and block_ids are valid once
+    ``stream`` has passed the call."""
+    _check(lib.msa_forward_host(ctypes.byref(params), _ptr(q_idx), _ptr(k_idx), _ptr(Q),
+                                _ptr(K), _ptr(V), _ptr(block_ids), _ptr(O), _ptr(lse),
+                                _ptr(device_buffer), device_buffer.numel(), _stream(stream)),
+           "msa_forward_host")
 
 
 def msa_get_device_error(workspace, stream=None) -> int:

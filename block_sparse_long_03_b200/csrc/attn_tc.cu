@@ -860,6 +860,8 @@ bool attn_tc_supported(const Shape &s) {
 
 size_t attn_tc_workspace(const Shape &s) { return make_plan(s).total; }
 
+int64_t attn_tc_rows_per_pass(const Shape &s) { return make_plan(s).rows_per_chunk; }
+
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st) {

@@ -85,6 +85,9 @@ cudaError_t launch_attention(const Shape &s, const void *Q, const void *K, const
 
 msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// Device buffer bytes of msa_forward_host (defined with that call below).
+size_t host_ws_size(const Shape &s);
+
 }  // namespace
 }  // namespace msa
 
@@ -110,6 +113,7 @@ size_t msa_workspace_size(const msa_params_t *params, int which) {
     if (make_shape(params, &s) != MSA_OK) return 0;
     if (which == MSA_WS_SPARSE_ATTN) return attn_ws(s);
     if (which == MSA_WS_FORWARD) return forward_ws(s);
+    if (which == MSA_WS_FORWARD_HOST) return host_ws_size(s);
     return 0;
 }
 
@@ -263,4 +267,258 @@ extern "C" msa_status_t msa_forward_noalloc(const msa_params_t *params, const vo
     if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
     if (e == cudaSuccess) e = launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
     return cuda_status(e);
+}
+
+// ---------------------------------------------------------------------------
+// msa_forward_host: the forward pass from page-locked host buffers, with the
+// copies in both directions overlapped with the kernels (see include/msa.h).
+// The caller's stream carries the kernels; two library-owned streams per
+// device carry the host-to-device and device-to-host copies, joined to it by
+// events.
+// ---------------------------------------------------------------------------
+#include <algorithm>
+#include <vector>
+
+namespace msa {
+namespace {
+
+// Sequences [b0, b0 + nb), query tokens [t0, t1) of each: the whole call
+// (nb = B, t0 = 0, t1 = T) or one chunk of one sequence (nb = 1).
+struct Piece {
+    int b0, nb, t0, t1;
+};
+
+// Query tokens per chunk, or 0 when sequences run whole.  Chunks are a
+// multiple of block (every chunk then ends on a block boundary of the keys),
+// about T / 16 and at least 4096 tokens, and at most one pass of the
+// tensor-core attention so that no chunk is split again inside the call.
+int64_t host_chunk(const Shape &s) {
+    if (!use_attn_tc(s)) return 0;
+    const int64_t blk = s.block;
+    int64_t c = ((int64_t)s.T / 16 + blk - 1) / blk * blk;
+    c = std::max<int64_t>(c, (4096 + blk - 1) / blk * blk);
+    Shape one = s;
+    one.B = 1;
+    c = std::min<int64_t>(c, attn_tc_rows_per_pass(one) / blk * blk);
+    if (c < 64 || c >= s.T) return 0;
+    return c;
+}
+
+// Chunks end at T, T - c, T - 2c, ...; a first chunk shorter than 64 tokens
+// (below the tensor-core attention's minimum) is folded into the next one.
+std::vector<Piece> host_pieces(const Shape &s, int64_t c, int n_seq) {
+    std::vector<Piece> v;
+    if (c == 0) {
+        v.push_back({0, s.B, 0, s.T});
+        return v;
+    }
+    const int64_t n = (s.T + c - 1) / c;
+    for (int b = 0; b < n_seq; ++b) {
+        int64_t lo = 0;
+        for (int64_t k = n - 1; k >= 0; --k) {
+            const int64_t hi = s.T - k * c;
+            if (k > 0 && hi - lo < 64) continue;
+            v.push_back({b, 1, (int)lo, (int)hi});
+            lo = hi;
+        }
+    }
+    return v;
+}
+
+// The shape a piece's attention call sees: its queries are the last t1 - t0
+// of the first S - T + t1 keys, so p(t) is unchanged.
+Shape piece_shape(const Shape &s, const Piece &p) {
+    Shape q = s;
+    q.B = p.nb;
+    q.T = p.t1 - p.t0;
+    q.S = s.S - s.T + p.t1;
+    q.NB = q.S / s.block;
+    return q;
+}
+
+size_t elem_bytes(const Shape &s) { return s.dtype == MSA_BF16 ? 2 : 4; }
+
+// Device buffer: [error word][attention scratch][block scores][block ids]
+// [q_idx][k_idx][Q][K][V][O][lse], each region 256-byte aligned.
+struct HostLayout {
+    size_t scratch, bs, ids, q_idx, k_idx, Q, K, V, O, lse, total;
+    size_t q_idx_bytes, k_idx_bytes, Q_bytes, KV_bytes, lse_bytes, ids_bytes;
+};
+
+HostLayout host_layout(const Shape &s) {
+    HostLayout L;
+    const size_t e = elem_bytes(s);
+    L.q_idx_bytes = (size_t)s.index_rows() * s.d_idx * e;
+    L.k_idx_bytes = (size_t)s.B * s.S * s.d_idx * e;
+    L.Q_bytes = (size_t)s.rows() * s.Hq * s.d * e;
+    L.KV_bytes = (size_t)s.B * s.S * s.Hkv * s.d * e;
+    L.lse_bytes = (size_t)s.rows() * s.Hq * sizeof(float);
+    L.ids_bytes = block_id_bytes(s);
+    size_t scratch = 0;
+    for (const Piece &p : host_pieces(s, host_chunk(s), 1))
+        scratch = std::max(scratch, attn_scratch(piece_shape(s, p)));
+    size_t o = kErrorBytes;
+    L.scratch = o; o += align_up(scratch);
+    L.bs = o;      o += align_up(block_score_bytes(s));
+    L.ids = o;     o += align_up(L.ids_bytes);
+    L.q_idx = o;   o += align_up(L.q_idx_bytes);
+    L.k_idx = o;   o += align_up(L.k_idx_bytes);
+    L.Q = o;       o += align_up(L.Q_bytes);
+    L.K = o;       o += align_up(L.KV_bytes);
+    L.V = o;       o += align_up(L.KV_bytes);
+    L.O = o;       o += align_up(L.Q_bytes);
+    L.lse = o;     o += align_up(L.lse_bytes);
+    L.total = o;
+    return L;
+}
+
+size_t host_ws_size(const Shape &s) { return host_layout(s).total; }
+
+// True when [p, p + bytes) starts and ends in page-locked host memory.
+bool page_locked(const void *p, size_t bytes) {
+    if (p == nullptr || bytes == 0) return false;
+    const char *ends[2] = {(const char *)p, (const char *)p + bytes - 1};
+    for (const char *q : ends) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, q) != cudaSuccess) {
+            cudaGetLastError();   // clear the sticky-free error of the query
+            return false;
+        }
+        if (a.type != cudaMemoryTypeHost) return false;
+    }
+    return true;
+}
+
+struct CopyStreams {
+    cudaStream_t up = nullptr, down = nullptr;   // host-to-device, device-to-host
+    std::vector<cudaEvent_t> ev;
+};
+std::mutex g_host_mu;
+CopyStreams g_copy[kMaxDevices];
+
+// Streams of the current device and at least n events (caller holds the lock).
+cudaError_t copy_streams(int dev, size_t n, CopyStreams **out) {
+    CopyStreams &c = g_copy[dev];
+    cudaError_t e = cudaSuccess;
+    if (c.up == nullptr) e = cudaStreamCreateWithFlags(&c.up, cudaStreamNonBlocking);
+    if (e == cudaSuccess && c.down == nullptr)
+        e = cudaStreamCreateWithFlags(&c.down, cudaStreamNonBlocking);
+    while (e == cudaSuccess && c.ev.size() < n) {
+        cudaEvent_t ev;
+        e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+        if (e == cudaSuccess) c.ev.push_back(ev);
+    }
+    *out = &c;
+    return e;
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void *q_idx,
+                                         const void *k_idx, const void *Q, const void *K,
+                                         const void *V, int32_t *block_ids, void *O, float *lse,
+                                         void *device_buffer, size_t device_buffer_bytes,
+                                         void *stream) {
+    Shape s;
+    msa_status_t rc = make_shape(params, &s);
+    if (rc != MSA_OK) return rc;
+    const HostLayout L = host_layout(s);
+    if (!device_buffer || ((uintptr_t)device_buffer % kAlign) != 0 ||
+        device_buffer_bytes < L.total)
+        return MSA_ERR_WORKSPACE;
+    if (!page_locked(q_idx, L.q_idx_bytes) || !page_locked(k_idx, L.k_idx_bytes) ||
+        !page_locked(Q, L.Q_bytes) || !page_locked(K, L.KV_bytes) ||
+        !page_locked(V, L.KV_bytes) || !page_locked(O, L.Q_bytes) ||
+        !page_locked(lse, L.lse_bytes) || (block_ids && !page_locked(block_ids, L.ids_bytes)))
+        return MSA_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return MSA_ERR_CUDA;
+
+    const std::vector<Piece> pieces = host_pieces(s, host_chunk(s), s.B);
+    std::lock_guard<std::mutex> lock(g_host_mu);
+    CopyStreams *cs = nullptr;
+    // events: start, index inputs, ids, two per piece, and the two joins
+    if (copy_streams(dev, 5 + 2 * pieces.size(), &cs) != cudaSuccess) return MSA_ERR_CUDA;
+    cudaEvent_t *ev = cs->ev.data();
+    cudaEvent_t ev_start = ev[0], ev_idx = ev[1], ev_ids = ev[2], ev_up = ev[3], ev_down = ev[4];
+    cudaEvent_t *ev_in = ev + 5, *ev_out = ev + 5 + pieces.size();
+    cudaStream_t st = (cudaStream_t)stream, up = cs->up, down = cs->down;
+
+    char *db = (char *)device_buffer;
+    uint32_t *err = (uint32_t *)db;
+    char *scratch = db + L.scratch;
+    float *bs = (float *)(db + L.bs);
+    int32_t *ids = (int32_t *)(db + L.ids);
+    char *dq_idx = db + L.q_idx, *dk_idx = db + L.k_idx, *dQ = db + L.Q, *dK = db + L.K;
+    char *dV = db + L.V, *dO = db + L.O;
+    float *dlse = (float *)(db + L.lse);
+    const char *hQ = (const char *)Q, *hK = (const char *)K, *hV = (const char *)V;
+    char *hO = (char *)O;
+    const size_t e = elem_bytes(s);
+    const size_t q_row = (size_t)s.Hq * s.d * e, kv_row = (size_t)s.Hkv * s.d * e;
+
+    cudaError_t ce = cudaEventRecord(ev_start, st);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(up, ev_start, 0);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_start, 0);
+    // index branch: its inputs first, then scores and Top-k for every query
+    if (ce == cudaSuccess)
+        ce = cudaMemcpyAsync(dq_idx, q_idx, L.q_idx_bytes, cudaMemcpyHostToDevice, up);
+    if (ce == cudaSuccess)
+        ce = cudaMemcpyAsync(dk_idx, k_idx, L.k_idx_bytes, cudaMemcpyHostToDevice, up);
+    if (ce == cudaSuccess) ce = cudaEventRecord(ev_idx, up);
+    if (ce == cudaSuccess) ce = cudaMemsetAsync(err, 0, kErrorBytes, st);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, ev_idx, 0);
+    if (ce == cudaSuccess) ce = launch_index(s, dq_idx, dk_idx, bs, false, err, st);
+    if (ce == cudaSuccess) ce = launch_topk(s, bs, ids, st);
+    if (ce == cudaSuccess && block_ids) {
+        ce = cudaEventRecord(ev_ids, st);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_ids, 0);
+        if (ce == cudaSuccess)
+            ce = cudaMemcpyAsync(block_ids, ids, L.ids_bytes, cudaMemcpyDeviceToHost, down);
+    }
+    // main branch, piece by piece
+    std::vector<int64_t> kv_done((size_t)s.B, 0);   // K/V rows already on the device
+    for (size_t i = 0; i < pieces.size() && ce == cudaSuccess; ++i) {
+        const Piece &p = pieces[i];
+        const Shape ps = piece_shape(s, p);
+        const int64_t row0 = (int64_t)p.b0 * s.T + p.t0;   // first query token
+        const size_t nq = (size_t)p.nb * (p.t1 - p.t0);    // query tokens of the piece
+        ce = cudaMemcpyAsync(dQ + row0 * q_row, hQ + row0 * q_row, nq * q_row,
+                             cudaMemcpyHostToDevice, up);
+        for (int b = p.b0; b < p.b0 + p.nb && ce == cudaSuccess; ++b) {
+            const int64_t lo = kv_done[b], hi = (int64_t)ps.S;
+            if (hi <= lo) continue;
+            const size_t off = ((size_t)b * s.S + lo) * kv_row, n = (size_t)(hi - lo) * kv_row;
+            ce = cudaMemcpyAsync(dK + off, hK + off, n, cudaMemcpyHostToDevice, up);
+            if (ce == cudaSuccess)
+                ce = cudaMemcpyAsync(dV + off, hV + off, n, cudaMemcpyHostToDevice, up);
+            kv_done[b] = hi;
+        }
+        if (ce == cudaSuccess) ce = cudaEventRecord(ev_in[i], up);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, ev_in[i], 0);
+        if (ce == cudaSuccess) {
+            const size_t kv0 = (size_t)p.b0 * s.S * kv_row;
+            ce = launch_attention(ps, dQ + row0 * q_row, dK + kv0, dV + kv0,
+                                  ids + row0 * s.G * s.topk, dO + row0 * q_row,
+                                  dlse + row0 * s.Hq, err, scratch, st);
+        }
+        if (ce == cudaSuccess) ce = cudaEventRecord(ev_out[i], st);
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_out[i], 0);
+        if (ce == cudaSuccess)
+            ce = cudaMemcpyAsync(hO + row0 * q_row, dO + row0 * q_row, nq * q_row,
+                                 cudaMemcpyDeviceToHost, down);
+        if (ce == cudaSuccess)
+            ce = cudaMemcpyAsync(lse + row0 * s.Hq, dlse + row0 * s.Hq,
+                                 nq * s.Hq * sizeof(float), cudaMemcpyDeviceToHost, down);
+    }
+    // whatever happened above, later work on the caller's stream waits for
+    // both copy streams
+    cudaError_t je = cudaEventRecord(ev_up, up);
+    if (je == cudaSuccess) je = cudaEventRecord(ev_down, down);
+    if (je == cudaSuccess) je = cudaStreamWaitEvent(st, ev_up, 0);
+    if (je == cudaSuccess) je = cudaStreamWaitEvent(st, ev_down, 0);
+    if (ce == cudaSuccess) ce = je;
+    return cuda_status(ce);
 }

@@ -57,6 +57,9 @@ cudaError_t launch_index_scores_tc(const Shape &s, const void *q_idx, const void
 // Tensor-core KV-block-outer sparse attention (bf16, d = 128) and its workspace.
 bool attn_tc_supported(const Shape &s);
 size_t attn_tc_workspace(const Shape &s);
+// Query tokens one pass of the tensor-core attention covers (its partials fit
+// a fixed budget); larger calls run several passes.
+int64_t attn_tc_rows_per_pass(const Shape &s);
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st);

@@ -19,10 +19,12 @@
  *   cb(t) = p(t) / block   the query's own ("current") block
  *
  * Conventions shared by every call:
- *   - Every tensor pointer is DEVICE memory, dense and row-major in the
- *     layout stated at the call, 16-byte aligned.  The caller allocates and
- *     owns all of it, workspace included; the library allocates nothing and
- *     keeps no state between calls other than per-device launch settings.
+ *   - Every tensor pointer is DEVICE memory (msa_forward_host alone takes
+ *     page-locked host buffers), dense and row-major in the layout stated at
+ *     the call, 16-byte aligned.  The caller allocates and owns all of it,
+ *     workspace included; the library allocates no memory and keeps no state
+ *     between calls other than per-device launch settings and the copy
+ *     streams and events of msa_forward_host.
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream).  A returned MSA_OK means the work was
  *     enqueued; device-side problems are recorded in the workspace's error
@@ -115,7 +117,9 @@ MSA_EXPORT msa_status_t msa_topk_blocks(const msa_params_t *params, const float 
                              int32_t *block_ids, void *stream);
 
 /* Workspace needs, in bytes, of msa_sparse_attn_fwd (which = 0) and
- * msa_forward (which = 1) for these shapes; 0 for invalid shapes. */
+ * msa_forward (which = 1) for these shapes, or the device buffer of
+ * msa_forward_host (which = 2, MSA_WS_FORWARD_HOST, defined with that call);
+ * 0 for invalid shapes. */
 #define MSA_WS_SPARSE_ATTN 0
 #define MSA_WS_FORWARD 1
 MSA_EXPORT size_t msa_workspace_size(const msa_params_t *params, int which);
@@ -196,6 +200,51 @@ MSA_EXPORT msa_status_t msa_forward_noalloc(const msa_params_t *params, const vo
                                             const void *k_idx, const void *Q, const void *K,
                                             const void *V, int32_t *block_ids, void *O,
                                             float *lse, void *stream);
+
+/*
+ * msa_forward for inputs and outputs in page-locked HOST memory.  The call
+ * copies the inputs to the device, runs the forward pass and copies O, lse
+ * (and the kept ids) back, with the copies in both directions overlapped
+ * with the kernels.  The paper has no counterpart of this call; the
+ * arithmetic is msa_forward's, and the outputs are bitwise those of
+ * msa_forward on the same inputs.
+ *
+ * Host buffers (same layouts and dtypes as msa_forward): q_idx, k_idx, Q, K,
+ * V are read, O and lse written, block_ids written when not NULL.  Each one
+ * must be page-locked over its whole extent (cudaHostAlloc, or a range
+ * registered with cudaHostRegister); otherwise MSA_ERR_INVALID_ARG.
+ *
+ * device_buffer: device memory of at least
+ * msa_workspace_size(params, MSA_WS_FORWARD_HOST) bytes, 256-byte aligned.
+ * It holds the device copies of every tensor and the forward scratch; its
+ * first 256 bytes are the device error word (msa_get_device_error).
+ *
+ * Schedule.  When a sequence is longer than one query chunk (a multiple of
+ * block, chosen from the shapes: about T/16 and at least 4096 tokens, and no
+ * more than one pass of the tensor-core attention), each sequence is split
+ * into chunks of consecutive queries, ending at T, T - C, T - 2C, ...
+ * The index tensors are copied first and the index scores and Top-k run for
+ * all queries while Q and the K/V rows each chunk needs are copied chunk by
+ * chunk; chunk c's attention starts once its rows are resident, and its O
+ * and lse rows are copied back while chunk c + 1 computes.  Shorter
+ * sequences run as one piece (copy in, compute, copy out).
+ *
+ * Streams.  The call is ordered on `stream` like every other call: its work
+ * starts after what was enqueued on `stream` before it, and work enqueued
+ * on `stream` after it starts once its last copy to the host has ended.
+ * The copies run on two non-blocking streams that the library creates once
+ * per device, with events from a per-device pool; those streams and events
+ * live until the process exits.  Calls on one device are serialised by a
+ * lock while they enqueue.  The host buffers must stay valid, and O, lse and
+ * block_ids unread, until `stream` has passed the call (e.g. after
+ * cudaStreamSynchronize(stream)).
+ */
+#define MSA_WS_FORWARD_HOST 2
+MSA_EXPORT msa_status_t msa_forward_host(const msa_params_t *params, const void *q_idx,
+                                         const void *k_idx, const void *Q, const void *K,
+                                         const void *V, int32_t *block_ids, void *O, float *lse,
+                                         void *device_buffer, size_t device_buffer_bytes,
+                                         void *stream);
 
 /*
  * Diagnostics: a check of the device failure path.  Launches one CTA that

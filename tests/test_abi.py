@@ -20,7 +20,7 @@ def test_header_declares_the_calls():
     names = declared_symbols()
     for want in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd", "msa_forward",
                  "msa_workspace_size", "msa_status_string", "msa_get_device_error",
-                 "msa_kernel_launches", "msa_selftest_wait_timeout"):
+                 "msa_kernel_launches", "msa_selftest_wait_timeout", "msa_forward_host"):
         assert want in names
 
 
@@ -59,6 +59,12 @@ def test_workspace_sizes():
     assert ws_fwd >= 256 + 4 * (1 * 256 * 2 * 2) + 4 * (1 * 256 * 2 * 2)
     assert binding.msa_workspace_size(_p(T=0), binding.MSA_WS_FORWARD) == 0
     assert binding.msa_workspace_size(p, 7) == 0
+    # the host-buffer call's device buffer holds the forward scratch plus a
+    # device copy of every input and output
+    ws_host = binding.msa_workspace_size(p, binding.MSA_WS_FORWARD_HOST)
+    tensors = 2 * (256 * 2 * 64 + 256 * 64 + 2 * 256 * 8 * 128 + 2 * 256 * 2 * 128) + 4 * 256 * 8
+    assert ws_host >= ws_fwd + tensors
+    assert binding.msa_workspace_size(_p(T=0), binding.MSA_WS_FORWARD_HOST) == 0
 
 
 BAD_SHAPES = [
@@ -81,6 +87,8 @@ def test_bad_shapes_rejected_on_host(kw, status):
                                    1 << 30, None) == status
     assert lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, ws,
                            1 << 30, None) == status
+    assert lib.msa_forward_host(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake,
+                                ws, 1 << 30, None) == status
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -102,4 +110,12 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.msa_sparse_attn_fwd(ctypes.byref(p), ok, ok, ok, ok, ok, ok,
                                    ctypes.c_void_p(0x20010), 1 << 30, None) == 5
     assert lib.msa_forward(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, ws, 16, None) == 5
+    # msa_forward_host checks its device buffer before looking at the host ones
+    need = binding.msa_workspace_size(p, binding.MSA_WS_FORWARD_HOST)
+    assert lib.msa_forward_host(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, None, need,
+                                None) == 5
+    assert lib.msa_forward_host(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, ws, need - 1,
+                                None) == 5
+    assert lib.msa_forward_host(ctypes.byref(p), None, ok, ok, ok, ok, None, ok, ok, ws, need,
+                                None) == 1
     assert lib.msa_get_device_error(None, None) == 5
