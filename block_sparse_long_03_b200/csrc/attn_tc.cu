@@ -637,7 +637,7 @@ namespace {
 // bytes, and all loads of a warp are independent (issued together).
 // Needs R | 32 and topk <= 64.
 template <int D, int kMaxPer>
-__global__ void __launch_bounds__(256, kMaxPer <= 8 ? 4 : 2)
+__global__ void __launch_bounds__(256, kMaxPer <= 8 ? 3 : 2)
 combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_o,
                                const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
                                float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
