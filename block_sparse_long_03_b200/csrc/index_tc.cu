@@ -42,7 +42,6 @@ struct IndexArgs {
     int MT;                        // 256-row tiles per batch entry
     int CPT;                       // chunks per row tile (max over tiles)
     int items;
-    int fill_noncausal;            // write -inf for blocks past the tile's key range
 };
 
 struct Item {
@@ -254,9 +253,6 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                 }
             }
-            if (a.fill_noncausal && row_ok && it.kt1 == it.nkt) {
-                for (int n = it.nkt * nbpt; n < a.NB; ++n) out[n] = -INFINITY;
-            }
         }
     }
     tc::tc_fence_before();
@@ -267,9 +263,41 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
+// Blocks that start after the query's position hold no causal key and score
+// -inf.  The scoring kernel writes every block up to the last key tile its
+// rows need; this kernel writes blocks cb(t) + 1 .. NB - 1 of every row (the
+// overlap is -inf on both sides), one warp per (token, group) row with
+// 16-byte stores.  Only the standalone index call needs it: the forward
+// pass's Top-k never reads past cb(t).
+__global__ void fill_noncausal_kernel(float *__restrict__ bs, int64_t rows, int T, int S, int G,
+                                      int NB, int block) {
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (x >= rows) return;
+    const int t = (int)((x / G) % T);
+    const int n0 = (int)(((int64_t)S - T + t) / block) + 1;
+    if (n0 >= NB) return;
+    const int64_t base = x * NB;
+    float *out = bs + base;
+    const int n_al = min(NB, n0 + (int)((4 - ((base + n0) & 3)) & 3));   // first 16-byte boundary
+    const int n_end = n_al + ((NB - n_al) & ~3);
+    if (lane < n_al - n0) out[n0 + lane] = -INFINITY;
+    const float4 ninf = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    for (int n = n_al + 4 * lane; n < n_end; n += 128) *(float4 *)(out + n) = ninf;
+    if (lane < NB - n_end) out[n_end + lane] = -INFINITY;
+}
+
 template <int DIDX, int STAGES>
 cudaError_t launch_tc(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
                       bool fill_noncausal, uint32_t *err, cudaStream_t st) {
+    if (fill_noncausal) {
+        const int64_t rows = s.index_rows();
+        fill_noncausal_kernel<<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
+            bs, rows, s.T, s.S, s.G, s.NB, s.block);
+        count_launches(1);
+        const cudaError_t ef = cudaGetLastError();
+        if (ef != cudaSuccess) return ef;
+    }
     CUtensorMap tq, tk;
     const uint64_t qd[2] = {(uint64_t)s.d_idx, (uint64_t)s.B * s.T * s.G};
     const uint64_t qs[1] = {(uint64_t)s.d_idx * 2};
@@ -285,7 +313,6 @@ cudaError_t launch_tc(const Shape &s, const void *q_idx, const void *k_idx, floa
     const int nkt_max = (s.S - 1) / kN + 1;
     a.CPT = (nkt_max + kKtChunk - 1) / kKtChunk;
     a.items = s.B * a.MT * a.CPT;
-    a.fill_noncausal = fill_noncausal ? 1 : 0;
     const size_t smem = 1024 + 4 * (size_t)kM * DIDX * 2 + (size_t)STAGES * kN * DIDX * 2 + 256;
     auto k = index_tc_kernel<DIDX, STAGES>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -96,10 +96,14 @@ def test_forward_matches_oracle(name):
                         ref["O"], ref["lse"], w.dtype, name)
 
 
-@pytest.mark.parametrize("name", ["tiny_fp32_prefill", "bf16_chunk_ragged", "bf16_decode_small"])
+@pytest.mark.parametrize("name", ["tiny_fp32_prefill", "bf16_chunk_ragged", "bf16_decode_small",
+                                  "bf16_prefill_odd_blocks", "bf16_prefill_B2_chunk",
+                                  "bf16_prefill_R1_didx128"])
 def test_index_scores_and_topk_calls(name):
-    """The two index-branch calls on their own: block scores bit-exact, and
-    Top-k run on the ORACLE's block scores gives the oracle's ids."""
+    """The two index-branch calls on their own: block scores bit-exact (the
+    -inf of every non-causal block included: odd block counts, T < S and
+    two sequences exercise the fill's unaligned head and tail), and Top-k
+    run on the ORACLE's block scores gives the oracle's ids."""
     msa = _msa()
     w = _case(name)
     inp = _inputs(w, seed=3)
