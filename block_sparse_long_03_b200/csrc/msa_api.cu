@@ -289,9 +289,9 @@ struct Piece {
 };
 
 // Query tokens per chunk, or 0 when sequences run whole.  Chunks are a
-// multiple of block (every chunk then ends on a block boundary of the keys),
-// about T / 16 and at least 4096 tokens, and at most one pass of the
-// tensor-core attention so that no chunk is split again inside the call.
+// multiple of block, about T / 16 and at least 4096 tokens, and at most one
+// pass of the tensor-core attention so that no chunk is split again inside
+// the call.
 int64_t host_chunk(const Shape &s) {
     if (!use_attn_tc(s)) return 0;
     const int64_t blk = s.block;
@@ -304,20 +304,41 @@ int64_t host_chunk(const Shape &s) {
     return c;
 }
 
-// Chunks end at T, T - c, T - 2c, ...; a first chunk shorter than 64 tokens
-// (below the tensor-core attention's minimum) is folded into the next one.
+// Pieces of each sequence.  Every piece but the last ends on a key-block
+// boundary of p(t) (its end e has (T - e) % block == 0), so each piece's call
+// of shape (T' = e - t0, S' = S - T + e) has S' a multiple of block.  The
+// first piece is short (about c / 8) so the first attention starts soon after
+// the copies begin, the last is short (about c / 4) so little is left to copy
+// back after the last kernel, and the pieces between hold c queries.  A piece
+// shorter than 128 queries is merged into the next one, so every piece runs
+// the same index and attention kernels as the whole call would (the tensor-
+// core kernels need 128 index rows and 64 queries) and gives the same bits.
 std::vector<Piece> host_pieces(const Shape &s, int64_t c, int n_seq) {
     std::vector<Piece> v;
     if (c == 0) {
         v.push_back({0, s.B, 0, s.T});
         return v;
     }
-    const int64_t n = (s.T + c - 1) / c;
+    const int64_t blk = s.block, T = s.T;
+    const int64_t phase = T % blk;                        // valid ends: phase + m * blk, and T
+    auto end_at_or_after = [&](int64_t x) {               // smallest valid end >= x
+        const int64_t m = x <= phase ? 0 : (x - phase + blk - 1) / blk;
+        return std::min<int64_t>(T, phase + m * blk);
+    };
+    const int64_t first = std::max<int64_t>(blk, c / 8 / blk * blk);
+    const int64_t last = std::max<int64_t>(blk, c / 4 / blk * blk);
+    std::vector<int64_t> ends;
+    int64_t e = end_at_or_after(std::max<int64_t>(64, first));
+    while (e < T) {
+        ends.push_back(e);
+        e = end_at_or_after(e < T - last ? std::min<int64_t>(e + c, T - last) : T);
+    }
+    ends.push_back(T);
     for (int b = 0; b < n_seq; ++b) {
         int64_t lo = 0;
-        for (int64_t k = n - 1; k >= 0; --k) {
-            const int64_t hi = s.T - k * c;
-            if (k > 0 && hi - lo < 64) continue;
+        for (size_t k = 0; k < ends.size(); ++k) {
+            const int64_t hi = ends[k];
+            if (hi - lo < 128 && k + 1 < ends.size()) continue;  // merge into the next piece
             v.push_back({b, 1, (int)lo, (int)hi});
             lo = hi;
         }
@@ -354,12 +375,14 @@ HostLayout host_layout(const Shape &s) {
     L.KV_bytes = (size_t)s.B * s.S * s.Hkv * s.d * e;
     L.lse_bytes = (size_t)s.rows() * s.Hq * sizeof(float);
     L.ids_bytes = block_id_bytes(s);
-    size_t scratch = 0;
-    for (const Piece &p : host_pieces(s, host_chunk(s), 1))
+    size_t scratch = 0, bs = 0;                 // the largest piece's needs
+    for (const Piece &p : host_pieces(s, host_chunk(s), 1)) {
         scratch = std::max(scratch, attn_scratch(piece_shape(s, p)));
+        bs = std::max(bs, block_score_bytes(piece_shape(s, p)));
+    }
     size_t o = kErrorBytes;
     L.scratch = o; o += align_up(scratch);
-    L.bs = o;      o += align_up(block_score_bytes(s));
+    L.bs = o;      o += align_up(bs);
     L.ids = o;     o += align_up(L.ids_bytes);
     L.q_idx = o;   o += align_up(L.q_idx_bytes);
     L.k_idx = o;   o += align_up(L.k_idx_bytes);
@@ -439,11 +462,11 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
     const std::vector<Piece> pieces = host_pieces(s, host_chunk(s), s.B);
     std::lock_guard<std::mutex> lock(g_host_mu);
     CopyStreams *cs = nullptr;
-    // events: start, index inputs, ids, two per piece, and the two joins
-    if (copy_streams(dev, 5 + 2 * pieces.size(), &cs) != cudaSuccess) return MSA_ERR_CUDA;
+    // events: start, the two joins, and three per piece
+    if (copy_streams(dev, 3 + 3 * pieces.size(), &cs) != cudaSuccess) return MSA_ERR_CUDA;
     cudaEvent_t *ev = cs->ev.data();
-    cudaEvent_t ev_start = ev[0], ev_idx = ev[1], ev_ids = ev[2], ev_up = ev[3], ev_down = ev[4];
-    cudaEvent_t *ev_in = ev + 5, *ev_out = ev + 5 + pieces.size();
+    cudaEvent_t ev_start = ev[0], ev_up = ev[1], ev_down = ev[2];
+    cudaEvent_t *ev_idx = ev + 3, *ev_in = ev_idx + pieces.size(), *ev_out = ev_in + pieces.size();
     cudaStream_t st = (cudaStream_t)stream, up = cs->up, down = cs->down;
 
     char *db = (char *)device_buffer;
@@ -454,39 +477,44 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
     char *dq_idx = db + L.q_idx, *dk_idx = db + L.k_idx, *dQ = db + L.Q, *dK = db + L.K;
     char *dV = db + L.V, *dO = db + L.O;
     float *dlse = (float *)(db + L.lse);
+    const char *hq_idx = (const char *)q_idx, *hk_idx = (const char *)k_idx;
     const char *hQ = (const char *)Q, *hK = (const char *)K, *hV = (const char *)V;
     char *hO = (char *)O;
     const size_t e = elem_bytes(s);
     const size_t q_row = (size_t)s.Hq * s.d * e, kv_row = (size_t)s.Hkv * s.d * e;
+    const size_t qi_row = (size_t)s.G * s.d_idx * e, ki_row = (size_t)s.d_idx * e;
+    const size_t id_row = (size_t)s.G * s.topk * sizeof(int32_t);
 
     cudaError_t ce = cudaEventRecord(ev_start, st);
     if (ce == cudaSuccess) ce = cudaStreamWaitEvent(up, ev_start, 0);
     if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_start, 0);
-    // index branch: its inputs first, then scores and Top-k for every query
-    if (ce == cudaSuccess)
-        ce = cudaMemcpyAsync(dq_idx, q_idx, L.q_idx_bytes, cudaMemcpyHostToDevice, up);
-    if (ce == cudaSuccess)
-        ce = cudaMemcpyAsync(dk_idx, k_idx, L.k_idx_bytes, cudaMemcpyHostToDevice, up);
-    if (ce == cudaSuccess) ce = cudaEventRecord(ev_idx, up);
     if (ce == cudaSuccess) ce = cudaMemsetAsync(err, 0, kErrorBytes, st);
-    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, ev_idx, 0);
-    if (ce == cudaSuccess) ce = launch_index(s, dq_idx, dk_idx, bs, false, err, st);
-    if (ce == cudaSuccess) ce = launch_topk(s, bs, ids, st);
-    if (ce == cudaSuccess && block_ids) {
-        ce = cudaEventRecord(ev_ids, st);
-        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_ids, 0);
-        if (ce == cudaSuccess)
-            ce = cudaMemcpyAsync(block_ids, ids, L.ids_bytes, cudaMemcpyDeviceToHost, down);
-    }
-    // main branch, piece by piece
-    std::vector<int64_t> kv_done((size_t)s.B, 0);   // K/V rows already on the device
+    // Piece by piece: the index rows go first, so the piece's scores and
+    // Top-k run while its Q and K/V rows are still being copied.
+    std::vector<int64_t> keys_done((size_t)s.B, 0);   // key rows already on the device
+    std::vector<int64_t> kv_done((size_t)s.B, 0);
     for (size_t i = 0; i < pieces.size() && ce == cudaSuccess; ++i) {
         const Piece &p = pieces[i];
         const Shape ps = piece_shape(s, p);
         const int64_t row0 = (int64_t)p.b0 * s.T + p.t0;   // first query token
         const size_t nq = (size_t)p.nb * (p.t1 - p.t0);    // query tokens of the piece
-        ce = cudaMemcpyAsync(dQ + row0 * q_row, hQ + row0 * q_row, nq * q_row,
+        const size_t kv0 = (size_t)p.b0 * s.S;              // first key row of the piece
+        // index branch inputs: the piece's index queries and the keys it newly needs
+        ce = cudaMemcpyAsync(dq_idx + row0 * qi_row, hq_idx + row0 * qi_row, nq * qi_row,
                              cudaMemcpyHostToDevice, up);
+        for (int b = p.b0; b < p.b0 + p.nb && ce == cudaSuccess; ++b) {
+            const int64_t lo = keys_done[b], hi = (int64_t)ps.S;
+            if (hi <= lo) continue;
+            const size_t off = ((size_t)b * s.S + lo) * ki_row;
+            ce = cudaMemcpyAsync(dk_idx + off, hk_idx + off, (size_t)(hi - lo) * ki_row,
+                                 cudaMemcpyHostToDevice, up);
+            keys_done[b] = hi;
+        }
+        if (ce == cudaSuccess) ce = cudaEventRecord(ev_idx[i], up);
+        // main branch inputs
+        if (ce == cudaSuccess)
+            ce = cudaMemcpyAsync(dQ + row0 * q_row, hQ + row0 * q_row, nq * q_row,
+                                 cudaMemcpyHostToDevice, up);
         for (int b = p.b0; b < p.b0 + p.nb && ce == cudaSuccess; ++b) {
             const int64_t lo = kv_done[b], hi = (int64_t)ps.S;
             if (hi <= lo) continue;
@@ -497,14 +525,19 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
             kv_done[b] = hi;
         }
         if (ce == cudaSuccess) ce = cudaEventRecord(ev_in[i], up);
+        // kernels of the piece
+        if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, ev_idx[i], 0);
+        if (ce == cudaSuccess)
+            ce = launch_index(ps, dq_idx + row0 * qi_row, dk_idx + kv0 * ki_row, bs, false, err,
+                              st);
+        if (ce == cudaSuccess) ce = launch_topk(ps, bs, ids + row0 * s.G * s.topk, st);
         if (ce == cudaSuccess) ce = cudaStreamWaitEvent(st, ev_in[i], 0);
-        if (ce == cudaSuccess) {
-            const size_t kv0 = (size_t)p.b0 * s.S * kv_row;
-            ce = launch_attention(ps, dQ + row0 * q_row, dK + kv0, dV + kv0,
+        if (ce == cudaSuccess)
+            ce = launch_attention(ps, dQ + row0 * q_row, dK + kv0 * kv_row, dV + kv0 * kv_row,
                                   ids + row0 * s.G * s.topk, dO + row0 * q_row,
                                   dlse + row0 * s.Hq, err, scratch, st);
-        }
         if (ce == cudaSuccess) ce = cudaEventRecord(ev_out[i], st);
+        // outputs of the piece
         if (ce == cudaSuccess) ce = cudaStreamWaitEvent(down, ev_out[i], 0);
         if (ce == cudaSuccess)
             ce = cudaMemcpyAsync(hO + row0 * q_row, dO + row0 * q_row, nq * q_row,
@@ -512,6 +545,9 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
         if (ce == cudaSuccess)
             ce = cudaMemcpyAsync(lse + row0 * s.Hq, dlse + row0 * s.Hq,
                                  nq * s.Hq * sizeof(float), cudaMemcpyDeviceToHost, down);
+        if (ce == cudaSuccess && block_ids)
+            ce = cudaMemcpyAsync((char *)block_ids + row0 * id_row, (char *)ids + row0 * id_row,
+                                 nq * id_row, cudaMemcpyDeviceToHost, down);
     }
     // whatever happened above, later work on the caller's stream waits for
     // both copy streams

@@ -219,14 +219,16 @@ MSA_EXPORT msa_status_t msa_forward_noalloc(const msa_params_t *params, const vo
  * It holds the device copies of every tensor and the forward scratch; its
  * first 256 bytes are the device error word (msa_get_device_error).
  *
- * Schedule.  When a sequence is longer than one query chunk (a multiple of
- * block, chosen from the shapes: about T/16 and at least 4096 tokens, and no
+ * Schedule.  When a sequence is longer than one query chunk C (a multiple
+ * of block chosen from the shapes: about T/16, at least 4096 tokens, and no
  * more than one pass of the tensor-core attention), each sequence is split
- * into chunks of consecutive queries, ending at T, T - C, T - 2C, ...
- * The index tensors are copied first and the index scores and Top-k run for
- * all queries while Q and the K/V rows each chunk needs are copied chunk by
- * chunk; chunk c's attention starts once its rows are resident, and its O
- * and lse rows are copied back while chunk c + 1 computes.  Shorter
+ * into pieces of consecutive queries: a short first piece (about C/8),
+ * pieces of C, and a short last piece (about C/4), each ending where
+ * T - end is a multiple of block.  For each piece the call copies its index
+ * queries and the index keys it newly needs, then its Q rows and the K/V
+ * rows it newly needs; the piece's index scores and Top-k run once its index
+ * rows are resident, its attention once its Q, K and V rows are, and its O,
+ * lse (and ids) are copied back while the next piece computes.  Shorter
  * sequences run as one piece (copy in, compute, copy out).
  *
  * Streams.  The call is ordered on `stream` like every other call: its work

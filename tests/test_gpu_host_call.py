@@ -5,11 +5,12 @@ Every query row's arithmetic is the same whichever call or chunk it runs in
 (index scores and Top-k run over all rows at once; the attention of a row
 depends only on its own kept blocks, and its partials are combined in slot
 order), so the host call must reproduce msa_forward exactly.  Shapes cover
-sequences split into query chunks (several chunks, two sequences, T < S, a
-short first chunk folded into the next) and shapes that run whole (decode,
-fp32, short prefill); the chunked case is also checked against the oracle on
-sampled rows, and the full 128K prefill in the configuration the end-to-end
-benchmark times."""
+sequences split into query chunks (several chunks, two sequences, T < S with
+T not a multiple of the block, a piece under 128 queries merged into the
+next, one KV group) and shapes that run whole (decode, fp32, short prefill);
+the chunked case is also checked against the oracle on sampled rows and both
+sides of every chunk boundary, and the full 128K prefill in the configuration
+the end-to-end benchmark times."""
 import pytest
 import torch
 
@@ -27,12 +28,16 @@ def _case(name):
     W = _synth().Workload
     bf = torch.bfloat16
     return {
-        # chunks of 4096 queries ending at 10240, 6144, 2048 in each of two sequences
+        # pieces [0, 512), [512, 4608), [4608, 8704), [8704, 9216), [9216, 10240)
+        # of each of two sequences
         "chunked_B2": W("chunked_B2", B=2, T=10240, S=10240, Hq=16, Hkv=2, d=128, d_idx=64,
                         block=128, topk=8, dtype=bf, hot_blocks_per_group=3),
-        # T < S; the first chunk (40 queries) is folded into the next one
-        "chunked_fold_T_lt_S": W("chunked_fold_T_lt_S", B=1, T=8232, S=8320, Hq=8, Hkv=2,
-                                 d=128, d_idx=64, block=64, topk=6, dtype=bf),
+        # T < S, T % block = 40: pieces [0, 552), [552, 4648), [4648, 7208), [7208, 8232)
+        "chunked_T_lt_S_offset": W("chunked_T_lt_S_offset", B=1, T=8232, S=8320, Hq=8, Hkv=2,
+                                   d=128, d_idx=64, block=64, topk=6, dtype=bf),
+        # one KV group; the 64-query piece [4608, 4672) merges into [4672, 5696)
+        "chunked_merge_G1": W("chunked_merge_G1", B=1, T=5696, S=5696, Hq=8, Hkv=1, d=128,
+                              d_idx=64, block=64, topk=6, dtype=bf),
         "whole_decode": W("whole_decode", B=4, T=1, S=8192, Hq=32, Hkv=8, d=128, d_idx=64,
                           block=64, topk=8, dtype=bf),
         "whole_fp32": _synth().WORKLOADS["tiny_fp32_prefill"],
@@ -65,8 +70,9 @@ def _run_both(w, seed=0):
     return inp, (O, lse, ids), (hO, hlse, hids)
 
 
-@pytest.mark.parametrize("name", ["chunked_B2", "chunked_fold_T_lt_S", "whole_decode",
-                                  "whole_fp32", "whole_short_prefill", "prefill_128k"])
+@pytest.mark.parametrize("name", ["chunked_B2", "chunked_T_lt_S_offset", "chunked_merge_G1",
+                                  "whole_decode", "whole_fp32", "whole_short_prefill",
+                                  "prefill_128k"])
 def test_host_call_equals_forward(name):
     w = _case(name)
     torch.cuda.empty_cache()
@@ -78,7 +84,8 @@ def test_host_call_equals_forward(name):
         f"{name}: O differs"
     if name == "chunked_B2":
         # sampled rows plus both sides of every chunk boundary
-        edges = [b * w.T + t for b in range(w.B) for t in (2047, 2048, 6143, 6144)]
+        edges = [b * w.T + t for b in range(w.B)
+                 for t in (511, 512, 4607, 4608, 8703, 8704, 9215, 9216)]
         rows = sorted(set(_synth().sample_rows(w, 24)) | set(edges))
         ref = parity.oracle_rows(inp, w, rows)
         parity.assert_ids_equal(parity.gather_rows(hids, rows, w.T), ref["ids"], name)
