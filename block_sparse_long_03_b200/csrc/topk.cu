@@ -11,12 +11,15 @@
 // order-preserving uint32 -- nothing is exponentiated.
 //
 // One warp per row.  The candidates' ordered keys are staged in shared
-// memory, then a 4-pass radix select (8 bits per pass, warp-private
-// histogram) finds the M-th largest score u*.  Every candidate above u* is
-// kept, and of the candidates equal to u* the lowest ids are kept until M is
-// reached.  A final pass in ascending id order emits the kept ids with
-// ballots, so the output is ascending without a sort; cb is appended last
-// (it is larger than every candidate) and unused slots get -1.
+// memory.  For M <= 64 a lower bound of the M-th largest score (the M-th
+// largest of the lanes' top-2 keys) usually leaves at most 64 candidates;
+// those are compacted in id order and the M-th largest score u* among them
+// is found bit by bit with warp ballots.  Otherwise a 4-pass radix select
+// (8 bits per pass, warp-private histogram) over all candidates finds u*.
+// Every candidate above u* is kept, and of the candidates equal to u* the
+// lowest ids are kept until M is reached.  The kept ids are emitted in
+// ascending id order with ballots, so the output needs no sort; cb is
+// appended last (it is larger than every candidate) and unused slots get -1.
 #include "msa_internal.cuh"
 
 namespace msa {
@@ -51,8 +54,78 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
         return;
     }
     const float *row = bs + r * NB;
-    for (int n = lane; n < cb; n += 32) keys[n] = ordered_key(row[n]);
+    uint32_t b1 = 0u, b2 = 0u;        // this lane's two largest keys (0: none)
+    for (int n = lane; n < cb; n += 32) {
+        const uint32_t v = ordered_key(row[n]);
+        keys[n] = v;
+        b2 = max(b2, min(v, b1));
+        b1 = max(b1, v);
+    }
     __syncwarp();
+
+    if (M <= 64) {
+        // A lower bound tau of the M-th largest key: the M-th largest of the 64
+        // per-lane top-2 keys (a subset of the candidates), found on its top 16
+        // bits (truncating only lowers it).  Every one of the M best candidates
+        // has key >= tau, and on these scores few others do.
+        uint32_t tau = 0u;
+        for (int bit = 31; bit >= 16; --bit) {
+            const uint32_t c = tau | (1u << bit);
+            const int cnt = __popc(__ballot_sync(0xffffffffu, b1 >= c)) +
+                            __popc(__ballot_sync(0xffffffffu, b2 >= c));
+            if (cnt >= M) tau = c;
+        }
+        // candidates with key >= tau, compacted in ascending id order
+        uint32_t *ck = hist, *ci = hist + 64;
+        int C = 0;
+        for (int base = 0; base < cb; base += 32) {
+            const int n = base + lane;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool f = n < cb && v >= tau;
+            const unsigned fb = __ballot_sync(0xffffffffu, f);
+            const int pos = C + __popc(fb & lt_mask);
+            if (f && pos < 64) {
+                ck[pos] = v;
+                ci[pos] = (uint32_t)n;
+            }
+            C += __popc(fb);
+        }
+        __syncwarp();
+        if (C <= 64) {
+            // the exact M-th largest key u* among the candidates (= over the
+            // row), bit by bit below the bits all candidates share
+            const bool ok0 = lane < C, ok1 = lane + 32 < C;
+            const uint32_t k0 = ok0 ? ck[lane] : 0u, k1 = ok1 ? ck[lane + 32] : 0u;
+            const uint32_t all1 = __reduce_and_sync(0xffffffffu, ok0 ? k0 : 0xffffffffu) &
+                                  __reduce_and_sync(0xffffffffu, ok1 ? k1 : 0xffffffffu);
+            const uint32_t any1 = __reduce_or_sync(0xffffffffu, ok0 ? k0 : 0u) |
+                                  __reduce_or_sync(0xffffffffu, ok1 ? k1 : 0u);
+            const uint32_t diff = all1 ^ any1;
+            const int top = diff ? 31 - __clz((int)diff) : -1;
+            uint32_t u = top >= 0 ? all1 & ~((2u << top) - 1u) : all1;
+            for (int bit = top; bit >= 0; --bit) {
+                const uint32_t c = u | (1u << bit);
+                const int cnt = __popc(__ballot_sync(0xffffffffu, ok0 && k0 >= c)) +
+                                __popc(__ballot_sync(0xffffffffu, ok1 && k1 >= c));
+                if (cnt >= M) u = c;
+            }
+            // all candidates above u*, then the ties at u* with the lowest ids
+            const int gt = __popc(__ballot_sync(0xffffffffu, ok0 && k0 > u)) +
+                           __popc(__ballot_sync(0xffffffffu, ok1 && k1 > u));
+            const int need = M - gt;
+            const unsigned e0 = __ballot_sync(0xffffffffu, ok0 && k0 == u);
+            const unsigned e1 = __ballot_sync(0xffffffffu, ok1 && k1 == u);
+            const bool t0 = ok0 && (k0 > u || (k0 == u && __popc(e0 & lt_mask) < need));
+            const bool t1 = ok1 && (k1 > u || (k1 == u && __popc(e0) + __popc(e1 & lt_mask) < need));
+            const unsigned tb0 = __ballot_sync(0xffffffffu, t0);
+            const unsigned tb1 = __ballot_sync(0xffffffffu, t1);
+            if (t0) out[__popc(tb0 & lt_mask)] = (int32_t)ci[lane];
+            if (t1) out[__popc(tb0) + __popc(tb1 & lt_mask)] = (int32_t)ci[lane + 32];
+            if (lane == 0) out[M] = cb;
+            return;
+        }
+        __syncwarp();                 // the radix select below reuses hist
+    }
 
     uint32_t prefix = 0, mask = 0;
     int remaining = M;                // how many still to take at or below prefix
