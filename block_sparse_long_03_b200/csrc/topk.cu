@@ -55,11 +55,19 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
     }
     const float *row = bs + r * NB;
     uint32_t b1 = 0u, b2 = 0u;        // this lane's two largest keys (0: none)
-    for (int n = lane; n < cb; n += 32) {
-        const uint32_t v = ordered_key(row[n]);
-        keys[n] = v;
-        b2 = max(b2, min(v, b1));
-        b1 = max(b1, v);
+    for (int n0 = lane; n0 < cb; n0 += 128) {
+        float f[4];                   // four loads in flight per lane
+#pragma unroll
+        for (int u = 0; u < 4; ++u) f[u] = n0 + 32 * u < cb ? row[n0 + 32 * u] : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (n0 + 32 * u < cb) {
+                const uint32_t v = ordered_key(f[u]);
+                keys[n0 + 32 * u] = v;
+                b2 = max(b2, min(v, b1));
+                b1 = max(b1, v);
+            }
+        }
     }
     __syncwarp();
 
