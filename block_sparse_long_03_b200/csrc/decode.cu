@@ -211,29 +211,16 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     const int64_t p = (int64_t)S - T_ + t;
     const int cb = (int)(p / BLOCK);
     const int32_t *row = ids + rg * topk;
-    // validity of this slot (same rule as every other phase)
+    // validity of this slot (same rule as every other phase): the range is
+    // checked before the block's copies are issued, repeats while they fly
     const int n = row[slot];
     if (n < 0) return;
-    bool repeat = false;
-    {
-        int prev = -1;
-        bool asc = true;
-        for (int i = 0; i < topk; ++i) {
-            const int v = row[i];
-            if (v < 0) continue;
-            if (v <= prev) asc = false;
-            prev = v;
-        }
-        if (!asc)
-            for (int i = 0; i < slot; ++i) repeat |= row[i] == n;
-    }
-    if (n >= NB || repeat) {
+    if (n >= NB) {
         if (threadIdx.x == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
         return;
     }
-    if (n > cb) return;                                    // no causal token
     const int64_t j0 = (int64_t)n * BLOCK;
-    const int nk = (int)((p - j0 + 1 < BLOCK) ? (p - j0 + 1) : BLOCK);
+    const int nk = (int)((p - j0 + 1 < BLOCK) ? (p - j0 + 1) : BLOCK);   // <= 0 past cb
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int g4 = lane / 4, t4 = lane % 4;
@@ -250,6 +237,17 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
         }
     }
     cp_async_commit();
+    // an id repeated within the row counts once: later slots are reported and skipped
+    bool repeat = false;
+    for (int i0 = 0; i0 < slot; i0 += 32) {
+        const int i = i0 + lane;
+        repeat |= __any_sync(0xffffffffu, i < slot && row[i] == n);
+    }
+    if (repeat || n > cb) {                                // n > cb: no causal token
+        cp_async_wait<0>();                                // this CTA's copies land first
+        if (repeat && threadIdx.x == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+        return;
+    }
     // B fragments of Q^T: column g4 = head (zero past R)
     uint32_t bq[D / 16][2];
 #pragma unroll

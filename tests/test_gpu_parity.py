@@ -133,11 +133,13 @@ def test_topk_heavy_ties_and_closed_form():
             assert np.all(ids[0, t, g, len(want):] == -1)
 
 
-def test_sparse_attn_permuted_and_bad_ids():
+@pytest.mark.parametrize("name", ["bf16_chunk_ragged", "bf16_decode_small", "bf16_decode_T4"])
+def test_sparse_attn_permuted_and_bad_ids(name):
     """Caller ids in any order give the same result; ids out of range or
-    repeated are skipped and reported through the device error word."""
+    repeated are skipped and reported through the device error word (the
+    tensor-core prefill path and the decode path)."""
     msa = _msa()
-    w = _case("bf16_chunk_ragged")
+    w = _case(name)
     inp = _inputs(w, seed=5)
     O, lse, ids, ws = msa.forward(inp.q_idx, inp.k_idx, inp.Q, inp.K, inp.V, block=w.block,
                                   topk=w.topk)
