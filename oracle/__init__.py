@@ -7,8 +7,10 @@ library never calls it and shares no code with it.
 The arithmetic lives in ``msa_oracle.c`` (plain C, fp64, OpenMP over rows),
 which follows "MiniMax Sparse Attention -- paper by Lai et al. (2026)",
 section "Summary" (index branch, per-group Top-k with the current block
-kept, exact softmax over the kept blocks) and section "Key points" (k blocks
-of B_k tokens give k * B_k attended tokens; LSE is a forward output).  This
+kept, exact softmax over the kept blocks, and the group-averaged Main
+Branch distribution the indexer's KL objective matches) and section "Key
+points" (k blocks of B_k tokens give k * B_k attended tokens; LSE is a
+forward output).  This
 module only marshals arrays into that C code.
 
 Every function works on a list of rows ``r = b * T + t`` so that large
@@ -48,8 +50,9 @@ def bind(path: str):
     lib.oracle_select_blocks.argtypes = [i64] * 5 + [vp, vp, i64, vp]
     lib.oracle_attention.argtypes = [i64] * 8 + [i32, dbl, vp, vp, vp, vp, vp, i64, vp, vp]
     lib.oracle_forward.argtypes = [i64] * 9 + [i32, dbl] + [vp] * 6 + [i64, vp, vp, vp, vp]
+    lib.oracle_block_mass.argtypes = [i64] * 8 + [i32, dbl, vp, vp, vp, vp, vp, i64, vp]
     for f in (lib.oracle_block_scores, lib.oracle_select_blocks, lib.oracle_attention,
-              lib.oracle_forward, lib.oracle_num_threads):
+              lib.oracle_forward, lib.oracle_block_mass, lib.oracle_num_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -150,6 +153,29 @@ def attention(Q_rows, K, V, ids, rows, *, T: int, block: int, scale: float = 0.0
     if rc != 0:
         raise ValueError(f"oracle_attention failed ({rc})")
     return O, lse
+
+
+def block_mass(Q_rows, K, ids, lse, rows, *, T: int, block: int, scale: float = 0.0,
+               lib=None) -> np.ndarray:
+    """Target of the indexer's KL objective: [nrows, G, topk] fp64, the mass
+    of each kept slot's block under the row's softmax (normalised by the
+    stored `lse` [nrows, Hq]), averaged over the heads of the group."""
+    q, dt = _as_raw(Q_rows)
+    k, dtk = _as_raw(K)
+    assert dt == dtk, "Q and K must share a dtype"
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    lse = np.ascontiguousarray(lse, dtype=np.float64)
+    r = _rows(rows)
+    nrows, Hq, d = q.shape
+    B, S, Hkv, _ = k.shape
+    topk = ids.shape[-1]
+    out = np.empty((nrows, Hkv, topk), np.float64)
+    rc = (lib or _load()).oracle_block_mass(B, T, S, Hq, Hkv, d, block, topk, dt, float(scale),
+                                            _ptr(q), _ptr(k), _ptr(ids), _ptr(lse), _ptr(r),
+                                            nrows, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_block_mass failed ({rc})")
+    return out
 
 
 def forward(q_idx_rows, k_idx, Q_rows, K, V, rows, *, T: int, block: int, topk: int,

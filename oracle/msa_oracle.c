@@ -293,6 +293,80 @@ int oracle_attention(int64_t B, int64_t T, int64_t S, int64_t Hq, int64_t Hkv,
 }
 
 /*
+ * Target of the indexer's KL objective ("MiniMax Sparse Attention",
+ * Summary, second paragraph: the indexer learns to match the Main Branch's
+ * distribution averaged over the heads of a GQA group; Key points, kernel
+ * design: the LSE that loss needs is a forward output).  For row r (query t
+ * at position p), group g and kept slot i holding block n = ids[ri, g, i]:
+ *   mass[ri, g, i] = (1 / R) * sum over heads h of g of
+ *                    sum over tokens j of block n with j <= p of
+ *                    exp(s_hj - lse[ri, h])
+ * with s_hj = scale * Q[b, t, h] . K[b, j, g] as in oracle_attention and
+ * lse the stored LSE of that row and head.  An empty slot (-1) gets 0, and
+ * a head whose lse is -inf adds 0.  With the LSE of the same kept set, a
+ * row's masses over its slots sum to 1.  Ids outside [0, NB) or listed
+ * twice are an error (-3), as in oracle_attention.
+ */
+int oracle_block_mass(int64_t B, int64_t T, int64_t S, int64_t Hq, int64_t Hkv,
+                      int64_t d, int64_t block, int64_t topk, int dtype, double scale,
+                      const void *Q_rows, const void *K, const int32_t *ids,
+                      const double *lse, const int64_t *rows, int64_t nrows, double *mass)
+{
+    if (B <= 0 || T <= 0 || S <= 0 || T > S || Hq <= 0 || Hkv <= 0 ||
+        Hq % Hkv != 0 || d <= 0 || block <= 0 || topk <= 0 || nrows < 0 ||
+        (dtype != ORACLE_F32 && dtype != ORACLE_BF16))
+        return -1;
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    const int64_t NB = ceil_div(S, block);
+    const int64_t R = Hq / Hkv;
+    int bad = 0;
+#pragma omp parallel
+    {
+        unsigned char *seen = (unsigned char *)calloc((size_t)NB, 1);
+        if (!seen) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t ri = 0; ri < nrows; ++ri) {
+            if (!seen) continue;
+            const int64_t r = rows[ri];
+            if (r < 0 || r >= B * T) { bad = 1; continue; }
+            const int64_t b = r / T, t = r % T;
+            const int64_t p = query_pos(T, S, t);
+            for (int64_t g = 0; g < Hkv; ++g) {
+                const int32_t *kept = ids + (ri * Hkv + g) * topk;
+                double *out = mass + (ri * Hkv + g) * topk;
+                memset(seen, 0, (size_t)NB);
+                for (int64_t i = 0; i < topk; ++i) {
+                    out[i] = 0.0;
+                    const int64_t n = kept[i];
+                    if (n < 0) continue;
+                    if (n >= NB || seen[n]) { bad = 3; continue; }
+                    seen[n] = 1;
+                    const int64_t first = n * block;
+                    const int64_t stop = (n + 1) * block < S ? (n + 1) * block : S;
+                    double head_sum = 0.0;
+                    for (int64_t hh = 0; hh < R; ++hh) {
+                        const int64_t h = g * R + hh;           /* head hh of group g */
+                        const double l = lse[ri * Hq + h];
+                        if (l == -INFINITY) continue;
+                        for (int64_t j = first; j < stop; ++j) {
+                            if (j > p) break;                   /* causal tokens only */
+                            double dot = 0.0;
+                            for (int64_t c = 0; c < d; ++c)
+                                dot += widen(Q_rows, dtype, (ri * Hq + h) * d + c) *
+                                       widen(K, dtype, ((b * S + j) * Hkv + g) * d + c);
+                            head_sum += exp(scale * dot - l);
+                        }
+                    }
+                    out[i] = head_sum / (double)R;
+                }
+            }
+        }
+        free(seen);
+    }
+    return bad ? -bad : 0;
+}
+
+/*
  * The whole forward pass for a list of rows: index scores, selection, then
  * attention.  ids_out [nrows, G, topk] (int32), O [nrows, Hq, d] and
  * lse [nrows, Hq] (double).  bs_out may be NULL; otherwise it receives the

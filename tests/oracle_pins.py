@@ -17,7 +17,10 @@ and mathematics fix:
   {0..k-2} plus the current one; constant values give a constant output; a
   single attended key gives that key's value; LSE brackets;
 * exactness of the inputs' grid: bf16 and fp32 copies of the same grid
-  values give bit-identical oracle results.
+  values give bit-identical oracle results;
+* the indexer's KL target (Summary: the indexer matches the group-averaged
+  Main Branch distribution): torch's masked softmax summed per block and
+  averaged over the group's heads, sum-to-one, and the equal-scores share.
 
 Inputs are small (a few hundred tokens) so every pin runs in well under a
 second on CPU.
@@ -264,5 +267,76 @@ def pin_bf16_widening(lib):
         assert np.array_equal(x, y), "bf16 and fp32 copies of the same values disagree"
 
 
+def _torch_block_mass(Q, K, allowed, scale, ids, block):
+    """Head-averaged softmax mass of each kept slot's block from torch (fp64):
+    softmax over the allowed tokens of the full score matrix, summed over the
+    block's tokens, averaged over the group's heads.  [B*T, Hkv, topk]."""
+    B, T, Hq, d = Q.shape
+    S, Hkv = K.shape[1], K.shape[2]
+    R = Hq // Hkv
+    q = torch.from_numpy(Q.astype(np.float64)).permute(0, 2, 1, 3)           # B Hq T d
+    k = torch.from_numpy(K.astype(np.float64)).permute(0, 2, 1, 3).repeat_interleave(R, dim=1)
+    m = torch.from_numpy(allowed).permute(0, 2, 1, 3)                        # B Hq T S
+    s = ((q @ k.transpose(-1, -2)) * scale).masked_fill(~m, float("-inf"))
+    probs = torch.nan_to_num(torch.softmax(s, dim=-1)).numpy()               # B Hq T S
+    tok_block = np.arange(S) // block
+    out = np.zeros((B * T, Hkv, ids.shape[-1]))
+    for b in range(B):
+        for t in range(T):
+            for g in range(Hkv):
+                for i, n in enumerate(ids[b * T + t, g]):
+                    if n >= 0:
+                        out[b * T + t, g, i] = probs[b, g * R:(g + 1) * R, t][:, tok_block == n] \
+                            .sum(axis=1).mean()
+    return out
+
+
+def pin_block_mass(lib):
+    """The indexer's KL target (head-averaged block mass under the stored
+    LSE) equals torch's masked softmax summed per block, for the dense limit
+    and for sparse kept sets; it sums to 1 per row and group; with all
+    scores equal it is the block's share of the attended tokens; with every
+    head's LSE at -inf it is 0."""
+    rng = np.random.default_rng(29)
+    for B, T, S, Hq, Hkv, d, d_idx, block, k in [(1, 40, 40, 4, 2, 8, 4, 8, 5),
+                                                (2, 24, 72, 6, 3, 16, 4, 8, 3),
+                                                (1, 64, 64, 8, 2, 8, 4, 8, 2)]:
+        NB = -(-S // block)
+        Q = rng.standard_normal((B, T, Hq, d)).astype(np.float32)
+        K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+        V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+        rows = _rows_all(B, T)
+        Qr = Q.reshape(B * T, Hq, d)
+        q_idx = _grid(rng, (B * T, Hkv, d_idx))
+        k_idx = _grid(rng, (B, S, d_idx))
+        for topk in (NB, k):                      # dense limit, then a sparse kept set
+            ids, O, lse = orc.forward(q_idx, k_idx, Qr, K, V, rows, T=T, block=block,
+                                      topk=topk, lib=lib)
+            mass = orc.block_mass(Qr, K, ids, lse, rows, T=T, block=block, lib=lib)
+            allowed = _allowed_from_ids(ids, B, T, S, Hq, Hkv, block)
+            ref = _torch_block_mass(Q, K, allowed, 1.0 / np.sqrt(d), ids, block)
+            np.testing.assert_allclose(mass, ref, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(mass.sum(-1), 1.0, rtol=0, atol=1e-12)
+            assert np.all(mass[ids < 0] == 0.0)
+        # all scores equal (K = 0): each kept block holds its share of the attended tokens
+        K0 = np.zeros_like(K)
+        ids, O, lse = orc.forward(q_idx, k_idx, Qr, K0, V, rows, T=T, block=block, topk=k,
+                                  lib=lib)
+        mass = orc.block_mass(Qr, K0, ids, lse, rows, T=T, block=block, lib=lib)
+        for ri in range(B * T):
+            p = S - T + ri % T
+            for g in range(Hkv):
+                kept = ids[ri, g]
+                count = {n: min(p + 1, (n + 1) * block, S) - n * block for n in kept if n >= 0}
+                total = sum(count.values())
+                for i, n in enumerate(kept):
+                    want = count[n] / total if n >= 0 else 0.0
+                    assert abs(mass[ri, g, i] - want) < 1e-15, (ri, g, i)
+        # no attended key anywhere (every LSE -inf): no mass
+        none = orc.block_mass(Qr, K, ids, np.full_like(lse, -np.inf), rows, T=T, block=block,
+                              lib=lib)
+        assert np.all(none == 0.0)
+
+
 ALL_PINS = [pin_brute_force_selection, pin_dense_limit, pin_masked_attention,
-            pin_closed_forms, pin_permutation_invariance, pin_bf16_widening]
+            pin_closed_forms, pin_permutation_invariance, pin_bf16_widening, pin_block_mass]

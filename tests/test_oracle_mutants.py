@@ -35,6 +35,11 @@ MUTANTS = {
     "values_read_from_keys": ("o[c] += w * widen(V, dtype,", "o[c] += w * widen(K, dtype,"),
     "bf16_widening_shift": ("<< 16;", "<< 15;"),
     "softmax_sign": ("const double w = exp(s[q] - m);", "const double w = exp(m - s[q]);"),
+    "mass_not_head_averaged": ("out[i] = head_sum / (double)R;", "out[i] = head_sum;"),
+    "mass_not_causal": ("if (j > p) break;                   /* causal tokens only */",
+                        "if (j > S) break;"),
+    "mass_wrong_head_of_group": ("const int64_t h = g * R + hh;", "const int64_t h = hh * Hkv + g;"),
+    "mass_unscaled_scores": ("head_sum += exp(scale * dot - l);", "head_sum += exp(dot - l);"),
 }
 # "current_block_not_forced" needs a two-part edit: candidates include cb and
 # the forced append is dropped.
