@@ -238,11 +238,20 @@ class Problem:
         self.ws = msa.alloc_workspace(self.params, msa.MSA_WS_FORWARD)
         self.ws_attn = msa.alloc_workspace(self.params, msa.MSA_WS_SPARSE_ATTN)
         self.bs = torch.empty((w.B, w.T, w.G, w.NB), dtype=torch.float32, device="cuda")
+        self.mass = None
 
     def step(self, stream=None):
         i = self.inp
         self.msa.msa_forward(self.params, i.q_idx, i.k_idx, i.Q, i.K, i.V, self.ids, self.O,
                              self.lse, self.ws, stream)
+
+    def step_mass(self, stream=None):
+        """The forward pass plus the indexer's KL target (msa_forward_mass)."""
+        i, w = self.inp, self.w
+        if self.mass is None:
+            self.mass = torch.empty((w.B, w.T, w.G, w.topk), dtype=torch.float32, device="cuda")
+        self.msa.msa_forward_mass(self.params, i.q_idx, i.k_idx, i.Q, i.K, i.V, self.ids, self.O,
+                                  self.lse, self.mass, self.ws, stream)
 
     def stage_times_ms(self, reps: int) -> dict:
         """Average device time of each call of the path, launched on its own."""
@@ -268,7 +277,7 @@ class Problem:
         return out
 
     def free(self):
-        for f in ("inp", "O", "lse", "ids", "ws", "ws_attn", "bs"):
+        for f in ("inp", "O", "lse", "ids", "ws", "ws_attn", "bs", "mass"):
             setattr(self, f, None)
         torch.cuda.empty_cache()
 
@@ -444,6 +453,12 @@ def run_ours(args, rank: int, ws: int):
                 "frac": (partial_floor_bytes(w) / (pk["hbm_gbs"] * 1e9) * 1e3)
                         / stages["sparse_attn_fwd"]},
             "index_tflops": idx_fl / (stages["index_block_scores"] / 1e3) / 1e12}
+    # the indexer's KL target as a third output of the same pass
+    kl_ms = time_steps(prob.step_mass, args.steps, args.warmup, ws)
+    ref_ms = time_steps(prob.step, args.steps, args.warmup, ws)    # adjacent, same clocks
+    kl = {"call": "msa_forward_mass", "ms_per_step": kl_ms, "extra_ms": kl_ms - ref_ms,
+          "value": aggregate_tokens_per_s(w.B * w.T, kl_ms, ws), "unit": "tokens/s",
+          "mass_bytes": int(prob.mass.numel() * 4)}
     e2e = None if args.no_e2e else e2e_prefill(prob, max(1, min(args.steps, 3)), 1, ws)
     prob.free()
     del prob
@@ -478,7 +493,7 @@ def run_ours(args, rank: int, ws: int):
                        "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx, "block": w.block,
                        "topk": w.topk, "parallelism": f"replicas x{ws}",
                        "l2": "inputs larger than L2 (Q alone 2 GiB); no flush"},
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "kl_target": kl,
             "gpu_launches": int(round(per_step * args.steps)),
             "clocks": clk.summary(), "decode": decode,
         }

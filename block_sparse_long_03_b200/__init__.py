@@ -7,7 +7,8 @@ in ``include/msa.h``); this package is its Python binding.
 """
 from .binding import (EXPORTS, MSA_BF16, MSA_F32, MSA_OK, MSA_WS_FORWARD, MSA_WS_FORWARD_HOST,
                       MSA_WS_SPARSE_ATTN, MsaError, Params, alloc_workspace, forward,
-                      index_block_scores, make_params, msa_forward, msa_forward_host,
+                      forward_with_mass, index_block_scores, make_params, msa_forward,
+                      msa_forward_host, msa_forward_mass, msa_sparse_attn_fwd_mass,
                       msa_get_device_error, msa_index_block_scores,
                       msa_kernel_launches, msa_selftest_wait_timeout,
                       msa_sparse_attn_fwd, msa_topk_blocks, msa_workspace_size, params_from,
@@ -16,7 +17,8 @@ from .binding import (EXPORTS, MSA_BF16, MSA_F32, MSA_OK, MSA_WS_FORWARD, MSA_WS
 __all__ = [
     "EXPORTS", "MSA_BF16", "MSA_F32", "MSA_OK", "MSA_WS_FORWARD", "MSA_WS_FORWARD_HOST",
     "MSA_WS_SPARSE_ATTN", "MsaError", "Params", "alloc_workspace", "forward",
-    "index_block_scores", "make_params", "msa_forward", "msa_forward_host",
+    "forward_with_mass", "index_block_scores", "make_params", "msa_forward", "msa_forward_host",
+    "msa_forward_mass", "msa_sparse_attn_fwd_mass",
     "msa_get_device_error", "msa_index_block_scores", "msa_kernel_launches",
     "msa_selftest_wait_timeout", "msa_sparse_attn_fwd",
     "msa_topk_blocks", "msa_workspace_size", "params_from", "sparse_attn_fwd", "status_string",

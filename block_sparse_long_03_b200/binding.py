@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
            "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
-           "msa_selftest_wait_timeout")
+           "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass")
 
 
 class MsaError(RuntimeError):
@@ -62,6 +62,10 @@ def _load():
     lib.msa_forward_noalloc.restype = st
     lib.msa_forward_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_forward_host.restype = st
+    lib.msa_sparse_attn_fwd_mass.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_sparse_attn_fwd_mass.restype = st
+    lib.msa_forward_mass.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.msa_forward_mass.restype = st
     lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.msa_selftest_wait_timeout.restype = st
     lib.msa_kernel_launches.argtypes = []
@@ -143,6 +147,25 @@ def msa_forward(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, worksp
                            workspace.numel(), _stream(stream)), "msa_forward")
 
 
+def msa_sparse_attn_fwd_mass(params: Params, Q, K, V, block_ids, O, lse, block_mass, workspace,
+                             stream=None):
+    """msa_sparse_attn_fwd plus block_mass [B, T, G, topk] fp32: each kept slot's share of
+    the row's softmax averaged over the group's heads (the indexer's KL target)."""
+    _check(lib.msa_sparse_attn_fwd_mass(ctypes.byref(params), _ptr(Q), _ptr(K), _ptr(V),
+                                        _ptr(block_ids), _ptr(O), _ptr(lse), _ptr(block_mass),
+                                        _ptr(workspace), workspace.numel(), _stream(stream)),
+           "msa_sparse_attn_fwd_mass")
+
+
+def msa_forward_mass(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, block_mass,
+                     workspace, stream=None):
+    """msa_forward plus block_mass (see msa_sparse_attn_fwd_mass)."""
+    _check(lib.msa_forward_mass(ctypes.byref(params), _ptr(q_idx), _ptr(k_idx), _ptr(Q),
+                                _ptr(K), _ptr(V), _ptr(block_ids), _ptr(O), _ptr(lse),
+                                _ptr(block_mass), _ptr(workspace), workspace.numel(),
+                                _stream(stream)), "msa_forward_mass")
+
+
 def msa_forward_host(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, device_buffer,
                      stream=None):
     """msa_forward on page-locked host tensors (``pin_memory()``); the copies to
@@ -214,3 +237,16 @@ def forward(q_idx, k_idx, Q, K, V, *, block: int, topk: int, scale: float = 0.0)
     ws = alloc_workspace(p, MSA_WS_FORWARD, Q.device)
     msa_forward(p, q_idx, k_idx, Q, K, V, ids, O, lse, ws)
     return O, lse, ids, ws
+
+
+def forward_with_mass(q_idx, k_idx, Q, K, V, *, block: int, topk: int, scale: float = 0.0):
+    """The whole forward pass plus the indexer's KL target; returns
+    (O, lse, block_ids, block_mass, workspace)."""
+    p = params_from(q_idx, Q, K, block=block, topk=topk, scale=scale)
+    O = torch.empty_like(Q)
+    lse = torch.empty(Q.shape[:3], dtype=torch.float32, device=Q.device)
+    ids = torch.empty((*Q.shape[:2], K.shape[2], topk), dtype=torch.int32, device=Q.device)
+    mass = torch.empty((*Q.shape[:2], K.shape[2], topk), dtype=torch.float32, device=Q.device)
+    ws = alloc_workspace(p, MSA_WS_FORWARD, Q.device)
+    msa_forward_mass(p, q_idx, k_idx, Q, K, V, ids, O, lse, mass, ws)
+    return O, lse, ids, mass, ws

@@ -11,7 +11,9 @@
 // which share the kept set.  Each kept block is staged in shared memory
 // (fp32), thread j scores key j against all R heads, a warp per head
 // updates that head's running max / normaliser (online softmax), and
-// thread c accumulates output channel c for all R heads.
+// thread c accumulates output channel c for all R heads.  On request it also
+// writes each kept slot's head-averaged share of the softmax (the indexer's
+// KL target), from per-block sums kept with the maxima they were taken at.
 #include <math.h>
 
 #include "msa_internal.cuh"
@@ -23,12 +25,12 @@ constexpr int kThreads = 128;
 constexpr int kMaxR = 16;
 constexpr int kMaxTopk = 256;
 
-template <typename T>
+template <typename T, bool kMass>
 __global__ void __launch_bounds__(kThreads)
 attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V,
                  const int32_t *__restrict__ ids, T *__restrict__ O, float *__restrict__ lse,
-                 uint32_t *err, int T_, int S, int Hq, int Hkv, int d, int block, int topk,
-                 int NB, float scale) {
+                 float *__restrict__ mass, uint32_t *err, int T_, int S, int Hq, int Hkv, int d,
+                 int block, int topk, int NB, float scale) {
     extern __shared__ float sm[];
     const int g = blockIdx.x % Hkv;
     const int64_t bt = blockIdx.x / Hkv;          // b * T + t
@@ -43,7 +45,10 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
     float *m_s = ss + R * block;                   // [R] running max
     float *l_s = m_s + kMaxR;                      // [R] running normaliser
     float *a_s = l_s + kMaxR;                      // [R] rescale factor of this block
+    float *bsum = a_s + kMaxR;                     // [topk][R] block sums (for mass)
+    float *bmax = bsum + topk * R;                 // [topk][R] the maxima they are taken at
     __shared__ int kept[kMaxTopk];
+    __shared__ int kslot[kMaxTopk];                // slot of each kept block
     __shared__ int nkept;
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -56,6 +61,7 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
             bool bad = n >= NB;
             for (int k = 0; k < n_ok && !bad; ++k) bad = kept[k] == n;
             if (bad) { record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1); continue; }
+            kslot[n_ok] = i;
             kept[n_ok++] = n;
         }
         nkept = n_ok;
@@ -63,6 +69,8 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
     for (int i = tid; i < R * d; i += kThreads)
         qs[i] = to_f32(Q[(bt * Hq + (int64_t)g * R) * d + i]) * scale;
     if (tid < R) { m_s[tid] = -INFINITY; l_s[tid] = 0.f; }
+    if (kMass)
+        for (int i = tid; i < topk; i += kThreads) mass[(bt * Hkv + g) * topk + i] = 0.f;
     __syncthreads();
 
     float acc[kMaxR];
@@ -115,6 +123,10 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
                 a_s[h] = alpha;
                 l_s[h] = l_s[h] * alpha + sum;
                 m_s[h] = m_new;
+                if (kMass) {
+                    bsum[kb * R + h] = sum;
+                    bmax[kb * R + h] = m_new;
+                }
             }
         }
         __syncthreads();
@@ -143,30 +155,43 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
         const float l = l_s[tid];
         lse[bt * Hq + (int64_t)g * R + tid] = (l > 0.f) ? m_s[tid] + logf(l) : -INFINITY;
     }
+    if (kMass) {
+        // the indexer's KL target: each kept block's share of the softmax,
+        // averaged over the group's heads (blocks past p(t) keep 0)
+        for (int kb = tid; kb < nkept; kb += kThreads) {
+            if ((int64_t)kept[kb] * block > p) continue;
+            float share = 0.f;
+            for (int h = 0; h < R; ++h)
+                if (l_s[h] > 0.f) share += bsum[kb * R + h] * expf(bmax[kb * R + h] - m_s[h]) / l_s[h];
+            mass[(bt * Hkv + g) * topk + kslot[kb]] = share / (float)R;
+        }
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
-                             cudaStream_t st) {
+                             cudaStream_t st, float *mass) {
     if (s.R > kMaxR || s.topk > kMaxTopk || s.d > kThreads) return cudaErrorInvalidConfiguration;
     const size_t smem = sizeof(float) * ((size_t)s.block * (s.d + 1) + (size_t)s.block * s.d +
-                                         (size_t)s.R * s.d + (size_t)s.R * s.block + 3 * kMaxR);
+                                         (size_t)s.R * s.d + (size_t)s.R * s.block + 3 * kMaxR +
+                                         2 * (size_t)s.topk * s.R);
     const dim3 grid((unsigned)(s.rows() * s.Hkv));
     if (s.dtype == MSA_F32) {
-        auto k = attn_simt_kernel<float>;
+        auto k = mass ? attn_simt_kernel<float, true> : attn_simt_kernel<float, false>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, kThreads, smem, st>>>((const float *)Q, (const float *)K, (const float *)V, ids,
-                                        (float *)O, lse, err, s.T, s.S, s.Hq, s.Hkv, s.d,
+                                        (float *)O, lse, mass, err, s.T, s.S, s.Hq, s.Hkv, s.d,
                                         s.block, s.topk, s.NB, s.scale);
     } else {
-        auto k = attn_simt_kernel<__nv_bfloat16>;
+        auto k = mass ? attn_simt_kernel<__nv_bfloat16, true>
+                      : attn_simt_kernel<__nv_bfloat16, false>;
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<grid, kThreads, smem, st>>>((const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K,
                                         (const __nv_bfloat16 *)V, ids, (__nv_bfloat16 *)O, lse,
-                                        err, s.T, s.S, s.Hq, s.Hkv, s.d, s.block, s.topk, s.NB,
-                                        s.scale);
+                                        mass, err, s.T, s.S, s.Hq, s.Hkv, s.d, s.block, s.topk,
+                                        s.NB, s.scale);
     }
     count_launches(1);
     return cudaGetLastError();

@@ -721,6 +721,46 @@ combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_
     if (part == 0 && s0 == 0) lse[r * Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
 }
 
+// The indexer's KL target for query rows [r0, r0 + rc), run after their
+// merge: slot sl's share of head h's softmax is exp(part_lse - lse) of that
+// slot (0 for slots no tile served), averaged over the group's R heads.  One
+// warp per (row, group), lanes laid out as in the merge (head l % R, slots
+// l / R + k * 32 / R), so the head average is a shuffle over R lanes.
+__global__ void __launch_bounds__(256)
+block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ part_lse,
+                  const float *__restrict__ lse, float *__restrict__ mass, int64_t r0, int64_t rc,
+                  int T_, int S, int Hq, int G, int R, int NB, int block, int topk) {
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (x >= rc * G) return;
+    const int64_t rl = x / G, r = r0 + rl;
+    const int g = (int)(x % G);
+    const int t = (int)(r % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (topk + sstep - 1) / sstep;
+    const float l = lse[r * Hq + (int64_t)g * R + h];
+    const int64_t base = x * topk * R;
+    float *mrow = mass + (r * G + g) * topk;
+    constexpr int kMaxPer = 16;                     // per <= 16 wherever the merge runs
+    float li[kMaxPer];                              // every load issued before any use
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        const int sl = s0 + k * sstep;
+        const bool okk = __shfl_sync(0xffffffffu, sl < 32 ? sp.ok0 : sp.ok1, sl & 31);
+        li[k] = (k < per && sl < topk && okk) ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        if (k >= per) break;                        // per is uniform across the warp
+        const int sl = s0 + k * sstep;
+        float share = (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
+        for (int off = 1; off < R; off *= 2) share += __shfl_xor_sync(0xffffffffu, share, off);
+        if (h == 0 && sl < topk) mrow[sl] = share / (float)R;
+    }
+}
+
 constexpr size_t kPartialBudget = (size_t)4 << 30;   // bytes of partials per chunk
 constexpr size_t kA = 256;
 size_t al(size_t x) { return (x + kA - 1) / kA * kA; }
@@ -757,7 +797,7 @@ Plan make_plan(const Shape &s) {
 template <int D, int BLOCK>
 cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void *V,
                        const int32_t *ids, void *O, float *lse, uint32_t *err, char *ws,
-                       cudaStream_t st) {
+                       cudaStream_t st, float *mass) {
     const Plan pl = make_plan(s);
     CUtensorMap tq, tk, tv;
     const uint64_t dims[3] = {(uint64_t)s.d, (uint64_t)s.Hkv, (uint64_t)s.B * s.S};
@@ -819,7 +859,7 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         a.scale = s.scale;
         a.scale_log2 = s.scale * kLog2e;
         kern<<<sms, kThreads, smem, st>>>(tq, tk, tv, a);
-        e = launch_combine(s, ids, part_o, part_lse, O, lse, r0, rc, st);
+        e = launch_combine(s, ids, part_o, part_lse, O, lse, r0, rc, st, mass);
         if (e != cudaSuccess) return e;
         count_launches(5);
         e = cudaGetLastError();
@@ -832,19 +872,22 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
-                           cudaStream_t st) {
+                           cudaStream_t st, float *mass) {
     const int64_t warps = rc * s.G * (128 / 32);
     const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
     const int per = (s.topk + 32 / s.R - 1) / (32 / s.R);
-    if (per <= 8)
-        combine_kernel<128, 8><<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O, lse,
-                                                     r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
-                                                     s.block, s.topk);
-    else
-        combine_kernel<128, 16><<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O,
-                                                      lse, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
-                                                      s.block, s.topk);
+    auto kern = per <= 8 ? combine_kernel<128, 8> : combine_kernel<128, 16>;
+    kern<<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S,
+                               s.Hq, s.G, s.R, s.NB, s.block, s.topk);
     count_launches(1);
+    if (mass != nullptr) {
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const unsigned mgrid = (unsigned)((rc * s.G * 32 + 255) / 256);
+        block_mass_kernel<<<mgrid, 256, 0, st>>>(ids, part_lse, lse, mass, r0, rc, s.T, s.S, s.Hq,
+                                                 s.G, s.R, s.NB, s.block, s.topk);
+        count_launches(1);
+    }
     return cudaGetLastError();
 }
 
@@ -864,10 +907,10 @@ int64_t attn_tc_rows_per_pass(const Shape &s) { return make_plan(s).rows_per_chu
 
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, float *mass) {
     if (s.block == 128)
-        return run_chunks<128, 128>(s, Q, K, V, ids, O, lse, err, (char *)ws, st);
-    return run_chunks<128, 64>(s, Q, K, V, ids, O, lse, err, (char *)ws, st);
+        return run_chunks<128, 128>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass);
+    return run_chunks<128, 64>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass);
 }
 
 }  // namespace msa

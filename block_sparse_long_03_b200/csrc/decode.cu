@@ -446,14 +446,14 @@ size_t decode_attn_workspace(const Shape &s) {
 
 cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
                                const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                               cudaStream_t st) {
+                               cudaStream_t st, float *mass) {
     __half *part_o = (__half *)ws;
     float *part_lse = (float *)((char *)ws + part_bytes_o(s));
     cudaError_t e = s.block == 64
                         ? launch_block_t<64>(s, Q, K, V, ids, part_o, part_lse, err, st)
                         : launch_block_t<128>(s, Q, K, V, ids, part_o, part_lse, err, st);
     if (e != cudaSuccess) return e;
-    return launch_combine(s, ids, part_o, part_lse, O, lse, 0, s.rows(), st);
+    return launch_combine(s, ids, part_o, part_lse, O, lse, 0, s.rows(), st, mass);
 }
 
 }  // namespace msa

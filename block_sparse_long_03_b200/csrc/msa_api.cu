@@ -77,10 +77,11 @@ size_t forward_ws(const Shape &s) {
 
 cudaError_t launch_attention(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
-                             char *scratch, cudaStream_t st) {
-    if (use_attn_tc(s)) return launch_attn_tc(s, Q, K, V, ids, O, lse, err, scratch, st);
-    if (use_attn_decode(s)) return launch_decode_attn(s, Q, K, V, ids, O, lse, err, scratch, st);
-    return launch_attn_simt(s, Q, K, V, ids, O, lse, err, st);
+                             char *scratch, cudaStream_t st, float *mass = nullptr) {
+    if (use_attn_tc(s)) return launch_attn_tc(s, Q, K, V, ids, O, lse, err, scratch, st, mass);
+    if (use_attn_decode(s))
+        return launch_decode_attn(s, Q, K, V, ids, O, lse, err, scratch, st, mass);
+    return launch_attn_simt(s, Q, K, V, ids, O, lse, err, st, mass);
 }
 
 msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
@@ -141,12 +142,20 @@ msa_status_t msa_topk_blocks(const msa_params_t *params, const float *block_scor
 msa_status_t msa_sparse_attn_fwd(const msa_params_t *params, const void *Q, const void *K,
                                  const void *V, const int32_t *block_ids, void *O, float *lse,
                                  void *workspace, size_t workspace_bytes, void *stream) {
+    return msa_sparse_attn_fwd_mass(params, Q, K, V, block_ids, O, lse, nullptr, workspace,
+                                    workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_fwd_mass(const msa_params_t *params, const void *Q, const void *K,
+                                      const void *V, const int32_t *block_ids, void *O,
+                                      float *lse, float *block_mass, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
     Shape s;
     msa_status_t rc = make_shape(params, &s);
     if (rc != MSA_OK) return rc;
     if (!Q || !K || !V || !block_ids || !O || !lse) return MSA_ERR_INVALID_ARG;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(block_ids) ||
-        !aligned16(O) || !aligned16(lse))
+        !aligned16(O) || !aligned16(lse) || (block_mass && !aligned16(block_mass)))
         return MSA_ERR_INVALID_ARG;
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < attn_ws(s))
         return MSA_ERR_WORKSPACE;
@@ -154,7 +163,8 @@ msa_status_t msa_sparse_attn_fwd(const msa_params_t *params, const void *Q, cons
     uint32_t *err = (uint32_t *)workspace;
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
     if (e == cudaSuccess)
-        e = launch_attention(s, Q, K, V, block_ids, O, lse, err, (char *)workspace + kErrorBytes, st);
+        e = launch_attention(s, Q, K, V, block_ids, O, lse, err, (char *)workspace + kErrorBytes,
+                             st, block_mass);
     return cuda_status(e);
 }
 
@@ -162,13 +172,21 @@ msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const vo
                          const void *Q, const void *K, const void *V, int32_t *block_ids,
                          void *O, float *lse, void *workspace, size_t workspace_bytes,
                          void *stream) {
+    return msa_forward_mass(params, q_idx, k_idx, Q, K, V, block_ids, O, lse, nullptr, workspace,
+                            workspace_bytes, stream);
+}
+
+msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx, const void *k_idx,
+                              const void *Q, const void *K, const void *V, int32_t *block_ids,
+                              void *O, float *lse, float *block_mass, void *workspace,
+                              size_t workspace_bytes, void *stream) {
     Shape s;
     msa_status_t rc = make_shape(params, &s);
     if (rc != MSA_OK) return rc;
     if (!q_idx || !k_idx || !Q || !K || !V || !O || !lse) return MSA_ERR_INVALID_ARG;
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(Q) || !aligned16(K) ||
         !aligned16(V) || !aligned16(O) || !aligned16(lse) ||
-        (block_ids && !aligned16(block_ids)))
+        (block_ids && !aligned16(block_ids)) || (block_mass && !aligned16(block_mass)))
         return MSA_ERR_INVALID_ARG;
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < forward_ws(s))
         return MSA_ERR_WORKSPACE;
@@ -182,7 +200,8 @@ msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const vo
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
     if (e == cudaSuccess) e = launch_index(s, q_idx, k_idx, bs, false, err, st);
     if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
-    if (e == cudaSuccess) e = launch_attention(s, Q, K, V, ids, O, lse, err, scratch, st);
+    if (e == cudaSuccess)
+        e = launch_attention(s, Q, K, V, ids, O, lse, err, scratch, st, block_mass);
     return cuda_status(e);
 }
 

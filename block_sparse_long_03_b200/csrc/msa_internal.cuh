@@ -60,9 +60,11 @@ size_t attn_tc_workspace(const Shape &s);
 // Query tokens one pass of the tensor-core attention covers (its partials fit
 // a fixed budget); larger calls run several passes.
 int64_t attn_tc_rows_per_pass(const Shape &s);
+// mass (optional, [rows, G, topk] fp32): each kept slot's share of the row's
+// softmax averaged over the group's heads (0 for slots that attend nothing).
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                           cudaStream_t st);
+                           cudaStream_t st, float *mass = nullptr);
 // Partial outputs (fp16, one row of d channels per (query row, head, kept
 // slot)) are stored in 16-byte chunks, blocked by 32 rows: the chunk c of row
 // prow is uint4 number partial_chunk(prow, c).  Consecutive rows of one chunk
@@ -78,7 +80,7 @@ bool combine_supported(const Shape &s);
 // for query rows [r0, r0 + rc) (d = 128).
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
-                           cudaStream_t st);
+                           cudaStream_t st, float *mass = nullptr);
 // Decode path (few query tokens per sequence): HBM-streaming index scoring and
 // one-CTA-per-kept-block attention feeding the same combine.
 bool decode_index_supported(const Shape &s);
@@ -88,10 +90,10 @@ bool decode_attn_supported(const Shape &s);
 size_t decode_attn_workspace(const Shape &s);
 cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
                                const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                               cudaStream_t st);
+                               cudaStream_t st, float *mass = nullptr);
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st);
 cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
-                             cudaStream_t st);
+                             cudaStream_t st, float *mass = nullptr);
 
 }  // namespace msa

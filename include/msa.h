@@ -163,6 +163,39 @@ MSA_EXPORT msa_status_t msa_forward(const msa_params_t *params, const void *q_id
                          void *stream);
 
 /*
+ * The same two calls with a third output: the target of the indexer's KL
+ * objective ("Summary", second paragraph: the indexer learns to match the
+ * Main Branch distribution averaged over a GQA group's heads; "Key points",
+ * kernel design: the LSE that loss needs comes out of the forward pass).
+ *
+ *   block_mass[b, t, g, i] = (1 / R) * sum over heads h of group g of
+ *       sum over the tokens j <= p(t) of block block_ids[b, t, g, i] of
+ *       exp(s_j - lse[b, t, h])
+ *
+ * i.e. each kept slot's share of the row's softmax, averaged over the
+ * group's heads, with s_j and lse as in msa_sparse_attn_fwd.  Empty slots
+ * (-1), skipped caller ids (out of range, repeated) and blocks with no
+ * causal token get 0; over a row's slots the masses sum to 1 (up to fp32
+ * rounding) whenever the row attends to any key.  The merge that produces O
+ * and lse already holds these shares, so the extra cost is the write of
+ * block_mass.
+ *
+ * block_mass [B, T, G, topk] float32 (written; 16-byte aligned).  Every other
+ * argument, layout and error is that of msa_sparse_attn_fwd / msa_forward
+ * (msa_forward_mass's block_ids may be NULL), with the same workspace sizes.
+ */
+MSA_EXPORT msa_status_t msa_sparse_attn_fwd_mass(const msa_params_t *params, const void *Q,
+                                                 const void *K, const void *V,
+                                                 const int32_t *block_ids, void *O, float *lse,
+                                                 float *block_mass, void *workspace,
+                                                 size_t workspace_bytes, void *stream);
+MSA_EXPORT msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx,
+                                         const void *k_idx, const void *Q, const void *K,
+                                         const void *V, int32_t *block_ids, void *O, float *lse,
+                                         float *block_mass, void *workspace,
+                                         size_t workspace_bytes, void *stream);
+
+/*
  * Read the device error word of a workspace (synchronises `stream`) and
  * clear it.  Returns MSA_OK when no kernel recorded a problem, otherwise
  * the recorded status (MSA_ERR_BAD_BLOCK_IDS, MSA_ERR_DEVICE_TIMEOUT).

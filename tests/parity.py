@@ -20,6 +20,27 @@ TOL = {
 }
 
 
+# The KL target's tolerance follows from the LSE tolerance: a slot's mass is a
+# head average of exp(lse_slot - lse), and both LSEs are within lse_max of the
+# exact value, so |d mass| <= mass * (exp(2 lse_max) - 1) <= 2.01 lse_max.
+MASS_TOL = {dt: 2.01 * t["lse_max"] for dt, t in TOL.items()}
+
+
+def oracle_mass_rows(inp, w, rows, ids_rows, lse_rows):
+    """The oracle's KL target [len(rows), G, topk] for sorted `rows`, from the
+    kept ids and the oracle's LSE of those rows (as returned by oracle_rows)."""
+    rows = np.asarray(sorted(rows), dtype=np.int64)
+    out = np.empty(ids_rows.shape, np.float64)
+    for b in np.unique(rows // w.T):
+        sel = np.nonzero(rows // w.T == b)[0]
+        ts = rows[sel] % w.T
+        tt = torch.from_numpy(ts)
+        Q = inp.Q[int(b)].index_select(0, tt.to(inp.Q.device)).cpu()
+        K = inp.K[int(b):int(b) + 1].cpu()
+        out[sel] = orc.block_mass(Q, K, ids_rows[sel], lse_rows[sel], ts, T=w.T, block=w.block)
+    return out
+
+
 def oracle_rows(inp, w, rows, *, want_scores=False, ids=None):
     """Run the oracle for `rows` (r = b * T + t) of the inputs `inp` (device or
     host tensors).  Returns dict of numpy arrays indexed like `rows`."""

@@ -20,7 +20,8 @@ def test_header_declares_the_calls():
     names = declared_symbols()
     for want in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd", "msa_forward",
                  "msa_workspace_size", "msa_status_string", "msa_get_device_error",
-                 "msa_kernel_launches", "msa_selftest_wait_timeout", "msa_forward_host"):
+                 "msa_kernel_launches", "msa_selftest_wait_timeout", "msa_forward_host",
+                 "msa_sparse_attn_fwd_mass", "msa_forward_mass"):
         assert want in names
 
 
@@ -89,6 +90,10 @@ def test_bad_shapes_rejected_on_host(kw, status):
                            1 << 30, None) == status
     assert lib.msa_forward_host(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake,
                                 ws, 1 << 30, None) == status
+    assert lib.msa_sparse_attn_fwd_mass(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake,
+                                        ws, 1 << 30, None) == status
+    assert lib.msa_forward_mass(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake,
+                                fake, ws, 1 << 30, None) == status
 
 
 def test_null_and_misaligned_pointers_rejected():
@@ -119,3 +124,10 @@ def test_null_and_misaligned_pointers_rejected():
     assert lib.msa_forward_host(ctypes.byref(p), None, ok, ok, ok, ok, None, ok, ok, ws, need,
                                 None) == 1
     assert lib.msa_get_device_error(None, None) == 5
+    # the mass output must be 16-byte aligned; the workspace rules are the base calls'
+    assert lib.msa_sparse_attn_fwd_mass(ctypes.byref(p), ok, ok, ok, ok, ok, ok, odd, ws,
+                                        1 << 30, None) == 1
+    assert lib.msa_forward_mass(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, odd, ws,
+                                1 << 30, None) == 1
+    assert lib.msa_forward_mass(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, ok, ws, 16,
+                                None) == 5
