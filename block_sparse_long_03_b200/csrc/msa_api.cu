@@ -3,7 +3,9 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
+#include <vector>
 
 #include "msa_internal.cuh"
 
@@ -67,11 +69,72 @@ cudaError_t launch_index(const Shape &s, const void *q_idx, const void *k_idx, f
     return launch_index_scores_simt(s, q_idx, k_idx, bs, st);
 }
 
+// Sequences [b0, b0 + nb), query tokens [t0, t1) of each: the whole call
+// (nb = B, t0 = 0, t1 = T) or a piece of one sequence (nb = 1).
+struct Piece {
+    int b0, nb, t0, t1;
+};
+
+// The shape a piece's calls see: its queries are the last t1 - t0 of the
+// first S - T + t1 keys, so p(t) is unchanged (t1 = T, or T - t1 a multiple
+// of block, keeps S' a multiple of block).
+Shape piece_shape(const Shape &s, const Piece &p) {
+    Shape q = s;
+    q.B = p.nb;
+    q.T = p.t1 - p.t0;
+    q.S = s.S - s.T + p.t1;
+    q.NB = q.S / s.block;
+    return q;
+}
+
+size_t elem_bytes(const Shape &s) { return s.dtype == MSA_BF16 ? 2 : 4; }
+
+// msa_forward keeps the whole block-score array [B, T, G, NB] while it fits
+// kScoreBudget; beyond that (long prefill: 128 GiB at T = S = 2^20 with four
+// groups) it scores and selects in pieces of queries whose scores take at
+// most kScorePiece, ending at T, T - C, T - 2C, ... of every sequence (a first
+// piece under 128 queries joins the next, so every piece runs the same
+// index kernel as the whole call would).  Every row's scores and ids are the
+// same either way.
+constexpr size_t kScoreBudget = (size_t)4 << 30;
+constexpr size_t kScorePiece = (size_t)1 << 30;
+
+int64_t score_piece_rows(const Shape &s) {
+    if (block_score_bytes(s) <= kScoreBudget) return 0;
+    const int64_t per_row = (int64_t)s.G * s.NB * (int64_t)sizeof(float);
+    const int64_t c = std::max<int64_t>(kScorePiece / per_row / s.block * s.block, 2 * s.block);
+    return c >= s.T ? 0 : c;
+}
+
+std::vector<Piece> score_pieces(const Shape &s) {
+    std::vector<Piece> v;
+    const int64_t c = score_piece_rows(s);
+    if (c == 0) {
+        v.push_back({0, s.B, 0, s.T});
+        return v;
+    }
+    for (int b = 0; b < s.B; ++b) {
+        int64_t lo = 0;
+        for (int64_t k = (s.T + c - 1) / c - 1; k >= 0; --k) {
+            const int64_t hi = s.T - k * c;
+            if (k > 0 && hi - lo < 128) continue;
+            v.push_back({b, 1, (int)lo, (int)hi});
+            lo = hi;
+        }
+    }
+    return v;
+}
+
+size_t score_bytes(const Shape &s) {
+    const int64_t c = score_piece_rows(s);
+    return c == 0 ? block_score_bytes(s) : (size_t)(c + 128) * s.G * s.NB * sizeof(float);
+}
+
 // Workspace layout: [error word 256 B][attention scratch]
 size_t attn_ws(const Shape &s) { return kErrorBytes + attn_scratch(s); }
-// msa_forward: [error word][attention scratch][block scores][block ids]
+// msa_forward: [error word][attention scratch][block scores (or one piece's)][block ids]
 size_t forward_ws(const Shape &s) {
-    return kErrorBytes + attn_scratch(s) + align_up(block_score_bytes(s)) +
+    return kErrorBytes + attn_scratch(s) + align_up(score_bytes(s)) +
            align_up(block_id_bytes(s));
 }
 
@@ -195,11 +258,18 @@ msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx, con
     uint32_t *err = (uint32_t *)ws;
     char *scratch = ws + kErrorBytes;
     float *bs = (float *)(scratch + attn_scratch(s));
-    int32_t *ids = block_ids ? block_ids
-                             : (int32_t *)((char *)bs + align_up(block_score_bytes(s)));
+    int32_t *ids = block_ids ? block_ids : (int32_t *)((char *)bs + align_up(score_bytes(s)));
     cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
-    if (e == cudaSuccess) e = launch_index(s, q_idx, k_idx, bs, false, err, st);
-    if (e == cudaSuccess) e = launch_topk(s, bs, ids, st);
+    const size_t e_sz = elem_bytes(s);
+    for (const Piece &p : score_pieces(s)) {
+        if (e != cudaSuccess) break;
+        const Shape ps = piece_shape(s, p);
+        const int64_t row0 = (int64_t)p.b0 * s.T + p.t0;
+        e = launch_index(ps, (const char *)q_idx + row0 * s.G * s.d_idx * e_sz,
+                         (const char *)k_idx + (int64_t)p.b0 * s.S * s.d_idx * e_sz, bs, false,
+                         err, st);
+        if (e == cudaSuccess) e = launch_topk(ps, bs, ids + row0 * s.G * s.topk, st);
+    }
     if (e == cudaSuccess)
         e = launch_attention(s, Q, K, V, ids, O, lse, err, scratch, st, block_mass);
     return cuda_status(e);
@@ -301,11 +371,6 @@ extern "C" msa_status_t msa_forward_noalloc(const msa_params_t *params, const vo
 namespace msa {
 namespace {
 
-// Sequences [b0, b0 + nb), query tokens [t0, t1) of each: the whole call
-// (nb = B, t0 = 0, t1 = T) or one chunk of one sequence (nb = 1).
-struct Piece {
-    int b0, nb, t0, t1;
-};
 
 // Query tokens per chunk, or 0 when sequences run whole.  Chunks are a
 // multiple of block, about T / 16 and at least 4096 tokens, and at most one
@@ -365,18 +430,6 @@ std::vector<Piece> host_pieces(const Shape &s, int64_t c, int n_seq) {
     return v;
 }
 
-// The shape a piece's attention call sees: its queries are the last t1 - t0
-// of the first S - T + t1 keys, so p(t) is unchanged.
-Shape piece_shape(const Shape &s, const Piece &p) {
-    Shape q = s;
-    q.B = p.nb;
-    q.T = p.t1 - p.t0;
-    q.S = s.S - s.T + p.t1;
-    q.NB = q.S / s.block;
-    return q;
-}
-
-size_t elem_bytes(const Shape &s) { return s.dtype == MSA_BF16 ? 2 : 4; }
 
 // Device buffer: [error word][attention scratch][block scores][block ids]
 // [q_idx][k_idx][Q][K][V][O][lse], each region 256-byte aligned.

@@ -12,7 +12,7 @@
 //
 // One warp per row.  The candidates' ordered keys are staged in shared
 // memory.  For M <= 64 a lower bound of the M-th largest score (the M-th
-// largest of the lanes' top-2 keys) usually leaves at most 64 candidates;
+// largest of the lanes' top-2 keys) usually leaves at most 128 candidates;
 // those are compacted in id order and the M-th largest score u* among them
 // is found bit by bit with warp ballots.  Otherwise a 4-pass radix select
 // (8 bits per pass, warp-private histogram) over all candidates finds u*.
@@ -28,6 +28,64 @@ namespace {
 __device__ __forceinline__ uint32_t ordered_key(float f) {
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Of C <= kMaxCand candidates (ordered keys ck, ids ci, in ascending id
+// order, with every one of the row's M best among them) keep the M best and
+// write them in ascending id order, then cb.  One warp, two or four
+// candidates per lane (candidate 32 q + lane in slot q): the M-th largest key u* is found
+// bit by bit with ballots below the bits all candidates share; every
+// candidate above u* is kept, then the ties at u* with the lowest ids.
+constexpr int kMaxCand = 128;
+
+template <int kSlots>
+__device__ __forceinline__ void select_slots(const uint32_t *ck, const uint32_t *ci, int C, int M,
+                                             int cb, int32_t *out, int lane) {
+    const unsigned lt_mask = (1u << lane) - 1u;
+    bool ok[kSlots];
+    uint32_t k[kSlots];
+    uint32_t all1 = 0xffffffffu, any1 = 0u;
+#pragma unroll
+    for (int q = 0; q < kSlots; ++q) {
+        ok[q] = 32 * q + lane < C;
+        k[q] = ok[q] ? ck[32 * q + lane] : 0u;
+        all1 &= __reduce_and_sync(0xffffffffu, ok[q] ? k[q] : 0xffffffffu);
+        any1 |= __reduce_or_sync(0xffffffffu, ok[q] ? k[q] : 0u);
+    }
+    const uint32_t diff = all1 ^ any1;
+    const int top = diff ? 31 - __clz((int)diff) : -1;
+    uint32_t u = top >= 0 ? all1 & ~((2u << top) - 1u) : all1;
+    for (int bit = top; bit >= 0; --bit) {
+        const uint32_t c = u | (1u << bit);
+        int cnt = 0;
+#pragma unroll
+        for (int q = 0; q < kSlots; ++q)
+            cnt += __popc(__ballot_sync(0xffffffffu, ok[q] && k[q] >= c));
+        if (cnt >= M) u = c;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int q = 0; q < kSlots; ++q) gt += __popc(__ballot_sync(0xffffffffu, ok[q] && k[q] > u));
+    const int need = M - gt;
+    int eq_before = 0, taken_before = 0;          // over the slots before slot q
+#pragma unroll
+    for (int q = 0; q < kSlots; ++q) {
+        const unsigned eb = __ballot_sync(0xffffffffu, ok[q] && k[q] == u);
+        const bool take = ok[q] && (k[q] > u || (k[q] == u && eq_before + __popc(eb & lt_mask) < need));
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        if (take) out[taken_before + __popc(tb & lt_mask)] = (int32_t)ci[32 * q + lane];
+        eq_before += __popc(eb);
+        taken_before += __popc(tb);
+    }
+    if (lane == 0) out[M] = cb;
+}
+
+__device__ __forceinline__ void select_candidates(const uint32_t *ck, const uint32_t *ci, int C,
+                                                  int M, int cb, int32_t *out, int lane) {
+    if (C <= 64)                                  // C is the same in every lane
+        select_slots<2>(ck, ci, C, M, cb, out, lane);
+    else
+        select_slots<4>(ck, ci, C, M, cb, out, lane);
 }
 
 __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids,
@@ -84,7 +142,7 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
             if (cnt >= M) tau = c;
         }
         // candidates with key >= tau, compacted in ascending id order
-        uint32_t *ck = hist, *ci = hist + 64;
+        uint32_t *ck = hist, *ci = hist + kMaxCand;
         int C = 0;
         for (int base = 0; base < cb; base += 32) {
             const int n = base + lane;
@@ -92,44 +150,15 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
             const bool f = n < cb && v >= tau;
             const unsigned fb = __ballot_sync(0xffffffffu, f);
             const int pos = C + __popc(fb & lt_mask);
-            if (f && pos < 64) {
+            if (f && pos < kMaxCand) {
                 ck[pos] = v;
                 ci[pos] = (uint32_t)n;
             }
             C += __popc(fb);
         }
         __syncwarp();
-        if (C <= 64) {
-            // the exact M-th largest key u* among the candidates (= over the
-            // row), bit by bit below the bits all candidates share
-            const bool ok0 = lane < C, ok1 = lane + 32 < C;
-            const uint32_t k0 = ok0 ? ck[lane] : 0u, k1 = ok1 ? ck[lane + 32] : 0u;
-            const uint32_t all1 = __reduce_and_sync(0xffffffffu, ok0 ? k0 : 0xffffffffu) &
-                                  __reduce_and_sync(0xffffffffu, ok1 ? k1 : 0xffffffffu);
-            const uint32_t any1 = __reduce_or_sync(0xffffffffu, ok0 ? k0 : 0u) |
-                                  __reduce_or_sync(0xffffffffu, ok1 ? k1 : 0u);
-            const uint32_t diff = all1 ^ any1;
-            const int top = diff ? 31 - __clz((int)diff) : -1;
-            uint32_t u = top >= 0 ? all1 & ~((2u << top) - 1u) : all1;
-            for (int bit = top; bit >= 0; --bit) {
-                const uint32_t c = u | (1u << bit);
-                const int cnt = __popc(__ballot_sync(0xffffffffu, ok0 && k0 >= c)) +
-                                __popc(__ballot_sync(0xffffffffu, ok1 && k1 >= c));
-                if (cnt >= M) u = c;
-            }
-            // all candidates above u*, then the ties at u* with the lowest ids
-            const int gt = __popc(__ballot_sync(0xffffffffu, ok0 && k0 > u)) +
-                           __popc(__ballot_sync(0xffffffffu, ok1 && k1 > u));
-            const int need = M - gt;
-            const unsigned e0 = __ballot_sync(0xffffffffu, ok0 && k0 == u);
-            const unsigned e1 = __ballot_sync(0xffffffffu, ok1 && k1 == u);
-            const bool t0 = ok0 && (k0 > u || (k0 == u && __popc(e0 & lt_mask) < need));
-            const bool t1 = ok1 && (k1 > u || (k1 == u && __popc(e0) + __popc(e1 & lt_mask) < need));
-            const unsigned tb0 = __ballot_sync(0xffffffffu, t0);
-            const unsigned tb1 = __ballot_sync(0xffffffffu, t1);
-            if (t0) out[__popc(tb0 & lt_mask)] = (int32_t)ci[lane];
-            if (t1) out[__popc(tb0) + __popc(tb1 & lt_mask)] = (int32_t)ci[lane + 32];
-            if (lane == 0) out[M] = cb;
+        if (C <= kMaxCand) {
+            select_candidates(ck, ci, C, M, cb, out, lane);
             return;
         }
         __syncwarp();                 // the radix select below reuses hist
@@ -197,9 +226,10 @@ __global__ void topk_kernel(const float *__restrict__ bs, int32_t *__restrict__ 
 }
 
 // Rows with many candidates (NB > kWarpRowMaxNB): one CTA of kCtaThreads
-// threads per row runs the same selection, the histogram and the ordered
-// emission shared by its warps; leading bits shared by every candidate need
-// no radix pass.
+// threads per row runs the same selection (the threshold filter first, the
+// radix select when it leaves more than 128 candidates), the histogram and the
+// ordered emission shared by its warps; leading bits shared by every
+// candidate need no radix pass.
 constexpr int kWarpRowMaxNB = 2048;
 constexpr int kCtaThreads = 256;
 
@@ -229,11 +259,14 @@ topk_cta_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int T_,
     }
     const float *row = bs + r * NB;
     uint32_t all_and = 0xffffffffu, all_or = 0u;
+    uint32_t b1 = 0u, b2 = 0u;                    // this thread's two largest keys (0: none)
     for (int n = tid; n < cb; n += kCtaThreads) {
         const uint32_t v = ordered_key(row[n]);
         keys[n] = v;
         all_and &= v;
         all_or |= v;
+        b2 = max(b2, min(v, b1));
+        b1 = max(b1, v);
     }
     all_and = __reduce_and_sync(0xffffffffu, all_and);
     all_or = __reduce_or_sync(0xffffffffu, all_or);
@@ -242,6 +275,54 @@ topk_cta_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int T_,
     all_and = 0xffffffffu; all_or = 0u;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) { all_and &= red[w]; all_or |= red[kWarps + w]; }
+    if (M <= 64) {
+        // As in the warp kernel: a lower bound tau of the M-th largest key
+        // (the M-th largest of the threads' top-2 keys, on its top 16 bits),
+        // the candidates >= tau compacted in id order, and if at most 128,
+        // warp 0 selects among them.  Counts cross the warps through a
+        // double-buffered shared array (one barrier per step).
+        __shared__ int cnt[2][kWarps];
+        uint32_t tau = 0u;
+        for (int bit = 31, it = 0; bit >= 16; --bit, ++it) {
+            const uint32_t c = tau | (1u << bit);
+            const int n_ge = __popc(__ballot_sync(0xffffffffu, b1 >= c)) +
+                             __popc(__ballot_sync(0xffffffffu, b2 >= c));
+            if (lane == 0) cnt[it & 1][warp] = n_ge;
+            __syncthreads();
+            int total = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) total += cnt[it & 1][w];
+            if (total >= M) tau = c;
+        }
+        uint32_t *ck = hist, *ci = hist + kMaxCand;   // the radix path re-zeroes hist
+        int C = 0;
+        for (int base = 0, it = 0; base < cb; base += kCtaThreads, ++it) {
+            const int n = base + tid;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool f = n < cb && v >= tau;
+            const unsigned fb = __ballot_sync(0xffffffffu, f);
+            if (lane == 0) cnt[it & 1][warp] = __popc(fb);
+            __syncthreads();
+            int before = C, total = C;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                before += w < warp ? cnt[it & 1][w] : 0;
+                total += cnt[it & 1][w];
+            }
+            const int pos = before + __popc(fb & lt_mask);
+            if (f && pos < kMaxCand) {
+                ck[pos] = v;
+                ci[pos] = (uint32_t)n;
+            }
+            C = total;
+        }
+        __syncthreads();
+        if (C <= kMaxCand) {                      // C is the same in every thread
+            if (warp == 0) select_candidates(ck, ci, C, M, cb, out, lane);
+            return;
+        }
+        __syncthreads();                          // hist is reused below
+    }
     const uint32_t diff = all_and ^ all_or;
     const int top = diff ? 31 - __clz(diff) : -1;
     uint32_t prefix = 0, mask = 0;

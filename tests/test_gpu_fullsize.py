@@ -54,3 +54,43 @@ def test_workload_full_size(name):
                         ref["O"], ref["lse"], w.dtype, name)
     del inp, O, lse, ids, ws
     torch.cuda.empty_cache()
+
+
+def test_forward_scores_in_pieces():
+    """A prefill whose block-score array exceeds the forward's 4 GiB budget
+    (147456 tokens, 8 groups, 1152 blocks: 5.4 GB) is scored and selected in
+    pieces of queries inside msa_forward: ids, O and LSE are bitwise those of
+    the three separate calls on the whole array, and match the oracle on
+    rows at and around the piece boundaries."""
+    import block_sparse_long_03_b200 as msa
+    from block_sparse_long_03_b200 import synthetic
+    w = synthetic.Workload("prefill_147k_g8", B=1, T=147456, S=147456, Hq=8, Hkv=8, d=128,
+                           d_idx=64, block=128, topk=8, dtype=torch.bfloat16,
+                           hot_blocks_per_group=4)
+    torch.cuda.empty_cache()
+    inp = synthetic.make_inputs(w, seed=2, device="cuda")
+    p = msa.params_from(inp.q_idx, inp.Q, inp.K, block=w.block, topk=w.topk)
+    full_bs = w.B * w.T * w.G * w.NB * 4
+    assert full_bs > 4 << 30
+    assert msa.msa_workspace_size(p, msa.MSA_WS_FORWARD) < full_bs   # one piece's scores only
+    O, lse, ids, ws = msa.forward(inp.q_idx, inp.k_idx, inp.Q, inp.K, inp.V, block=w.block,
+                                  topk=w.topk)
+    bs = msa.index_block_scores(inp.q_idx, inp.k_idx, block=w.block)
+    ids2 = msa.topk_blocks(bs, S=w.S, block=w.block, topk=w.topk)
+    del bs
+    O2, lse2, ws2 = msa.sparse_attn_fwd(inp.Q, inp.K, inp.V, ids2, block=w.block)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    assert torch.equal(ids, ids2), "piecewise scoring changed the kept ids"
+    assert torch.equal(lse, lse2)
+    assert torch.equal(O.view(torch.int16), O2.view(torch.int16))
+    _check_all_rows_valid(ids, w)
+    c = (1 << 30) // (w.G * w.NB * 4) // w.block * w.block     # rows per piece
+    edges = sorted({t for k in range(1, 4) for t in (w.T - k * c - 1, w.T - k * c)} |
+                   {0, w.T - 1})
+    ref = parity.oracle_rows(inp, w, edges)
+    parity.assert_ids_equal(parity.gather_rows(ids, edges, w.T), ref["ids"], "pieces")
+    parity.assert_close(parity.gather_rows(O, edges, w.T), parity.gather_rows(lse, edges, w.T),
+                        ref["O"], ref["lse"], w.dtype, "pieces")
+    del inp, O, lse, ids, ws, O2, lse2, ids2, ws2
+    torch.cuda.empty_cache()
