@@ -465,12 +465,12 @@ def run_ours(args, rank: int, ws: int):
 
     decode = None
     if not args.no_decode:
-        dp = Problem(DECODE, seed=rank_seed(rank) + 1)
+        dp = Problem(args.decode_workload, seed=rank_seed(rank) + 1)
         with ClockSampler(local) as dclk:
             dms = time_steps(dp.step, max(args.steps, 10), args.warmup, ws)
         dst = dp.stage_times_ms(max(args.steps, 10))
         db = decode_bytes(dp.w)
-        decode = {"workload": DECODE, "us_per_step": dms * 1e3, "bytes_per_step": db,
+        decode = {"workload": args.decode_workload, "us_per_step": dms * 1e3, "bytes_per_step": db,
                   "achieved_gbs": db / (dms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                   "frac": db / (dms / 1e3) / 1e9 / pk["hbm_gbs"], "stage_ms": dst,
                   "clocks": dclk.summary()}
@@ -492,7 +492,8 @@ def run_ours(args, rank: int, ws: int):
             "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq,
                        "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx, "block": w.block,
                        "topk": w.topk, "parallelism": f"replicas x{ws}",
-                       "l2": "inputs larger than L2 (Q alone 2 GiB); no flush"},
+                       "l2": f"inputs larger than L2 (Q alone "
+                             f"{w.B * w.T * w.Hq * w.d * 2 / 2**30:.1f} GiB); no flush"},
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "kl_target": kl,
             "gpu_launches": int(round(per_step * args.steps)),
             "clocks": clk.summary(), "decode": decode,
@@ -507,6 +508,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=PREFILL)
+    ap.add_argument("--decode-workload", default=DECODE)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

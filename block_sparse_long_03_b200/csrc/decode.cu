@@ -184,8 +184,10 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
 
 constexpr int kAttnThreads = 128;
 
-// One CTA = one kept slot of one (query row, group): the partial softmax of
-// the R query heads over that block's causal keys.
+// One CTA = one kept slot of one (query row, group) and up to 8 of the
+// group's query heads (the width of one mma tile): the partial softmax of
+// those heads over that block's causal keys.  With R = 16 two CTAs share a
+// slot, heads 0-7 and 8-15.
 template <int D, int BLOCK>
 __global__ void __launch_bounds__(kAttnThreads)
 decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
@@ -203,8 +205,11 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     float *sMax = sRed + 4 * 8;                            // [8] per-head maximum
     __half *sO = (__half *)(sMax + 8);                     // [8 heads][D]
 
-    const int slot = blockIdx.x % topk;
-    const int64_t rg = blockIdx.x / topk;                  // (b * T + t) * G + g
+    const int nhalf = (R + 7) / 8;                         // CTAs per kept slot
+    const int h0 = (int)(blockIdx.x % nhalf) * 8;          // first head of this CTA
+    const int Rh = R - h0 < 8 ? R - h0 : 8;                // heads of this CTA
+    const int slot = (int)((blockIdx.x / nhalf) % topk);
+    const int64_t rg = blockIdx.x / nhalf / topk;          // (b * T + t) * G + g
     const int g = (int)(rg % Hkv);
     const int64_t bt = rg / Hkv;
     const int b = (int)(bt / T_), t = (int)(bt % T_);
@@ -216,7 +221,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     const int n = row[slot];
     if (n < 0) return;
     if (n >= NB) {
-        if (threadIdx.x == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+        if (threadIdx.x == 0 && h0 == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
         return;
     }
     const int64_t j0 = (int64_t)n * BLOCK;
@@ -245,15 +250,16 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     }
     if (repeat || n > cb) {                                // n > cb: no causal token
         cp_async_wait<0>();                                // this CTA's copies land first
-        if (repeat && threadIdx.x == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+        if (repeat && threadIdx.x == 0 && h0 == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
         return;
     }
     // B fragments of Q^T: column g4 = head (zero past R)
     uint32_t bq[D / 16][2];
 #pragma unroll
     for (int ks = 0; ks < D / 16; ++ks) {
-        if (g4 < R) {
-            const __nv_bfloat16 *q = Q + (bt * Hq + (int64_t)g * R + g4) * D + ks * 16 + 2 * t4;
+        if (g4 < Rh) {
+            const __nv_bfloat16 *q =
+                Q + (bt * Hq + (int64_t)g * R + h0 + g4) * D + ks * 16 + 2 * t4;
             bq[ks][0] = *(const uint32_t *)q;
             bq[ks][1] = *(const uint32_t *)(q + 8);
         } else {
@@ -357,14 +363,14 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
         }
     }
     __syncthreads();
-    // write the R partial rows in the blocked chunk layout (partial_chunk)
-    // and their LSE
-    const int64_t prow0 = (rg * topk + slot) * R;
-    for (int c = tid; c < R * kChunks; c += kAttnThreads) {
-        const int h = c % R, ch = c / R;
+    // write this CTA's Rh partial rows in the blocked chunk layout
+    // (partial_chunk) and their LSE
+    const int64_t prow0 = (rg * topk + slot) * R + h0;
+    for (int c = tid; c < Rh * kChunks; c += kAttnThreads) {
+        const int h = c % Rh, ch = c / Rh;
         ((uint4 *)part_o)[partial_chunk(prow0 + h, ch, D)] = *(const uint4 *)(sO + h * D + ch * 8);
     }
-    if (tid < R) {
+    if (tid < Rh) {
         const int h = tid;
         const float l = sRed[h] + sRed[8 + h] + sRed[16 + h] + sRed[24 + h];
         part_lse[prow0 + h] = sMax[h] * scale + logf(l);
@@ -407,7 +413,7 @@ cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const v
     auto k = decode_block_kernel<D, BLOCK>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t ctas = s.index_rows() * s.topk;
+    const int64_t ctas = s.index_rows() * s.topk * ((s.R + 7) / 8);
     const float scale_log2 = s.scale * 1.4426950408889634f;
     k<<<(unsigned)ctas, kAttnThreads, smem, st>>>(
         (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, ids, part_o,
@@ -436,8 +442,8 @@ cudaError_t launch_decode_index(const Shape &s, const void *q_idx, const void *k
 }
 
 bool decode_attn_supported(const Shape &s) {
-    return s.dtype == MSA_BF16 && s.d == 128 && s.R <= 8 && (s.block == 64 || s.block == 128) &&
-           s.index_rows() * s.topk < (1ll << 31) && combine_supported(s);
+    return s.dtype == MSA_BF16 && s.d == 128 && s.R <= 16 && (s.block == 64 || s.block == 128) &&
+           s.index_rows() * s.topk * ((s.R + 7) / 8) < (1ll << 31) && combine_supported(s);
 }
 
 size_t decode_attn_workspace(const Shape &s) {

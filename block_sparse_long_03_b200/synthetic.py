@@ -68,6 +68,15 @@ WORKLOADS = {
     "chunked_prefill_1m": Workload("chunked_prefill_1m", B=1, T=4096, S=1 << 20, Hq=32, Hkv=4,
                                    d=128, d_idx=64, block=128, topk=64, dtype=torch.bfloat16,
                                    hot_blocks_per_group=32),
+    # The pages' own long-context shape (64 query heads, 4 KV heads, head
+    # dimension 128, B_k = 128, k = 16) at 2^20 tokens: a full prefill, and
+    # decode steps of 16 sequences (the decode batch is not stated; d_idx as
+    # in the other workloads).
+    "prefill_1m": Workload("prefill_1m", B=1, T=1 << 20, S=1 << 20, Hq=64, Hkv=4, d=128,
+                           d_idx=64, block=128, topk=16, dtype=torch.bfloat16,
+                           hot_blocks_per_group=8),
+    "decode_1m": Workload("decode_1m", B=16, T=1, S=1 << 20, Hq=64, Hkv=4, d=128, d_idx=64,
+                          block=128, topk=16, dtype=torch.bfloat16),
     # Reduced sizes of the same shapes, small enough for profiler captures
     # (a few GB on the device).
     "prefill_8k": Workload("prefill_8k", B=1, T=8192, S=8192, Hq=64, Hkv=8, d=128, d_idx=64,

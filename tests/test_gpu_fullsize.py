@@ -1,6 +1,6 @@
-"""The five workloads at full size, in the launch configuration the benchmark
-times (msa_forward on device-resident inputs), against the oracle on a
-sample of rows; plus properties checked on EVERY row: each (row, group)
+"""The five workloads at full size, and the pages' own 1M shape (prefill and
+decode), in the launch configuration the benchmark times (msa_forward on
+device-resident inputs), against the oracle on a sample of rows; plus properties checked on EVERY row: each (row, group)
 keeps exactly min(k, cb + 1) distinct ascending ids, all <= cb, with cb
 among them, and LSE is finite."""
 import numpy as np
@@ -12,7 +12,7 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 N_SAMPLE = {"tiny_fp32_prefill": 0, "prefill_32k": 48, "prefill_128k": 32, "decode_128k": 16,
-            "chunked_prefill_1m": 32}
+            "chunked_prefill_1m": 32, "prefill_1m": 6, "decode_1m": 8}
 
 
 def _check_all_rows_valid(ids, w):
@@ -33,7 +33,8 @@ def _check_all_rows_valid(ids, w):
 
 
 @pytest.mark.parametrize("name", ["tiny_fp32_prefill", "prefill_32k", "prefill_128k",
-                                  "decode_128k", "chunked_prefill_1m"])
+                                  "decode_128k", "chunked_prefill_1m", "prefill_1m",
+                                  "decode_1m"])
 def test_workload_full_size(name):
     import block_sparse_long_03_b200 as msa
     from block_sparse_long_03_b200 import synthetic

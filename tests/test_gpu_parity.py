@@ -59,6 +59,9 @@ def _case(name):
         # an odd number of 64-key blocks: the last 128-key index tile holds one block
         "bf16_prefill_odd_blocks": W("bf16_prefill_odd_blocks", B=2, T=700, S=1088, Hq=8, Hkv=2,
                                      d=128, d_idx=64, block=64, topk=5, dtype=bf),
+        # decode with 16 heads per group: two CTAs of 8 heads per kept block
+        "bf16_decode_R16": W("bf16_decode_R16", B=3, T=1, S=4096, Hq=32, Hkv=2, d=128,
+                             d_idx=64, block=128, topk=6, dtype=bf),
         # more than 2048 candidate blocks per row: the CTA-per-row Top-k
         "bf16_chunk_many_blocks": W("bf16_chunk_many_blocks", B=1, T=64, S=139264, Hq=8, Hkv=2,
                                     d=128, d_idx=64, block=64, topk=9, dtype=bf),
@@ -70,7 +73,7 @@ CASES = ["tiny_fp32_prefill", "bf16_prefill_2x1024", "bf16_chunk_ragged", "bf16_
          "bf16_d64_mha", "bf16_dense_limit", "bf16_topk1", "fp32_gqa8", "bf16_prefill_R16",
          "bf16_prefill_R1_didx128", "bf16_prefill_B2_chunk", "bf16_decode_block128",
          "bf16_decode_T4", "bf16_decode_topk64", "bf16_prefill_odd_blocks",
-         "bf16_chunk_many_blocks"]
+         "bf16_chunk_many_blocks", "bf16_decode_R16"]
 
 
 def _inputs(w, seed=0):
@@ -133,7 +136,8 @@ def test_topk_heavy_ties_and_closed_form():
             assert np.all(ids[0, t, g, len(want):] == -1)
 
 
-@pytest.mark.parametrize("name", ["bf16_chunk_ragged", "bf16_decode_small", "bf16_decode_T4"])
+@pytest.mark.parametrize("name", ["bf16_chunk_ragged", "bf16_decode_small", "bf16_decode_T4",
+                                  "bf16_decode_R16"])
 def test_sparse_attn_permuted_and_bad_ids(name):
     """Caller ids in any order give the same result; ids out of range or
     repeated are skipped and reported through the device error word (the
