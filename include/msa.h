@@ -155,7 +155,11 @@ MSA_EXPORT msa_status_t msa_sparse_attn_fwd(const msa_params_t *params, const vo
  * where that pays.  Same meaning and layouts as the three calls above.
  * block_ids may be NULL (the ids then live in the workspace only); when not
  * NULL it receives the kept ids [B, T, G, topk].  workspace must hold
- * msa_workspace_size(params, 1) bytes.
+ * msa_workspace_size(params, 1) bytes.  The block scores never leave the
+ * workspace; when all of them would take more than 4 GiB (long prefill),
+ * the call scores and selects in pieces of consecutive queries of at most
+ * 1 GiB of scores each, with the same result, so the workspace stays
+ * bounded.
  */
 MSA_EXPORT msa_status_t msa_forward(const msa_params_t *params, const void *q_idx, const void *k_idx,
                          const void *Q, const void *K, const void *V, int32_t *block_ids,
