@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED",
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
            "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
-           "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass")
+           "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass",
+           "msa_query_pieces")
 
 
 class MsaError(RuntimeError):
@@ -66,6 +67,8 @@ def _load():
     lib.msa_sparse_attn_fwd_mass.restype = st
     lib.msa_forward_mass.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_forward_mass.restype = st
+    lib.msa_query_pieces.argtypes = [P, ctypes.c_int, vp, ctypes.c_int64]
+    lib.msa_query_pieces.restype = ctypes.c_int64
     lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.msa_selftest_wait_timeout.restype = st
     lib.msa_kernel_launches.argtypes = []
@@ -188,6 +191,17 @@ def msa_selftest_wait_timeout(workspace, limit_us: int, stream=None):
     """Run the device wait-timeout check (see include/msa.h)."""
     _check(lib.msa_selftest_wait_timeout(_ptr(workspace), workspace.numel(), int(limit_us),
                                          _stream(stream)), "msa_selftest_wait_timeout")
+
+
+def msa_query_pieces(params: Params, which: int) -> list:
+    """The (sequence, first query, end query) pieces a call splits its work into
+    (which = MSA_WS_FORWARD or MSA_WS_FORWARD_HOST); sequence -1 means all."""
+    n = int(lib.msa_query_pieces(ctypes.byref(params), int(which), None, 0))
+    if n <= 0:
+        return []
+    buf = (ctypes.c_int32 * (3 * n))()
+    lib.msa_query_pieces(ctypes.byref(params), int(which), buf, n)
+    return [tuple(buf[3 * i:3 * i + 3]) for i in range(n)]
 
 
 def msa_kernel_launches() -> int:

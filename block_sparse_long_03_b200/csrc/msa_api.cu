@@ -381,10 +381,11 @@ int64_t host_chunk(const Shape &s) {
     const int64_t blk = s.block;
     int64_t c = ((int64_t)s.T / 16 + blk - 1) / blk * blk;
     c = std::max<int64_t>(c, (4096 + blk - 1) / blk * blk);
-    Shape one = s;
+    Shape one = s;                                  // the partial budget's rows, not capped by T
     one.B = 1;
+    one.T = 1 << 30;
     c = std::min<int64_t>(c, attn_tc_rows_per_pass(one) / blk * blk);
-    if (c < 64 || c >= s.T) return 0;
+    if (c < 4096 || c >= s.T) return 0;             // short sequences run whole
     return c;
 }
 
@@ -629,4 +630,25 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
     if (je == cudaSuccess) je = cudaStreamWaitEvent(st, ev_down, 0);
     if (ce == cudaSuccess) ce = je;
     return cuda_status(ce);
+}
+
+extern "C" int64_t msa_query_pieces(const msa_params_t *params, int which, int32_t *pieces,
+                                    int64_t cap) {
+    Shape s;
+    if (make_shape(params, &s) != MSA_OK) return 0;
+    if (cap > 0 && pieces == nullptr) return -1;
+    std::vector<Piece> v;
+    if (which == MSA_WS_FORWARD)
+        v = score_pieces(s);
+    else if (which == MSA_WS_FORWARD_HOST)
+        v = host_pieces(s, host_chunk(s), s.B);
+    else
+        return 0;
+    for (int64_t i = 0; i < (int64_t)v.size() && i < cap; ++i) {
+        const bool whole = v.size() == 1 && v[i].t0 == 0 && v[i].t1 == s.T;
+        pieces[3 * i] = (whole || v[i].nb > 1) ? -1 : v[i].b0;
+        pieces[3 * i + 1] = v[i].t0;
+        pieces[3 * i + 2] = v[i].t1;
+    }
+    return (int64_t)v.size();
 }

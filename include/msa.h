@@ -286,6 +286,20 @@ MSA_EXPORT msa_status_t msa_forward_host(const msa_params_t *params, const void 
                                          void *stream);
 
 /*
+ * Diagnostics: the query pieces a call splits its work into, computed on the
+ * host (no GPU is touched).  which = MSA_WS_FORWARD: the pieces msa_forward
+ * scores and selects in (one piece when the block scores fit its budget);
+ * which = MSA_WS_FORWARD_HOST: the copy/compute pieces of msa_forward_host.
+ * Writes min(count, cap) pieces into `pieces` as int32 triples
+ * (sequence, first query, end query), pieces of one sequence in order; a
+ * piece that covers every sequence whole is reported as (-1, 0, T).
+ * Returns the number of pieces, 0 for invalid shapes or `which`, and -1
+ * when `pieces` is NULL with cap > 0.
+ */
+MSA_EXPORT int64_t msa_query_pieces(const msa_params_t *params, int which, int32_t *pieces,
+                                    int64_t cap);
+
+/*
  * Diagnostics: a check of the device failure path.  Launches one CTA that
  * takes the library's bounded mbarrier wait on a barrier nothing completes,
  * with a limit of limit_us microseconds (1 .. 1,000,000).  When the wait
