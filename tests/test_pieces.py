@@ -90,3 +90,21 @@ def test_query_pieces_rejects():
     p, _ = _p()
     assert binding.lib.msa_query_pieces(ctypes.byref(p), 7, None, 0) == 0
     assert binding.lib.msa_query_pieces(ctypes.byref(p), msa.MSA_WS_FORWARD, None, 4) == -1
+
+
+def test_workspace_stays_bounded_for_long_prefill():
+    """msa_forward's workspace holds one piece's scores once the whole array
+    passes 4 GiB (128 GiB at the pages' 1M shape), and the host call's buffer
+    holds at least every tensor it copies plus that scratch."""
+    import block_sparse_long_03_b200 as msa
+    p, sh = _p(T=1 << 20, S=1 << 20, Hkv=4, topk=16)
+    full_scores = sh["T"] * sh["Hkv"] * (sh["S"] // sh["block"]) * 4
+    ws = msa.msa_workspace_size(p, msa.MSA_WS_FORWARD)
+    assert full_scores == 128 << 30
+    assert ws < 8 << 30                                   # partial budget + one piece of scores
+    host = msa.msa_workspace_size(p, msa.MSA_WS_FORWARD_HOST)
+    T, S, Hq, Hkv, d, d_idx = sh["T"], sh["S"], sh["Hq"], sh["Hkv"], sh["d"], sh["d_idx"]
+    tensors = 2 * (T * Hkv * d_idx + S * d_idx + 2 * T * Hq * d + 2 * S * Hkv * d) + 4 * T * Hq
+    assert host >= tensors
+    p, _ = _p()                                           # 128K: the whole array, 4 GiB
+    assert msa.msa_workspace_size(p, msa.MSA_WS_FORWARD) >= 4 << 30
