@@ -265,6 +265,9 @@ def pin_bf16_widening(lib):
                     topk=k, lib=lib, want_scores=True)
     for x, y in zip(a, b):
         assert np.array_equal(x, y), "bf16 and fp32 copies of the same values disagree"
+    ma = orc.block_mass(Q, K, a[0], a[2], rows, T=T, block=block, lib=lib)
+    mb = orc.block_mass(Q.float(), K.float(), b[0], b[2], rows, T=T, block=block, lib=lib)
+    assert np.array_equal(ma, mb), "bf16 and fp32 copies give different block masses"
 
 
 def _torch_block_mass(Q, K, allowed, scale, ids, block):
@@ -336,6 +339,25 @@ def pin_block_mass(lib):
         none = orc.block_mass(Qr, K, ids, np.full_like(lse, -np.inf), rows, T=T, block=block,
                               lib=lib)
         assert np.all(none == 0.0)
+    # a slot's mass is the head average of exp(LSE over that block alone - LSE over
+    # the whole kept set), the single-block LSEs taken from the attention routine
+    B, T, S, Hq, Hkv, d, d_idx, block, k = 1, 48, 96, 6, 2, 8, 4, 8, 4
+    R = Hq // Hkv
+    Q = rng.standard_normal((B * T, Hq, d)).astype(np.float32)
+    K = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    V = rng.standard_normal((B, S, Hkv, d)).astype(np.float32)
+    rows = _rows_all(B, T)
+    q_idx = _grid(rng, (B * T, Hkv, d_idx))
+    k_idx = _grid(rng, (B, S, d_idx))
+    ids, O, lse = orc.forward(q_idx, k_idx, Q, K, V, rows, T=T, block=block, topk=k, lib=lib)
+    mass = orc.block_mass(Q, K, ids, lse, rows, T=T, block=block, lib=lib)
+    for i in range(k):
+        one = np.full_like(ids, -1)
+        one[..., 0] = ids[..., i]
+        _, lse_i = orc.attention(Q, K, V, one, rows, T=T, block=block, lib=lib)
+        want = np.exp(lse_i - lse).reshape(B * T, Hkv, R).mean(-1)
+        want[ids[..., i] < 0] = 0.0
+        np.testing.assert_allclose(mass[..., i], want, rtol=1e-12, atol=1e-15)
 
 
 ALL_PINS = [pin_brute_force_selection, pin_dense_limit, pin_masked_attention,
