@@ -131,3 +131,19 @@ def test_null_and_misaligned_pointers_rejected():
                                 1 << 30, None) == 1
     assert lib.msa_forward_mass(ctypes.byref(p), ok, ok, ok, ok, ok, None, ok, ok, ok, ws, 16,
                                 None) == 5
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without libmsa.so the package refuses to import: there is no other
+    implementation to fall back to."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "block_sparse_long_03_b200")
+    dst = tmp_path / "block_sparse_long_03_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "*.so.*", "csrc",
+                                                            "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_long_03_b200"],
+                       cwd=str(tmp_path), capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libmsa.so" in r.stderr
