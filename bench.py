@@ -63,46 +63,55 @@ def index_flops(w) -> float:
     return float(w.B * w.G * 2 * w.d_idx * (p + 1).sum())
 
 
+def kept_slots(w) -> int:
+    """(query, group, kept slot) triples of a forward pass: min(k, cb + 1)
+    per (query, group)."""
+    p = w.S - w.T + np.arange(w.T, dtype=np.int64)
+    return int(w.B * w.G * np.minimum(w.topk, p // w.block + 1).sum())
+
+
 def partial_floor_bytes(w) -> float:
     """HBM bytes the KV-block-outer schedule of the sparse attention call must
     move whatever the kernels do: each (query, group, kept slot, head) partial
-    (d fp16 values + an fp32 LSE) written once and read once by the combine,
+    (d bf16 values + an fp32 LSE) written once and read once by the combine,
     plus Q, K, V read once and O, LSE written once."""
     e = 2 if w.dtype == torch.bfloat16 else 4
-    p = w.S - w.T + np.arange(w.T, dtype=np.int64)
-    slots = w.B * w.G * np.minimum(w.topk, p // w.block + 1).sum()
+    slots = kept_slots(w)
     partials = slots * (w.Hq // w.Hkv) * (w.d * 2 + 4) * 2
     io = w.B * w.T * w.Hq * (2 * w.d * e + 4) + 2 * w.B * w.S * w.G * w.d * e
     return float(partials + io)
 
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
-# msa_sparse_attn_fwd call, summed over its kernels (17 row chunks of CSR
-# build, attention and combine), averaged over the five calls on
-# device-resident inputs in a one-pass ncu launch list of
-# `python bench.py --steps 1 --warmup 1 --no-cpu-baseline`, with the SHA-256
-# of the attention source the counters hold for.  The bench reports the
-# figure only while that source is unchanged.  (The counters were taken with
-# the source of SHA-256 521daa93...; the source since only gained the
-# optional KL-target kernel and its launch, which this call does not run, so
-# every kernel the call launches is the one measured.)
-MEASURED_TRAFFIC = {
-    "prefill_128k": {"bytes": 151745748171,
-                     "read_bytes": 81879823308, "write_bytes": 69865924863,
-                     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-                     "source_sha256": "b1e957704b92a81f6e963e00e585f0978c9c1a8e234ec85b77c49ebab424f63f"},
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the sparse
+# attention call's two main kernels, from a one-pass ncu capture of ONE row
+# chunk (the last, 8037 rows, every row keeping k blocks) of the workload
+# `prefill_32k_h64` (the 128K prefill's heads, group size and k at 32K tokens:
+# each chunk is one of the same 8065-row passes the 128K call makes, and Q is
+# larger than L2 as there):
+#   python bench.py --workload prefill_32k_h64 --attn-call-once
+# under ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
+# dram__bytes_write.sum -k regex:"attn_tc_kernel|combine_kernel" -s 6 -c 2.
+# The figures are per kept (query, group) slot of the chunk; a call's traffic
+# is that times its kept slots (the partials, the Q gather and the combine's
+# reads all grow with the slots; K/V and the CSR kernels add < 1 %).  Held
+# with the SHA-256 of the attention source: null once that source changes.
+MEASURED_TRAFFIC = None
 
 
-def measured_traffic(name: str):
+def measured_traffic(w):
+    """(bytes, read, write) of one msa_sparse_attn_fwd call on workload `w`,
+    scaled from the per-slot capture, or None."""
     import hashlib
-    m = MEASURED_TRAFFIC.get(name)
+    m = MEASURED_TRAFFIC
     if m is None:
         return None
     with open(os.path.join(ROOT, m["source"]), "rb") as f:
         if hashlib.sha256(f.read()).hexdigest() != m["source_sha256"]:
             return None
-    return m
+    slots = kept_slots(w)
+    rd = sum(k["read"] for k in m["kernels"].values()) / m["slots"] * slots
+    wr = sum(k["write"] for k in m["kernels"].values()) / m["slots"] * slots
+    return {"bytes": rd + wr, "read_bytes": rd, "write_bytes": wr, "from": m["workload"]}
 
 
 def decode_bytes(w) -> float:
@@ -214,6 +223,16 @@ def _max_over_ranks(x: float, ws: int) -> float:
     return float(t.item())
 
 
+def workload_config(w, ws: int) -> dict:
+    """The `config` of a bench line (the same in both arms)."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    return {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
+            "d": w.d, "d_idx": w.d_idx, "block": w.block, "topk": w.topk,
+            "parallelism": f"replicas x{ws}",
+            "l2": f"inputs larger than L2 (Q alone {w.B * w.T * w.Hq * w.d * e / 2**30:.1f} "
+                  f"GiB); no flush"}
+
+
 def rank_seed(rank: int) -> int:
     """Every rank works on its own independent problem (weak scaling)."""
     return 1000 * rank
@@ -240,7 +259,7 @@ class Problem:
         self.ids = torch.empty((w.B, w.T, w.G, w.topk), dtype=torch.int32, device="cuda")
         self.ws = msa.alloc_workspace(self.params, msa.MSA_WS_FORWARD)
         self.ws_attn = msa.alloc_workspace(self.params, msa.MSA_WS_SPARSE_ATTN)
-        self.bs = torch.empty((w.B, w.T, w.G, w.NB), dtype=torch.float32, device="cuda")
+        self.bs = None                  # the standalone calls' block scores, on first use
         self.mass = None
 
     def step(self, stream=None):
@@ -256,9 +275,28 @@ class Problem:
         self.msa.msa_forward_mass(self.params, i.q_idx, i.k_idx, i.Q, i.K, i.V, self.ids, self.O,
                                   self.lse, self.mass, self.ws, stream)
 
+    def block_scores(self):
+        w = self.w
+        if self.bs is None:
+            self.bs = torch.empty((w.B, w.T, w.G, w.NB), dtype=torch.float32, device="cuda")
+        return self.bs
+
+    def attn_call_once(self):
+        """Index scores and Top-k as separate calls, then ONE msa_sparse_attn_fwd
+        call (the launch sequence a profiler capture of that call selects from)."""
+        m, i = self.msa, self.inp
+        m.msa_index_block_scores(self.params, i.q_idx, i.k_idx, self.block_scores())
+        m.msa_topk_blocks(self.params, self.bs, self.ids)
+        torch.cuda.synchronize()
+        m.msa_sparse_attn_fwd(self.params, i.Q, i.K, i.V, self.ids, self.O, self.lse,
+                              self.ws_attn)
+        torch.cuda.synchronize()
+        return m.msa_get_device_error(self.ws_attn)
+
     def stage_times_ms(self, reps: int) -> dict:
         """Average device time of each call of the path, launched on its own."""
         m, i, s = self.msa, self.inp, torch.cuda.current_stream()
+        self.block_scores()
         stages = {
             "index_block_scores": lambda: m.msa_index_block_scores(self.params, i.q_idx, i.k_idx,
                                                                    self.bs),
@@ -363,7 +401,9 @@ def oracle_sample(name: str, budget_s: float, max_rows: int = 4096, seed: int = 
     if host is None:
         raise RuntimeError("workload too large to generate on the host")
     rng = np.random.default_rng(seed)
-    done, elapsed, batch = 0, 0.0, 2
+    threads = oracle.num_threads()
+    # every oracle call gets at least one row per thread (rows run in parallel)
+    done, elapsed, batch = 0, 0.0, max(2, threads)
     while elapsed < budget_s and done < max_rows:
         rows = np.sort(rng.integers(0, w.B * w.T, size=batch))
         for b in np.unique(rows // w.T):
@@ -375,8 +415,8 @@ def oracle_sample(name: str, budget_s: float, max_rows: int = 4096, seed: int = 
                            T=w.T, block=w.block, topk=w.topk)
             elapsed += time.perf_counter() - t0
         done += batch
-        batch = min(batch * 2, 64)
-    return done / elapsed, done, elapsed, oracle.num_threads()
+        batch = min(batch * 2, max(64, threads))
+    return done / elapsed, done, elapsed, threads
 
 
 def run_reference(args, rank: int, ws: int):
@@ -387,7 +427,7 @@ def run_reference(args, rank: int, ws: int):
     host = synthetic.make_inputs(w, 7, device="cpu")
     budget = float(os.environ.get("MSA_REF_STEP_SECONDS", "8"))
     for _ in range(args.warmup):
-        oracle_sample(args.workload, 0.5, max_rows=2, host=host)
+        oracle_sample(args.workload, 0.5, max_rows=1, host=host)
     rates, rows_total, secs_total, threads = [], 0, 0.0, 1
     for _ in range(args.steps):
         rate, rows, secs, threads = oracle_sample(args.workload, budget / max(args.steps, 1),
@@ -404,8 +444,7 @@ def run_reference(args, rank: int, ws: int):
         "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs_total / max(args.steps, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv,
-                   "d": w.d, "d_idx": w.d_idx, "block": w.block, "topk": w.topk},
+        "config": workload_config(w, ws),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -437,15 +476,18 @@ def run_ours(args, rank: int, ws: int):
     else:
         ach = attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12
         dominant = "sparse_attn_fwd"
-    mt = measured_traffic(w.name) if dominant == "sparse_attn_fwd" else None
+    mt = measured_traffic(w) if dominant == "sparse_attn_fwd" else None
     roof = {"kernel": dominant, "bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": ach / pk["bf16_tflops"],
             "traffic": None if mt is None else float(mt["bytes"]),
-            "traffic_note": ("DRAM bytes of one call (all its kernels, ncu launch list); "
-                             + ("null: the attention source changed since the capture"
+            "traffic_note": ("DRAM bytes of one call: attention and combine kernels, "
+                             "per kept slot from a one-chunk ncu capture, times the call's "
+                             "kept slots; "
+                             + ("null: no capture of the current attention source"
                                 if mt is None else
                                 f"read {mt['read_bytes'] / 1e9:.1f} GB, "
-                                f"written {mt['write_bytes'] / 1e9:.1f} GB")),
+                                f"written {mt['write_bytes'] / 1e9:.1f} GB, "
+                                f"captured on {mt['from']}")),
             "peak_source": pk["source"] + " bf16 burst (of " + pk["source"] + ")",
             "stage_ms": stages,
             "attention_tflops": attn_fl / (stages["sparse_attn_fwd"] / 1e3) / 1e12,
@@ -479,6 +521,30 @@ def run_ours(args, rank: int, ws: int):
                   "clocks": dclk.summary()}
         dp.free()
 
+    # the pages' own 1M-token shape (prefill, and decode steps of 16 sequences)
+    long_ctx = None
+    if not args.no_1m:
+        long_ctx = {}
+        p1 = Problem("prefill_1m", seed=rank_seed(rank) + 2)
+        with ClockSampler(local) as c1:
+            ms1 = time_steps(p1.step, max(2, min(args.steps, 3)), args.warmup, ws)
+        long_ctx["prefill_1m"] = {
+            "tokens_per_s": aggregate_tokens_per_s(p1.w.B * p1.w.T, ms1, ws),
+            "ms_per_step": ms1, "attention_flops": attention_flops(p1.w),
+            "index_flops": index_flops(p1.w), "clocks": c1.summary()}
+        p1.free()
+        del p1
+        d1 = Problem("decode_1m", seed=rank_seed(rank) + 3)
+        with ClockSampler(local) as c2:
+            dms1 = time_steps(d1.step, max(args.steps, 10), args.warmup, ws)
+        db1 = decode_bytes(d1.w)
+        long_ctx["decode_1m"] = {
+            "us_per_step": dms1 * 1e3, "bytes_per_step": db1,
+            "achieved_gbs": db1 / (dms1 / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
+            "frac": db1 / (dms1 / 1e3) / 1e9 / pk["hbm_gbs"], "clocks": c2.summary()}
+        d1.free()
+        del d1
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, rows, secs, threads = oracle_sample(args.workload, args.cpu_seconds)
@@ -492,14 +558,10 @@ def run_ours(args, rank: int, ws: int):
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; Q/K/V ~ N(0,1), index q/k on a 1/4 grid, hot blocks)",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "S": w.S, "Hq": w.Hq,
-                       "Hkv": w.Hkv, "d": w.d, "d_idx": w.d_idx, "block": w.block,
-                       "topk": w.topk, "parallelism": f"replicas x{ws}",
-                       "l2": f"inputs larger than L2 (Q alone "
-                             f"{w.B * w.T * w.Hq * w.d * 2 / 2**30:.1f} GiB); no flush"},
+            "config": workload_config(w, ws),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "kl_target": kl,
             "gpu_launches": int(round(per_step * args.steps)),
-            "clocks": clk.summary(), "decode": decode,
+            "clocks": clk.summary(), "decode": decode, "long_context": long_ctx,
         }
         print(json.dumps(line), flush=True)
 
@@ -515,12 +577,23 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-1m", action="store_true",
+                    help="skip the 1M-token prefill and decode figures")
+    ap.add_argument("--attn-call-once", action="store_true",
+                    help="run one msa_sparse_attn_fwd call on --workload and exit "
+                         "(the command a profiler capture of that call wraps)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
         run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
         return
+    if args.attn_call_once:
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        prob = Problem(args.workload, seed=0)
+        status = prob.attn_call_once()
+        print(json.dumps({"attn_call_once": args.workload, "device_error": status}), flush=True)
+        sys.exit(1 if status else 0)
     rank, ws = _dist()
     try:
         run_ours(args, rank, ws)

@@ -53,12 +53,12 @@ attn_simt_kernel(const T *__restrict__ Q, const T *__restrict__ K, const T *__re
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int32_t *row_ids = ids + bt * Hkv * topk + (int64_t)g * topk;
-    if (tid == 0) {   // validate the caller's ids: in range, no repeats
+    if (tid == 0) {   // validate the caller's ids: in range, causal, no repeats
         int n_ok = 0;
         for (int i = 0; i < topk; ++i) {
             const int n = row_ids[i];
             if (n < 0) continue;
-            bool bad = n >= NB;
+            bool bad = n >= NB || (int64_t)n * block > p;
             for (int k = 0; k < n_ok && !bad; ++k) bad = kept[k] == n;
             if (bad) { record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1); continue; }
             kslot[n_ok] = i;

@@ -16,12 +16,11 @@
 // heads = 128 rows, against the 128 (or 64) keys of block n:
 //   phase 1  S = Q K_n^T (tcgen05, SS), block-local softmax in registers,
 //            P (bf16) to TMEM, O_n = P V_n (tcgen05, A from TMEM), written as
-//            a normalised fp16 partial plus its LSE, one per (query, head,
+//            a normalised bf16 partial plus its LSE, one per (query, head,
 //            kept slot);
 //   phase 2  per (query, head): LSE-weighted combine of the partials of its
 //            kept slots -> O (bf16) and lse (fp32).
 // Work is chunked over query rows so the partial buffer stays bounded.
-#include <cuda_fp16.h>
 #include <math.h>
 
 #include <algorithm>
@@ -39,7 +38,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // Validity of the kept slots lane and lane + 32 of a row (topk <= 64),
 // computed by one warp: in range, holding a causal token, and not a repeat
 // (a strictly ascending row, the form msa_topk_blocks writes, cannot repeat;
-// otherwise earlier slots are scanned).  bad = an id >= NB or a repeat.
+// otherwise earlier slots are scanned).  bad = an id >= NB, an id above cb
+// (a block with no causal token) or a repeat; bad slots are skipped and
+// counted in the error word.
 struct SlotPair {
     int id0, id1;
     bool ok0, ok1, bad0, bad1;
@@ -70,10 +71,10 @@ __device__ __forceinline__ SlotPair warp_slots(const int32_t *row, int topk, int
         for (int q = 0; q < lane && r.id0 >= 0; ++q) rep0 |= row[q] == r.id0;
         for (int q = 0; q < lane + 32 && r.id1 >= 0; ++q) rep1 |= row[q] == r.id1;
     }
-    r.bad0 = r.id0 >= NB || (r.id0 >= 0 && rep0);
-    r.bad1 = r.id1 >= NB || (r.id1 >= 0 && rep1);
-    r.ok0 = r.id0 >= 0 && !r.bad0 && r.id0 <= cb;
-    r.ok1 = r.id1 >= 0 && !r.bad1 && r.id1 <= cb;
+    r.bad0 = r.id0 >= NB || r.id0 > cb || (r.id0 >= 0 && rep0);
+    r.bad1 = r.id1 >= NB || r.id1 > cb || (r.id1 >= 0 && rep1);
+    r.ok0 = r.id0 >= 0 && !r.bad0;
+    r.ok1 = r.id1 >= 0 && !r.bad1;
     return r;
 }
 
@@ -181,7 +182,7 @@ struct AttnArgs {
     const __nv_bfloat16 *Q;     // [B, T, Hq, D]
     const int *recs;            // tile records (rec_ints(tpt) ints each)
     const int *n_tiles;         // device-side tile count
-    __half *part_o;             // normalised partial O, blocked chunks (partial_chunk)
+    __nv_bfloat16 *part_o;      // normalised partial O, blocked chunks (partial_chunk)
     float *part_lse;            // [n_prows]
     int64_t n_prows;            // rc * G * topk * R
     uint32_t *err;
@@ -213,7 +214,7 @@ __device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int
 //                   cp.async), warp 1 issues the S products, warp 2 the PV
 //                   products;
 //   warpgroups 1-2  softmax, tiles 0, 2, 4, ... and 1, 3, 5, ...;
-//   warpgroup 3     epilogue of every tile: O from TMEM to an fp16 partial.
+//   warpgroup 3     epilogue of every tile: O from TMEM to a bf16 partial.
 // TMEM: three S/P buffers (S: BLOCK fp32 columns; P: bf16 pairs in the first
 // BLOCK/2 of them; partial row, row max m and row sum l in the last three) at
 // columns 0, 128, 256 and one O accumulator at 384.  The epilogue divides O
@@ -574,7 +575,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // Every tile in order: wait for its PV product, read the O row and the
         // softmax's partial row, m and l from TMEM (which frees the accumulator
         // for the next PV and, with PV done, the tile's S/P buffer), then O / l
-        // to fp16, stored in 32-row blocked chunk planes (partial_chunk) so that
+        // to bf16 (the range of fp32: no V the inputs can hold overflows it),
+        // stored in 32-row blocked chunk planes (partial_chunk) so that
         // the rows of a warp store to consecutive addresses, and
         // LSE = m * scale + ln l.  No tile metadata is read from memory.
         const int quad = warp % 4;
@@ -600,8 +602,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const float inv = 1.f / l;
 #pragma unroll
             for (int c = 0; c < D; c += 2) {
-                __half2 hv = __floats2half2_rn(__uint_as_float(ov[c]) * inv,
-                                               __uint_as_float(ov[c + 1]) * inv);
+                __nv_bfloat162 hv = __floats2bfloat162_rn(__uint_as_float(ov[c]) * inv,
+                                                          __uint_as_float(ov[c + 1]) * inv);
                 ov[c / 2] = *(uint32_t *)&hv;
             }
             if (prow >= 0) {
@@ -638,7 +640,7 @@ namespace {
 // Needs R | 32 and topk <= 64.
 template <int D, int kMaxPer>
 __global__ void __launch_bounds__(256, kMaxPer <= 8 ? 3 : 2)
-combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_o,
+combine_kernel(const int32_t *__restrict__ ids, const __nv_bfloat16 *__restrict__ part_o,
                                const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
                                float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
                                int Hq, int G, int R, int NB, int block, int topk) {
@@ -684,7 +686,7 @@ combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[c][q] = 0.f;
     // k < per is uniform across the warp, so the loads are issued together;
-    // a slot that holds no partial (weight 0) has its data replaced by 0
+    // a slot that holds no partial (weight 0) issues no load and adds 0
 #pragma unroll
     for (int k = 0; k < kMaxPer; ++k) {
         if (k < per) {
@@ -692,12 +694,12 @@ combine_kernel(const int32_t *__restrict__ ids, const __half *__restrict__ part_
             const bool use = w[k] > 0.f;
 #pragma unroll
             for (int c = 0; c < kChunksPerWarp; ++c) {
-                uint4 u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
-                if (!use) u = make_uint4(0u, 0u, 0u, 0u);
-                const __half2 *hp = (const __half2 *)&u;
+                uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                if (use) u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
+                const __nv_bfloat162 *hp = (const __nv_bfloat162 *)&u;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float2 f = __half22float2(hp[q]);
+                    const float2 f = __bfloat1622float2(hp[q]);
                     acc[c][2 * q] = fmaf(w[k], f.x, acc[c][2 * q]);
                     acc[c][2 * q + 1] = fmaf(w[k], f.y, acc[c][2 * q + 1]);
                 }
@@ -788,7 +790,7 @@ Plan make_plan(const Shape &s) {
     p.toffs = o;    o += al(sizeof(int) * (p.L + 1));
     // at most ceil(slots / tpt) full tiles plus one partial tile per list
     p.recs = o;     o += al(sizeof(int) * rec_ints(p.tpt) * ((slots + p.tpt - 1) / p.tpt + p.L));
-    p.part_o = o;   o += al(sizeof(__half) * ((slots * s.R + 31) / 32 * 32) * s.d);
+    p.part_o = o;   o += al(sizeof(__nv_bfloat16) * ((slots * s.R + 31) / 32 * 32) * s.d);
     p.part_lse = o; o += al(sizeof(float) * slots * s.R);
     p.total = o;
     return p;
@@ -825,7 +827,7 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
     int *counts = (int *)(ws + pl.counts), *cursor = (int *)(ws + pl.cursor);
     int *toffs = (int *)(ws + pl.toffs);
     int *recs = (int *)(ws + pl.recs);
-    __half *part_o = (__half *)(ws + pl.part_o);
+    __nv_bfloat16 *part_o = (__nv_bfloat16 *)(ws + pl.part_o);
     float *part_lse = (float *)(ws + pl.part_lse);
     const size_t smem = 1024 + 3 * (size_t)kRows * D * 2 + 4 * (size_t)BLOCK * D * 2 + 256;
     auto kern = attn_tc_kernel<D, BLOCK>;
@@ -870,7 +872,7 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 }  // namespace
 
-cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
+cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st, float *mass) {
     const int64_t warps = rc * s.G * (128 / 32);

@@ -22,7 +22,6 @@
 // in the same layout as the prefill kernel, so one combine kernel serves
 // both paths.  The work is spread over B * T * G * topk CTAs, enough to keep
 // HBM busy with a single kept block per CTA.
-#include <cuda_fp16.h>
 #include <math.h>
 
 #include "msa_internal.cuh"
@@ -173,7 +172,7 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
                     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
                     v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
                     const int col = cg * 8 + 2 * t4 + e;
-                    if (g4 == 0 && col < TG) bs[((int64_t)b * TG + col) * NB + n] = v;
+                    if (g4 == 0 && col < TG) bs[((int64_t)b * TG + col) * NB + n] = canon_zero(v);
                     best[cg][e] = -INFINITY;
                 }
         }
@@ -192,7 +191,7 @@ template <int D, int BLOCK>
 __global__ void __launch_bounds__(kAttnThreads)
 decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                     const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ ids,
-                    __half *__restrict__ part_o, float *__restrict__ part_lse, uint32_t *err,
+                    __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_lse, uint32_t *err,
                     int T_, int S, int Hq, int Hkv, int R, int NB, int topk, float scale_log2,
                     float scale, int64_t n_prows) {
     constexpr int kRowBytes = D * 2;
@@ -203,7 +202,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     __nv_bfloat16 *sP = (__nv_bfloat16 *)(sV + BLOCK * kRowBytes);   // [8 heads][BLOCK]
     float *sRed = (float *)(sP + 8 * BLOCK);               // [4 warps][8] maxima, then sums
     float *sMax = sRed + 4 * 8;                            // [8] per-head maximum
-    __half *sO = (__half *)(sMax + 8);                     // [8 heads][D]
+    __nv_bfloat16 *sO = (__nv_bfloat16 *)(sMax + 8);       // [8 heads][D]
 
     const int nhalf = (R + 7) / 8;                         // CTAs per kept slot
     const int h0 = (int)(blockIdx.x % nhalf) * 8;          // first head of this CTA
@@ -250,7 +249,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     }
     if (repeat || n > cb) {                                // n > cb: no causal token
         cp_async_wait<0>();                                // this CTA's copies land first
-        if (repeat && threadIdx.x == 0 && h0 == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+        if (threadIdx.x == 0 && h0 == 0) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
         return;
     }
     // B fragments of Q^T: column g4 = head (zero past R)
@@ -349,7 +348,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
         }
     }
     __syncthreads();                                       // sRed (sums) complete
-    // normalise and stage O[head][channel] as fp16
+    // normalise and stage O[head][channel] as bf16
 #pragma unroll
     for (int di = 0; di < kDT; ++di) {
         const int d0 = (warp * kDT + di) * 16 + g4;
@@ -358,8 +357,8 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
             const int h = 2 * t4 + e;
             const float l = sRed[h] + sRed[8 + h] + sRed[16 + h] + sRed[24 + h];
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            sO[h * D + d0] = __float2half_rn(o[di][e] * inv);
-            sO[h * D + d0 + 8] = __float2half_rn(o[di][2 + e] * inv);
+            sO[h * D + d0] = __float2bfloat16_rn(o[di][e] * inv);
+            sO[h * D + d0 + 8] = __float2bfloat16_rn(o[di][2 + e] * inv);
         }
     }
     __syncthreads();
@@ -406,7 +405,7 @@ cudaError_t launch_index_d(const Shape &s, const void *q, const void *k, float *
 
 template <int BLOCK>
 cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const void *V,
-                           const int32_t *ids, __half *part_o, float *part_lse, uint32_t *err,
+                           const int32_t *ids, __nv_bfloat16 *part_o, float *part_lse, uint32_t *err,
                            cudaStream_t st) {
     constexpr int D = 128;
     const size_t smem = 2 * (size_t)BLOCK * D * 2 + 8 * BLOCK * 2 + 40 * 4 + 8 * D * 2;
@@ -453,7 +452,7 @@ size_t decode_attn_workspace(const Shape &s) {
 cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
                                const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                                cudaStream_t st, float *mass) {
-    __half *part_o = (__half *)ws;
+    __nv_bfloat16 *part_o = (__nv_bfloat16 *)ws;
     float *part_lse = (float *)((char *)ws + part_bytes_o(s));
     cudaError_t e = s.block == 64
                         ? launch_block_t<64>(s, Q, K, V, ids, part_o, part_lse, err, st)

@@ -242,6 +242,8 @@ index_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         cm[c] = fmaxf(m0, m1);
                     }
                 }
+                cm[0] = canon_zero(cm[0]);
+                cm[1] = canon_zero(cm[1]);
                 if (row_ok) {
                     if (nbpt == 1) {
                         out[kt] = fmaxf(cm[0], cm[1]);

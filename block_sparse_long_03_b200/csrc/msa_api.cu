@@ -34,7 +34,7 @@ msa_status_t make_shape(const msa_params_t *p, Shape *s) {
     if (p->d != 64 && p->d != 128) return MSA_ERR_UNSUPPORTED;
     if (p->block != 64 && p->block != 128) return MSA_ERR_UNSUPPORTED;
     if (p->d_idx % 16 != 0 || p->d_idx > 128) return MSA_ERR_UNSUPPORTED;
-    if (p->Hq / p->Hkv > 16 || p->topk > 256) return MSA_ERR_UNSUPPORTED;
+    if (p->Hq / p->Hkv > 16 || p->topk > 256 || p->Hkv > 256) return MSA_ERR_UNSUPPORTED;
     // every flat index must fit comfortably in int64 and the grids in 2^31
     const double q_elems = (double)p->B * p->T * p->Hq * p->d;
     const double kv_elems = (double)p->B * p->S * p->Hkv * p->d;
@@ -167,7 +167,7 @@ const char *msa_status_string(msa_status_t status) {
         case MSA_ERR_CUDA: return "MSA_ERR_CUDA: a CUDA runtime call failed";
         case MSA_ERR_DEVICE_TIMEOUT: return "MSA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
         case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace missing, misaligned or too small";
-        case MSA_ERR_BAD_BLOCK_IDS: return "MSA_ERR_BAD_BLOCK_IDS: caller block ids out of range or repeated";
+        case MSA_ERR_BAD_BLOCK_IDS: return "MSA_ERR_BAD_BLOCK_IDS: caller block ids out of range, not causal or repeated";
     }
     return "unknown msa_status_t";
 }

@@ -32,6 +32,13 @@ __device__ __forceinline__ void record_error(uint32_t *err, uint32_t code, int c
     atomicAdd(err + counter, 1u);
 }
 
+// A block score of -0.0 (every product of a zero dot product negative zero)
+// is stored as +0.0: scores compare as numbers, and the stored bits then
+// match a sum that starts from +0.0.
+__device__ __forceinline__ float canon_zero(float x) {
+    return __float_as_uint(x) == 0x80000000u ? 0.f : x;
+}
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
@@ -65,7 +72,7 @@ int64_t attn_tc_rows_per_pass(const Shape &s);
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st, float *mass = nullptr);
-// Partial outputs (fp16, one row of d channels per (query row, head, kept
+// Partial outputs (bf16, one row of d channels per (query row, head, kept
 // slot)) are stored in 16-byte chunks, blocked by 32 rows: the chunk c of row
 // prow is uint4 number partial_chunk(prow, c).  Consecutive rows of one chunk
 // are adjacent (coalesced stores), and all chunks of 32 rows share one
@@ -78,7 +85,7 @@ __host__ __device__ __forceinline__ int64_t partial_chunk(int64_t prow, int c, i
 bool combine_supported(const Shape &s);
 // LSE-weighted combine of per-(row, head, kept slot) partials into O and lse
 // for query rows [r0, r0 + rc) (d = 128).
-cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __half *part_o,
+cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st, float *mass = nullptr);
 // Decode path (few query tokens per sequence): HBM-streaming index scoring and

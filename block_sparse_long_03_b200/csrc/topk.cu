@@ -25,8 +25,10 @@
 namespace msa {
 namespace {
 
+// Scores compare as numbers: -0.0 and +0.0 are equal (the lower id wins the
+// tie), so -0.0 takes the key of +0.0.
 __device__ __forceinline__ uint32_t ordered_key(float f) {
-    const uint32_t u = __float_as_uint(f);
+    const uint32_t u = __float_as_uint(canon_zero(f));
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

@@ -70,11 +70,13 @@ typedef struct {
     int32_t T;       /* query tokens per sequence, 1 <= T <= S              */
     int32_t S;       /* keys per sequence, a multiple of block              */
     int32_t Hq;      /* query heads                                         */
-    int32_t Hkv;     /* KV heads = GQA groups = index heads; Hq % Hkv == 0  */
+    int32_t Hkv;     /* KV heads = GQA groups = index heads; Hq % Hkv == 0, */
+                     /* Hq / Hkv <= 16, Hkv <= 256                          */
     int32_t d;       /* head dimension: 64 or 128                           */
     int32_t d_idx;   /* index head dimension: a multiple of 16, <= 128      */
     int32_t block;   /* KV block size B_k: 64 or 128                        */
-    int32_t topk;    /* blocks kept per (query, group), current one included */
+    int32_t topk;    /* blocks kept per (query, group), current one included; */
+                     /* <= 256                                              */
     int32_t dtype;   /* msa_dtype_t                                         */
     float scale;     /* softmax scale; <= 0 selects 1/sqrt(d)               */
 } msa_params_t;
@@ -135,10 +137,11 @@ MSA_EXPORT size_t msa_workspace_size(const msa_params_t *params, int which);
  *   O[b, t, h, :] = sum_j softmax(s)_j V[b, j, g, :]
  *   lse[b, t, h]  = log(sum_j exp(s_j))      (natural log)
  * The order of the ids in a row does not matter.  Caller ids are not
- * trusted: an id >= NB, or an id repeated within a row, is skipped (a repeat
- * counts once) and the device error word records MSA_ERR_BAD_BLOCK_IDS.  An
- * id above cb(t) holds no causal token and adds nothing.  A row with no
- * attended key gets O = 0 and lse = -infinity.
+ * trusted: an id >= NB, an id above cb(t) (a block with no causal token), or
+ * an id repeated within a row is skipped (a repeat counts once) and the
+ * device error word records MSA_ERR_BAD_BLOCK_IDS; the other ids of the row
+ * are attended as usual.  A row with no attended key gets O = 0 and
+ * lse = -infinity.
  *
  * Q [B, T, Hq, d], K and V [B, S, Hkv, d] (dtype, read);
  * block_ids [B, T, G, topk] int32 (read); O [B, T, Hq, d] (dtype, written);
@@ -180,9 +183,11 @@ MSA_EXPORT msa_status_t msa_forward(const msa_params_t *params, const void *q_id
  * group's heads, with s_j and lse as in msa_sparse_attn_fwd.  Empty slots
  * (-1), skipped caller ids (out of range, repeated) and blocks with no
  * causal token get 0; over a row's slots the masses sum to 1 (up to fp32
- * rounding) whenever the row attends to any key.  The merge that produces O
- * and lse already holds these shares, so the extra cost is the write of
- * block_mass.
+ * rounding) whenever the row attends to any key.  Cost: on the tensor-core
+ * and decode paths one more kernel per row chunk, after the merge, reads the
+ * chunk's per-(row, head, slot) partial LSEs (4 bytes each: about 1.1 GB at
+ * T = 131072, Hq = 64, topk = 32) and writes block_mass; the CUDA-core path
+ * keeps per-block sums in the attention kernel itself.
  *
  * block_mass [B, T, G, topk] float32 (written; 16-byte aligned).  Every other
  * argument, layout and error is that of msa_sparse_attn_fwd / msa_forward
@@ -207,18 +212,26 @@ MSA_EXPORT msa_status_t msa_forward_mass(const msa_params_t *params, const void 
 MSA_EXPORT msa_status_t msa_get_device_error(void *workspace, void *stream);
 
 /*
- * msa_forward for callers that cannot allocate device memory: code that
- * runs where cudaMalloc is unavailable or forbidden (for example inside a
- * host callback, a custom allocator's own hooks, or an embedding runtime
- * that owns all device allocations), or that must not add allocations to a
- * tightly budgeted process.  The paper has no counterpart of this call.
+ * msa_forward for callers that cannot allocate device memory: a custom
+ * allocator's own hooks (which must not re-enter the allocator they
+ * implement), an embedding runtime that owns every device allocation of the
+ * process, or code that must not add allocations to a tightly budgeted
+ * process.  The call must still be made from an ordinary host thread: CUDA
+ * forbids CUDA API calls inside a host function enqueued on a stream
+ * (cudaLaunchHostFunc or a stream callback), and this call makes several
+ * (device query, symbol lookup, memset, kernel launches).  The paper has no
+ * counterpart of this call.
  *
- * Same meaning, layouts and outputs as msa_forward, but no workspace is
- * passed: the block scores, ids and error word live in a fixed scratch
- * array of MSA_NOALLOC_SCRATCH_BYTES that the library defines as a device
- * global.  Every GPU that loads the library holds that array until the
- * process exits.  The call itself allocates nothing (no cudaMalloc, no
- * cudaFree, no allocating library routine).
+ * Same meaning and layouts as msa_forward, but no workspace is passed: the
+ * block scores, ids and error word live in a fixed scratch array of
+ * MSA_NOALLOC_SCRATCH_BYTES that the library defines as a device global.
+ * Every GPU that loads the library holds that array until the process
+ * exits.  The call itself allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).  It always runs the CUDA-core kernels (the
+ * ones msa_forward uses for fp32): its block ids are bitwise those of
+ * msa_forward, and for bf16 its O and lse agree with msa_forward's within
+ * the bf16 tolerance (max-abs 2e-2 on O, 2e-3 on lse) rather than bitwise;
+ * it is much slower than msa_forward on the tensor-core shapes.
  *   - Shapes whose scratch (msa_workspace_size(params, MSA_WS_FORWARD))
  *     exceeds MSA_NOALLOC_SCRATCH_BYTES are rejected with MSA_ERR_WORKSPACE
  *     before anything is enqueued.
@@ -229,8 +242,10 @@ MSA_EXPORT msa_status_t msa_get_device_error(void *workspace, void *stream);
  *     call's contents.  Calls that may overlap on the GPU (different
  *     streams, or host threads racing on the same device) race on it:
  *     serialise them.
- *   - The call clears the error word itself; the ids come from the call's
- *     own Top-k, so no caller id is checked.
+ *   - The call clears the array's error word before its kernels run.  No
+ *     call reads that word back (msa_get_device_error takes a caller
+ *     workspace), so device-side errors of this call cannot be observed;
+ *     the ids come from the call's own Top-k, so none are expected.
  */
 #define MSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 MSA_EXPORT msa_status_t msa_forward_noalloc(const msa_params_t *params, const void *q_idx,

@@ -41,9 +41,10 @@ def oracle_mass_rows(inp, w, rows, ids_rows, lse_rows):
     return out
 
 
-def oracle_rows(inp, w, rows, *, want_scores=False, ids=None):
+def oracle_rows(inp, w, rows, *, want_scores=False, ids=None, scale=0.0):
     """Run the oracle for `rows` (r = b * T + t) of the inputs `inp` (device or
-    host tensors).  Returns dict of numpy arrays indexed like `rows`."""
+    host tensors), with softmax scale `scale` (<= 0: 1/sqrt(d)).  Returns dict
+    of numpy arrays indexed like `rows`."""
     rows = np.asarray(sorted(rows), dtype=np.int64)
     T = w.T
     out = {"rows": rows, "ids": [], "O": [], "lse": [], "bs": []}
@@ -60,7 +61,7 @@ def oracle_rows(inp, w, rows, *, want_scores=False, ids=None):
         Q = inp.Q[b].index_select(0, tt.to(inp.Q.device)).cpu()
         if ids is None:
             res = orc.forward(q_idx, k_idx, Q, K, V, ts, T=T, block=w.block, topk=w.topk,
-                              want_scores=want_scores)
+                              want_scores=want_scores, scale=scale)
             out["ids"].append(res[0])
             out["O"].append(res[1])
             out["lse"].append(res[2])
@@ -68,7 +69,7 @@ def oracle_rows(inp, w, rows, *, want_scores=False, ids=None):
                 out["bs"].append(res[3])
         else:
             id_rows = ids[b].index_select(0, tt.to(ids.device)).cpu().numpy()
-            O, lse = orc.attention(Q, K, V, id_rows, ts, T=T, block=w.block)
+            O, lse = orc.attention(Q, K, V, id_rows, ts, T=T, block=w.block, scale=scale)
             out["ids"].append(id_rows)
             out["O"].append(O)
             out["lse"].append(lse)
@@ -83,6 +84,19 @@ def gather_rows(x, rows, T):
     idx = torch.as_tensor(np.asarray(sorted(rows)), device=x.device)
     return flat.index_select(0, idx).float().cpu().numpy() if x.dtype != torch.int32 else \
         flat.index_select(0, idx).cpu().numpy()
+
+
+def assert_bits_equal(got, want, where=""):
+    """Block scores compared by bit pattern (as float64): -0.0 differs from
+    +0.0 here, which a numeric comparison would hide."""
+    g = np.ascontiguousarray(got, dtype=np.float64).view(np.int64)
+    w = np.ascontiguousarray(want, dtype=np.float64).view(np.int64)
+    if not np.array_equal(g, w):
+        bad = np.argwhere(g != w)
+        r = tuple(bad[0])
+        raise AssertionError(f"{where}: block score bits differ at {len(bad)} places; first "
+                             f"{r}: got {float(np.asarray(got)[r])!r} want "
+                             f"{float(np.asarray(want)[r])!r}")
 
 
 def assert_ids_equal(got, want, where=""):

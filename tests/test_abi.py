@@ -72,6 +72,7 @@ BAD_SHAPES = [
     (dict(T=0), 1), (dict(T=512), 1), (dict(Hq=6, Hkv=4), 1), (dict(topk=0), 1),
     (dict(B=-1), 1), (dict(S=320), 2), (dict(d=96), 2), (dict(block=32), 2),
     (dict(d_idx=24), 2), (dict(Hq=64, Hkv=2), 2), (dict(topk=1000), 2),
+    (dict(Hq=512, Hkv=512), 2),
 ]
 
 

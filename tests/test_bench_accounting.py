@@ -78,10 +78,31 @@ def test_decode_bytes(bench):
     assert kidx + kv < b < (kidx + kv) * 1.01
 
 
+def test_kept_slots(bench):
+    W = _workloads().Workload
+    w = W("t", B=2, T=50, S=200, Hq=8, Hkv=2, d=16, d_idx=8, block=32, topk=3,
+          dtype=torch.bfloat16)
+    want = w.B * w.G * sum(min(w.topk, (w.S - w.T + t) // w.block + 1) for t in range(w.T))
+    assert bench.kept_slots(w) == want
+
+
 def test_measured_traffic_guard(bench, monkeypatch):
-    m = bench.measured_traffic("prefill_128k")
-    assert m is not None and m["bytes"] == m["read_bytes"] + m["write_bytes"]
-    assert bench.measured_traffic("prefill_32k") is None
-    bad = dict(bench.MEASURED_TRAFFIC["prefill_128k"], source_sha256="0" * 64)
-    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "prefill_128k", bad)
-    assert bench.measured_traffic("prefill_128k") is None
+    """The per-slot capture scales with a call's kept slots, and is dropped
+    once the attention source no longer has the captured hash."""
+    import hashlib
+    src = "block_sparse_long_03_b200/csrc/attn_tc.cu"
+    with open(os.path.join(ROOT, src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    fake = {"source": src, "source_sha256": sha, "workload": "prefill_32k_h64", "slots": 1000,
+            "kernels": {"attn_tc_kernel": {"read": 3000.0, "write": 5000.0},
+                        "combine_kernel": {"read": 6000.0, "write": 500.0}}}
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", fake)
+    w = _workloads().WORKLOADS["prefill_128k"]
+    m = bench.measured_traffic(w)
+    slots = bench.kept_slots(w)
+    assert m is not None and abs(m["read_bytes"] - 9.0 * slots) < 1e-3 * slots
+    assert abs(m["write_bytes"] - 5.5 * slots) < 1e-3 * slots
+    assert m["bytes"] == m["read_bytes"] + m["write_bytes"]
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", dict(fake, source_sha256="0" * 64))
+    assert bench.measured_traffic(w) is None
+

@@ -3,6 +3,8 @@ decode), in the launch configuration the benchmark times (msa_forward on
 device-resident inputs), against the oracle on a sample of rows; plus properties checked on EVERY row: each (row, group)
 keeps exactly min(k, cb + 1) distinct ascending ids, all <= cb, with cb
 among them, and LSE is finite."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -55,6 +57,42 @@ def test_workload_full_size(name):
                         ref["O"], ref["lse"], w.dtype, name)
     del inp, O, lse, ids, ws
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", [
+    "prefill_32k", "chunked_prefill_1m",
+    # about 10 minutes of oracle time on 16 host threads: run on request
+    pytest.param("prefill_128k", marks=[pytest.mark.slow, pytest.mark.skipif(
+        os.environ.get("MSA_FULL_ROWS_128K") != "1",
+        reason="set MSA_FULL_ROWS_128K=1 for the full-row 128K check")]),
+])
+def test_every_row_ids_match_oracle(name):
+    """Block selection of EVERY (row, group) at full size, in the launch
+    configuration the benchmark times (msa_forward on device-resident
+    inputs), bit-exact against the oracle's block scores and selection."""
+    import block_sparse_long_03_b200 as msa
+    import oracle as orc
+    from block_sparse_long_03_b200 import synthetic
+    w = synthetic.WORKLOADS[name]
+    torch.cuda.empty_cache()
+    inp = synthetic.make_inputs(w, seed=0, device="cuda")
+    O, lse, ids, ws = msa.forward(inp.q_idx, inp.k_idx, inp.Q, inp.K, inp.V, block=w.block,
+                                  topk=w.topk)
+    torch.cuda.synchronize()
+    assert msa.msa_get_device_error(ws) == 0
+    got = ids.cpu().numpy()
+    q_idx = inp.q_idx.cpu()
+    k_idx = inp.k_idx.cpu()
+    del inp, O, lse, ids, ws
+    torch.cuda.empty_cache()
+    step = 1024
+    for b in range(w.B):
+        for t0 in range(0, w.T, step):
+            ts = np.arange(t0, min(w.T, t0 + step), dtype=np.int64)
+            bs = orc.block_scores(q_idx[b, t0:t0 + len(ts)], k_idx[b:b + 1], ts, T=w.T,
+                                  block=w.block)
+            ref = orc.select_blocks(bs, ts, T=w.T, S=w.S, block=w.block, topk=w.topk)
+            parity.assert_ids_equal(got[b, t0:t0 + len(ts)], ref, f"{name} rows {t0}..")
 
 
 def test_forward_scores_in_pieces():

@@ -114,7 +114,7 @@ def test_index_scores_and_topk_calls(name):
     rows = list(range(w.B * w.T))
     ref = parity.oracle_rows(inp, w, rows, want_scores=True)
     got = parity.gather_rows(bs, rows, w.T)
-    assert np.array_equal(got.astype(np.float64), ref["bs"]), "block scores differ"
+    parity.assert_bits_equal(got, ref["bs"], name)
     ref_bs = torch.from_numpy(ref["bs"].astype(np.float32)).reshape(w.B, w.T, w.G, w.NB).cuda()
     ids = msa.topk_blocks(ref_bs, S=w.S, block=w.block, topk=w.topk)
     parity.assert_ids_equal(parity.gather_rows(ids, rows, w.T), ref["ids"], name)

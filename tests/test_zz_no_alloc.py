@@ -64,6 +64,35 @@ def test_noalloc_matches_forward_on_two_calls():
         assert torch.equal(O2, O) and torch.equal(lse2, lse)
 
 
+def test_noalloc_many_groups():
+    """32 GQA groups (more than the 16 the CUDA-core index tile took before it
+    sized its query tile by the group count): ids bitwise those of
+    msa_forward, O and lse within the bf16 tolerance."""
+    import block_sparse_long_03_b200 as msa
+    from block_sparse_long_03_b200 import binding, synthetic
+    lib = binding.lib
+    w = synthetic.Workload("noalloc_g32", B=1, T=192, S=256, Hq=32, Hkv=32, d=128, d_idx=64,
+                           block=64, topk=3, dtype=torch.bfloat16)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    inp = synthetic.make_inputs(w, 21, device="cuda")
+    p = msa.params_from(inp.q_idx, inp.Q, inp.K, block=w.block, topk=w.topk)
+    O_ref, lse_ref, ids_ref, ws = msa.forward(inp.q_idx, inp.k_idx, inp.Q, inp.K, inp.V,
+                                              block=w.block, topk=w.topk)
+    O = torch.empty_like(inp.Q)
+    lse = torch.empty(inp.Q.shape[:3], dtype=torch.float32, device="cuda")
+    ids = torch.empty((w.B, w.T, w.G, w.topk), dtype=torch.int32, device="cuda")
+    rc = lib.msa_forward_noalloc(ctypes.byref(p), _ptr(inp.q_idx), _ptr(inp.k_idx), _ptr(inp.Q),
+                                 _ptr(inp.K), _ptr(inp.V), _ptr(ids), _ptr(O), _ptr(lse), stream)
+    assert rc == 0, binding.status_string(rc)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ids_ref)
+    rows = list(range(w.B * w.T))
+    parity.assert_close(parity.gather_rows(O, rows, w.T), parity.gather_rows(lse, rows, w.T),
+                        parity.gather_rows(O_ref, rows, w.T).astype(np.float64),
+                        parity.gather_rows(lse_ref, rows, w.T).astype(np.float64),
+                        w.dtype, "noalloc G=32")
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     import block_sparse_long_03_b200 as msa
     from block_sparse_long_03_b200 import binding
