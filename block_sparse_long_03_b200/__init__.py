@@ -17,8 +17,9 @@ if not _os.path.exists(_LIB):
                       "(run python block_sparse_long_03_b200/build.py)")
 
 __all__ = [
-    "EXPORTS", "MSA_BF16", "MSA_F32", "MSA_OK", "MSA_WS_FORWARD", "MSA_WS_FORWARD_HOST",
-    "MSA_WS_SPARSE_ATTN", "MsaError", "Params", "alloc_workspace", "forward",
+    "EXPORTS", "MSA_BF16", "MSA_F32", "MSA_OK", "MSA_WS_DECODE_PAGED", "MSA_WS_FORWARD",
+    "MSA_WS_FORWARD_HOST", "MSA_WS_SPARSE_ATTN", "MsaError", "Params", "alloc_workspace",
+    "decode_paged", "forward", "msa_decode_paged",
     "forward_with_mass", "index_block_scores", "make_params", "msa_forward", "msa_forward_host",
     "msa_forward_mass", "msa_query_pieces", "msa_sparse_attn_fwd_mass",
     "msa_get_device_error", "msa_index_block_scores", "msa_kernel_launches",

@@ -18,16 +18,17 @@ LIB_PATH = os.path.join(_HERE, "libmsa.so")
 
 MSA_OK = 0
 MSA_F32, MSA_BF16 = 0, 1
-MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD, MSA_WS_FORWARD_HOST = 0, 1, 2
+MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD, MSA_WS_FORWARD_HOST, MSA_WS_DECODE_PAGED = 0, 1, 2, 3
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
-                4: "MSA_ERR_DEVICE_TIMEOUT", 5: "MSA_ERR_WORKSPACE", 6: "MSA_ERR_BAD_BLOCK_IDS"}
+                4: "MSA_ERR_DEVICE_TIMEOUT", 5: "MSA_ERR_WORKSPACE", 6: "MSA_ERR_BAD_BLOCK_IDS",
+                7: "MSA_ERR_BAD_PAGE_TABLE"}
 
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
            "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
            "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass",
-           "msa_query_pieces")
+           "msa_query_pieces", "msa_decode_paged")
 
 
 class MsaError(RuntimeError):
@@ -67,6 +68,9 @@ def _load():
     lib.msa_sparse_attn_fwd_mass.restype = st
     lib.msa_forward_mass.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.msa_forward_mass.restype = st
+    i32 = ctypes.c_int32
+    lib.msa_decode_paged.argtypes = [P, vp, vp, i32, i32, i32] + [vp] * 8 + [vp, sz, vp]
+    lib.msa_decode_paged.restype = st
     lib.msa_query_pieces.argtypes = [P, ctypes.c_int, vp, ctypes.c_int64]
     lib.msa_query_pieces.restype = ctypes.c_int64
     lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
@@ -182,6 +186,19 @@ def msa_forward_host(params: Params, q_idx, k_idx, Q, K, V, block_ids, O, lse, d
            "msa_forward_host")
 
 
+def msa_decode_paged(params: Params, seq_lens, block_table, page_size: int, num_pages: int,
+                     q_idx, k_idx_cache, Q, K_cache, V_cache, block_ids, O, lse, workspace,
+                     stream=None):
+    """Decode steps over a paged cache: seq_lens [B] and block_table
+    [B, max_pages] int32 CUDA tensors; caches [num_pages, page_size, ...]."""
+    _check(lib.msa_decode_paged(ctypes.byref(params), _ptr(seq_lens), _ptr(block_table),
+                                int(page_size), int(block_table.shape[1]), int(num_pages),
+                                _ptr(q_idx), _ptr(k_idx_cache), _ptr(Q), _ptr(K_cache),
+                                _ptr(V_cache), _ptr(block_ids), _ptr(O), _ptr(lse),
+                                _ptr(workspace), workspace.numel(), _stream(stream)),
+           "msa_decode_paged")
+
+
 def msa_get_device_error(workspace, stream=None) -> int:
     """The status recorded on the device by the last call that used `workspace`."""
     return int(lib.msa_get_device_error(_ptr(workspace), _stream(stream)))
@@ -264,3 +281,21 @@ def forward_with_mass(q_idx, k_idx, Q, K, V, *, block: int, topk: int, scale: fl
     ws = alloc_workspace(p, MSA_WS_FORWARD, Q.device)
     msa_forward_mass(p, q_idx, k_idx, Q, K, V, ids, O, lse, mass, ws)
     return O, lse, ids, mass, ws
+
+
+def decode_paged(q_idx, k_idx_cache, Q, K_cache, V_cache, seq_lens, block_table, *, S: int,
+                 block: int, topk: int, scale: float = 0.0):
+    """Decode steps over a paged KV cache with per-sequence lengths; returns
+    (O, lse, block_ids, workspace).  S is the capacity (a multiple of block,
+    at most block_table.shape[1] * page_size)."""
+    B, T, Hq, d = Q.shape
+    num_pages, page_size, Hkv, _ = K_cache.shape
+    p = make_params(B=B, T=T, S=S, Hq=Hq, Hkv=Hkv, d=d, d_idx=q_idx.shape[-1], block=block,
+                    topk=topk, dtype=Q.dtype, scale=scale)
+    O = torch.empty_like(Q)
+    lse = torch.empty((B, T, Hq), dtype=torch.float32, device=Q.device)
+    ids = torch.empty((B, T, Hkv, topk), dtype=torch.int32, device=Q.device)
+    ws = alloc_workspace(p, MSA_WS_DECODE_PAGED, Q.device)
+    msa_decode_paged(p, seq_lens, block_table, page_size, num_pages, q_idx, k_idx_cache, Q,
+                     K_cache, V_cache, ids, O, lse, ws)
+    return O, lse, ids, ws

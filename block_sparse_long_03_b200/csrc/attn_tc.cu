@@ -643,7 +643,8 @@ __global__ void __launch_bounds__(256, kMaxPer <= 8 ? 3 : 2)
 combine_kernel(const int32_t *__restrict__ ids, const __nv_bfloat16 *__restrict__ part_o,
                                const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
                                float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
-                               int Hq, int G, int R, int NB, int block, int topk) {
+                               int Hq, int G, int R, int NB, int block, int topk,
+                               const int32_t *__restrict__ lens) {
     constexpr int kChunksPerWarp = 4;             // kMaxPer: slots per lane, >= topk * R / 32
     constexpr int kWarpsPerRow = D / 8 / kChunksPerWarp;
     const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
@@ -655,7 +656,8 @@ combine_kernel(const int32_t *__restrict__ ids, const __nv_bfloat16 *__restrict_
     const int g = (int)(rgl % G);
     const int64_t r = r0 + rl;
     const int t = (int)(r % T_);
-    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / block);
     const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
     const int h = lane % R, s0 = lane / R, sstep = 32 / R;
     const int per = (topk + sstep - 1) / sstep;
@@ -731,14 +733,16 @@ combine_kernel(const int32_t *__restrict__ ids, const __nv_bfloat16 *__restrict_
 __global__ void __launch_bounds__(256)
 block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ part_lse,
                   const float *__restrict__ lse, float *__restrict__ mass, int64_t r0, int64_t rc,
-                  int T_, int S, int Hq, int G, int R, int NB, int block, int topk) {
+                  int T_, int S, int Hq, int G, int R, int NB, int block, int topk,
+                  const int32_t *__restrict__ lens) {
     const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
     const int64_t rl = x / G, r = r0 + rl;
     const int g = (int)(x % G);
     const int t = (int)(r % T_);
-    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / block);
     const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
     const int h = lane % R, s0 = lane / R, sstep = 32 / R;
     const int per = (topk + sstep - 1) / sstep;
@@ -874,20 +878,20 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
-                           cudaStream_t st, float *mass) {
+                           cudaStream_t st, float *mass, const int32_t *lens) {
     const int64_t warps = rc * s.G * (128 / 32);
     const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
     const int per = (s.topk + 32 / s.R - 1) / (32 / s.R);
     auto kern = per <= 8 ? combine_kernel<128, 8> : combine_kernel<128, 16>;
     kern<<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S,
-                               s.Hq, s.G, s.R, s.NB, s.block, s.topk);
+                               s.Hq, s.G, s.R, s.NB, s.block, s.topk, lens);
     count_launches(1);
     if (mass != nullptr) {
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const unsigned mgrid = (unsigned)((rc * s.G * 32 + 255) / 256);
         block_mass_kernel<<<mgrid, 256, 0, st>>>(ids, part_lse, lse, mass, r0, rc, s.T, s.S, s.Hq,
-                                                 s.G, s.R, s.NB, s.block, s.topk);
+                                                 s.G, s.R, s.NB, s.block, s.topk, lens);
         count_launches(1);
     }
     return cudaGetLastError();

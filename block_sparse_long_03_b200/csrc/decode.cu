@@ -70,12 +70,14 @@ __device__ __forceinline__ int swz(int r, int c, int row_bytes) {
 
 // One warp scores whole KV blocks of one sequence, 64 keys (a "sub-block")
 // at a time, against up to 8*NCG (token, group) columns; sub-blocks are
-// double-buffered in shared memory.
+// double-buffered in shared memory.  Key rows are found through `rows`
+// (dense or paged); keys at or past the sequence's length L are never read
+// (zero in shared memory, and masked: every query sits before L).
 template <int DIDX, int NCG, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32)
 decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
                     float *__restrict__ bs, int T_, int S, int G, int NB, int block,
-                    int blocks_per_warp) {
+                    int blocks_per_warp, KeyRows rows, const int32_t *__restrict__ lens) {
     constexpr int kRowBytes = DIDX * 2;
     constexpr int kChunks = DIDX / 8;
     constexpr int kSub = 64;                               // keys per staged sub-block
@@ -86,6 +88,16 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
     const int TG = T_ * G;
     uint8_t *buf0 = sm + (size_t)warp * 2 * kTileBytes;
     const int g4 = lane / 4, t4 = lane % 4;
+    const int64_t L = seq_len(lens, b, S);
+    const int first_blk = (blockIdx.x * WARPS + warp) * blocks_per_warp;
+    const int last_blk = min(NB, first_blk + blocks_per_warp);
+    if ((int64_t)first_blk * block >= L) {                 // no key of these blocks exists
+        for (int i = lane; i < (last_blk - first_blk) * TG; i += 32) {
+            const int col = i % TG, n = first_blk + i / TG;
+            bs[((int64_t)b * TG + col) * NB + n] = -INFINITY;
+        }
+        return;
+    }
 
     // B fragments: column n = 8 * cg + g4 is (token, group) pair n of this sequence
     uint32_t bq[NCG][DIDX / 16][2];
@@ -110,18 +122,20 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int n = cg * 8 + 2 * t4 + e;
-            pcol[cg][e] = (int64_t)S - T_ + (n < TG ? n / G : 0);
+            pcol[cg][e] = L - T_ + (n < TG ? n / G : 0);
         }
 
     const int spb = block / kSub;                          // sub-blocks per block
-    const int first_blk = (blockIdx.x * WARPS + warp) * blocks_per_warp;
-    const int last_blk = min(NB, first_blk + blocks_per_warp);
     const int first = first_blk * spb, last = last_blk * spb;
     auto stage = [&](int sb, uint8_t *dst) {
-        const __nv_bfloat16 *src = k_idx + ((int64_t)b * S + (int64_t)sb * kSub) * DIDX;
         for (int c = lane; c < kSub * kChunks; c += 32) {
             const int r = c / kChunks, ch = c % kChunks;
-            cp_async16(dst + swz(r, ch, kRowBytes), src + (int64_t)r * DIDX + ch * 8);
+            const int64_t j = (int64_t)sb * kSub + r;
+            const int64_t row = j < L ? rows.row(b, j) : -1;
+            if (row >= 0)
+                cp_async16(dst + swz(r, ch, kRowBytes), k_idx + row * DIDX + ch * 8);
+            else
+                *(uint4 *)(dst + swz(r, ch, kRowBytes)) = make_uint4(0u, 0u, 0u, 0u);
         }
         cp_async_commit();
     };
@@ -193,7 +207,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
                     const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ ids,
                     __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_lse, uint32_t *err,
                     int T_, int S, int Hq, int Hkv, int R, int NB, int topk, float scale_log2,
-                    float scale, int64_t n_prows) {
+                    float scale, int64_t n_prows, KeyRows rows, const int32_t *__restrict__ lens) {
     constexpr int kRowBytes = D * 2;
     constexpr int kChunks = D / 8;
     extern __shared__ __align__(128) uint8_t sm[];
@@ -212,7 +226,8 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     const int g = (int)(rg % Hkv);
     const int64_t bt = rg / Hkv;
     const int b = (int)(bt / T_), t = (int)(bt % T_);
-    const int64_t p = (int64_t)S - T_ + t;
+    const int64_t p = seq_len(lens, b, S) - T_ + t;
+    if (p < 0) return;                                     // a sequence marked as doing no work
     const int cb = (int)(p / BLOCK);
     const int32_t *row = ids + rg * topk;
     // validity of this slot (same rule as every other phase): the range is
@@ -231,8 +246,9 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     // stage K and V rows of the block (zero rows past the last causal key)
     for (int c = tid; c < BLOCK * kChunks; c += kAttnThreads) {
         const int r = c / kChunks, ch = c % kChunks;
-        if (r < nk) {
-            const int64_t src = (((int64_t)b * S + j0 + r) * Hkv + g) * D + ch * 8;
+        const int64_t kr = r < nk ? rows.row(b, j0 + r) : -1;
+        if (kr >= 0) {
+            const int64_t src = (kr * Hkv + g) * D + ch * 8;
             cp_async16(sK + swz(r, ch, kRowBytes), K + src);
             cp_async16(sV + swz(r, ch, kRowBytes), V + src);
         } else {
@@ -378,7 +394,7 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
 
 template <int DIDX, int NCG>
 cudaError_t launch_index_t(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
-                           cudaStream_t st) {
+                           cudaStream_t st, const KeyRows &rows, const int32_t *lens) {
     constexpr int W = DIDX == 64 ? 8 : 4;
     const size_t smem = (size_t)W * 2 * 64 * DIDX * 2;
     auto k = decode_index_kernel<DIDX, NCG, W>;
@@ -387,26 +403,27 @@ cudaError_t launch_index_t(const Shape &s, const void *q_idx, const void *k_idx,
     const int bpw = 4;                                     // blocks per warp
     const dim3 grid((unsigned)((s.NB + W * bpw - 1) / (W * bpw)), (unsigned)s.B);
     k<<<grid, W * 32, smem, st>>>((const __nv_bfloat16 *)q_idx, (const __nv_bfloat16 *)k_idx, bs,
-                                  s.T, s.S, s.G, s.NB, s.block, bpw);
+                                  s.T, s.S, s.G, s.NB, s.block, bpw, rows, lens);
     count_launches(1);
     return cudaGetLastError();
 }
 
 template <int DIDX>
-cudaError_t launch_index_d(const Shape &s, const void *q, const void *k, float *bs, cudaStream_t st) {
+cudaError_t launch_index_d(const Shape &s, const void *q, const void *k, float *bs, cudaStream_t st,
+                           const KeyRows &rows, const int32_t *lens) {
     const int ncg = (s.T * s.G + 7) / 8;
     switch (ncg) {
-        case 1: return launch_index_t<DIDX, 1>(s, q, k, bs, st);
-        case 2: return launch_index_t<DIDX, 2>(s, q, k, bs, st);
-        case 3: return launch_index_t<DIDX, 3>(s, q, k, bs, st);
-        default: return launch_index_t<DIDX, 4>(s, q, k, bs, st);
+        case 1: return launch_index_t<DIDX, 1>(s, q, k, bs, st, rows, lens);
+        case 2: return launch_index_t<DIDX, 2>(s, q, k, bs, st, rows, lens);
+        case 3: return launch_index_t<DIDX, 3>(s, q, k, bs, st, rows, lens);
+        default: return launch_index_t<DIDX, 4>(s, q, k, bs, st, rows, lens);
     }
 }
 
 template <int BLOCK>
 cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, __nv_bfloat16 *part_o, float *part_lse, uint32_t *err,
-                           cudaStream_t st) {
+                           cudaStream_t st, const KeyRows &rows, const int32_t *lens) {
     constexpr int D = 128;
     const size_t smem = 2 * (size_t)BLOCK * D * 2 + 8 * BLOCK * 2 + 40 * 4 + 8 * D * 2;
     auto k = decode_block_kernel<D, BLOCK>;
@@ -417,9 +434,33 @@ cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const v
     k<<<(unsigned)ctas, kAttnThreads, smem, st>>>(
         (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, ids, part_o,
         part_lse, err, s.T, s.S, s.Hq, s.Hkv, s.R, s.NB, s.topk, scale_log2, s.scale,
-        (int64_t)s.index_rows() * s.topk * s.R);
+        (int64_t)s.index_rows() * s.topk * s.R, rows, lens);
     count_launches(1);
     return cudaGetLastError();
+}
+
+// One warp per sequence of a paged call.
+__global__ void paged_check_kernel(const int32_t *__restrict__ lens, KeyRows rows,
+                                   int32_t *__restrict__ lens_ok, uint32_t *err, int B, int T_,
+                                   int64_t S) {
+    const int b = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32);
+    const int lane = threadIdx.x % 32;
+    if (b >= B) return;
+    const int64_t L = lens[b];
+    bool ok = L >= T_ && L <= S;
+    bool bad_page = false;
+    if (ok) {
+        const int64_t npages = (L + rows.page_size - 1) / rows.page_size;   // <= max_pages
+        for (int64_t i = lane; i < npages; i += 32) {
+            const int pg = rows.table[(int64_t)b * rows.max_pages + i];
+            bad_page |= pg < 0 || pg >= rows.num_pages;
+        }
+    }
+    ok = ok && !__any_sync(0xffffffffu, bad_page);
+    if (lane == 0) {
+        lens_ok[b] = ok ? (int32_t)L : 0;
+        if (!ok) record_error(err, MSA_ERR_BAD_PAGE_TABLE, 3);
+    }
 }
 
 size_t part_bytes_o(const Shape &s) {
@@ -429,15 +470,24 @@ size_t part_bytes_o(const Shape &s) {
 
 }  // namespace
 
+cudaError_t launch_paged_check(const Shape &s, const int32_t *lens, const KeyRows &rows,
+                               int32_t *lens_ok, uint32_t *err, cudaStream_t st) {
+    paged_check_kernel<<<(unsigned)((s.B * 32 + 255) / 256), 256, 0, st>>>(lens, rows, lens_ok,
+                                                                          err, s.B, s.T, s.S);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 bool decode_index_supported(const Shape &s) {
     return s.dtype == MSA_BF16 && (s.d_idx == 64 || s.d_idx == 128) && s.T * s.G <= 32 &&
            (s.block == 64 || s.block == 128);
 }
 
 cudaError_t launch_decode_index(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
-                                cudaStream_t st) {
-    if (s.d_idx == 64) return launch_index_d<64>(s, q_idx, k_idx, bs, st);
-    return launch_index_d<128>(s, q_idx, k_idx, bs, st);
+                                cudaStream_t st, const KeyRows *rows, const int32_t *lens) {
+    const KeyRows r = rows ? *rows : dense_rows(s.S);
+    if (s.d_idx == 64) return launch_index_d<64>(s, q_idx, k_idx, bs, st, r, lens);
+    return launch_index_d<128>(s, q_idx, k_idx, bs, st, r, lens);
 }
 
 bool decode_attn_supported(const Shape &s) {
@@ -451,14 +501,16 @@ size_t decode_attn_workspace(const Shape &s) {
 
 cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
                                const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                               cudaStream_t st, float *mass) {
+                               cudaStream_t st, float *mass, const KeyRows *rows,
+                               const int32_t *lens) {
     __nv_bfloat16 *part_o = (__nv_bfloat16 *)ws;
     float *part_lse = (float *)((char *)ws + part_bytes_o(s));
+    const KeyRows r = rows ? *rows : dense_rows(s.S);
     cudaError_t e = s.block == 64
-                        ? launch_block_t<64>(s, Q, K, V, ids, part_o, part_lse, err, st)
-                        : launch_block_t<128>(s, Q, K, V, ids, part_o, part_lse, err, st);
+                        ? launch_block_t<64>(s, Q, K, V, ids, part_o, part_lse, err, st, r, lens)
+                        : launch_block_t<128>(s, Q, K, V, ids, part_o, part_lse, err, st, r, lens);
     if (e != cudaSuccess) return e;
-    return launch_combine(s, ids, part_o, part_lse, O, lse, 0, s.rows(), st, mass);
+    return launch_combine(s, ids, part_o, part_lse, O, lse, 0, s.rows(), st, mass, lens);
 }
 
 }  // namespace msa

@@ -151,6 +151,9 @@ msa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA
 
 // Device buffer bytes of msa_forward_host (defined with that call below).
 size_t host_ws_size(const Shape &s);
+// Workspace bytes of msa_decode_paged (defined with that call below); 0 when
+// the shapes have no paged path.
+size_t paged_ws_size(const Shape &s);
 
 }  // namespace
 }  // namespace msa
@@ -168,6 +171,7 @@ const char *msa_status_string(msa_status_t status) {
         case MSA_ERR_DEVICE_TIMEOUT: return "MSA_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
         case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE: workspace missing, misaligned or too small";
         case MSA_ERR_BAD_BLOCK_IDS: return "MSA_ERR_BAD_BLOCK_IDS: caller block ids out of range, not causal or repeated";
+        case MSA_ERR_BAD_PAGE_TABLE: return "MSA_ERR_BAD_PAGE_TABLE: a sequence length or page id of a paged call is out of range";
     }
     return "unknown msa_status_t";
 }
@@ -178,6 +182,7 @@ size_t msa_workspace_size(const msa_params_t *params, int which) {
     if (which == MSA_WS_SPARSE_ATTN) return attn_ws(s);
     if (which == MSA_WS_FORWARD) return forward_ws(s);
     if (which == MSA_WS_FORWARD_HOST) return host_ws_size(s);
+    if (which == MSA_WS_DECODE_PAGED) return paged_ws_size(s);
     return 0;
 }
 
@@ -651,4 +656,80 @@ extern "C" int64_t msa_query_pieces(const msa_params_t *params, int which, int32
         pieces[3 * i + 2] = v[i].t1;
     }
     return (int64_t)v.size();
+}
+
+// ---------------------------------------------------------------------------
+// msa_decode_paged: decode steps over a paged KV cache with per-sequence
+// lengths (see include/msa.h).  The decode kernels read every key row
+// through the block table; a check kernel first validates the lengths and
+// the page ids each sequence uses, so no kernel reads an invalid page.
+// ---------------------------------------------------------------------------
+namespace msa {
+namespace {
+
+bool paged_supported(const Shape &s) {
+    return decode_index_supported(s) && decode_attn_supported(s);
+}
+
+// Workspace: [error word][checked lengths][decode attention scratch]
+// [block scores][block ids]
+struct PagedLayout {
+    size_t lens, scratch, bs, ids, total;
+};
+
+PagedLayout paged_layout(const Shape &s) {
+    PagedLayout L;
+    size_t o = kErrorBytes;
+    L.lens = o;    o += align_up(sizeof(int32_t) * (size_t)s.B);
+    L.scratch = o; o += align_up(decode_attn_workspace(s));
+    L.bs = o;      o += align_up(block_score_bytes(s));
+    L.ids = o;     o += align_up(block_id_bytes(s));
+    L.total = o;
+    return L;
+}
+
+size_t paged_ws_size(const Shape &s) { return paged_supported(s) ? paged_layout(s).total : 0; }
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status_t msa_decode_paged(const msa_params_t *params, const int32_t *seq_lens,
+                                         const int32_t *block_table, int32_t page_size,
+                                         int32_t max_pages, int32_t num_pages, const void *q_idx,
+                                         const void *k_idx_cache, const void *Q,
+                                         const void *K_cache, const void *V_cache,
+                                         int32_t *block_ids, void *O, float *lse,
+                                         void *workspace, size_t workspace_bytes, void *stream) {
+    Shape s;
+    msa_status_t rc = make_shape(params, &s);
+    if (rc != MSA_OK) return rc;
+    if (page_size <= 0 || max_pages <= 0 || num_pages <= 0 ||
+        (int64_t)max_pages * page_size < (int64_t)s.S)
+        return MSA_ERR_INVALID_ARG;
+    if (!seq_lens || !block_table || !q_idx || !k_idx_cache || !Q || !K_cache || !V_cache || !O ||
+        !lse)
+        return MSA_ERR_INVALID_ARG;
+    if (!aligned16(seq_lens) || !aligned16(block_table) || !aligned16(q_idx) ||
+        !aligned16(k_idx_cache) || !aligned16(Q) || !aligned16(K_cache) || !aligned16(V_cache) ||
+        !aligned16(O) || !aligned16(lse) || (block_ids && !aligned16(block_ids)))
+        return MSA_ERR_INVALID_ARG;
+    if (!paged_supported(s)) return MSA_ERR_UNSUPPORTED;
+    const PagedLayout L = paged_layout(s);
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < L.total)
+        return MSA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    uint32_t *err = (uint32_t *)ws;
+    int32_t *lens_ok = (int32_t *)(ws + L.lens);
+    float *bs = (float *)(ws + L.bs);
+    int32_t *ids = block_ids ? block_ids : (int32_t *)(ws + L.ids);
+    const KeyRows rows{block_table, (int64_t)s.S, max_pages, page_size, num_pages};
+    cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
+    if (e == cudaSuccess) e = launch_paged_check(s, seq_lens, rows, lens_ok, err, st);
+    if (e == cudaSuccess) e = launch_decode_index(s, q_idx, k_idx_cache, bs, st, &rows, lens_ok);
+    if (e == cudaSuccess) e = launch_topk(s, bs, ids, st, lens_ok);
+    if (e == cudaSuccess)
+        e = launch_decode_attn(s, Q, K_cache, V_cache, ids, O, lse, err, ws + L.scratch, st,
+                               nullptr, &rows, lens_ok);
+    return cuda_status(e);
 }

@@ -24,6 +24,7 @@ struct Shape {
 //   word[0]: first recorded msa_status_t (0 = none)
 //   word[1]: number of caller block ids skipped as invalid
 //   word[2]: number of bounded device waits that gave up
+//   word[3]: number of sequences a paged call skipped (bad length or page id)
 constexpr size_t kErrorBytes = 256;
 
 __device__ __forceinline__ void record_error(uint32_t *err, uint32_t code, int counter) {
@@ -50,6 +51,30 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Where key row j (0 <= j < its sequence's length) of sequence b lives in
+// the index-key, K and V arrays: sequences of S rows one after another
+// (table == nullptr), or pages of page_size rows found through a block
+// table [B, max_pages] of page ids (the paged KV cache of msa_decode_paged).
+struct KeyRows {
+    const int32_t *table;
+    int64_t S;
+    int max_pages, page_size, num_pages;
+    // the row index, or -1 when the page id is out of range (never loaded)
+    __device__ __forceinline__ int64_t row(int b, int64_t j) const {
+        if (table == nullptr) return (int64_t)b * S + j;
+        const int pg = __ldg(table + (int64_t)b * max_pages + j / page_size);
+        if (pg < 0 || pg >= num_pages) return -1;
+        return (int64_t)pg * page_size + j % page_size;
+    }
+};
+inline KeyRows dense_rows(int64_t S) { return KeyRows{nullptr, S, 0, 1, 0}; }
+
+// Keys of sequence b: lens[b] when per-sequence lengths are given (a length
+// of 0 marks a sequence that does no work), S otherwise.
+__device__ __forceinline__ int64_t seq_len(const int32_t *lens, int b, int64_t S) {
+    return lens == nullptr ? S : (int64_t)__ldg(lens + b);
+}
+
 // Every kernel launch of the library is counted (msa_kernel_launches).
 void count_launches(int n);
 
@@ -61,6 +86,8 @@ bool index_tc_supported(const Shape &s);
 cudaError_t launch_index_scores_tc(const Shape &s, const void *q_idx, const void *k_idx,
                                    float *bs, bool fill_noncausal, uint32_t *err,
                                    cudaStream_t st);
+// lens (optional, [B]): per-sequence key counts (query t of sequence b then
+// sits at lens[b] - T + t; a length of 0 leaves the sequence's ids at -1).
 // Tensor-core KV-block-outer sparse attention (bf16, d = 128) and its workspace.
 bool attn_tc_supported(const Shape &s);
 size_t attn_tc_workspace(const Shape &s);
@@ -87,18 +114,27 @@ bool combine_supported(const Shape &s);
 // for query rows [r0, r0 + rc) (d = 128).
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
-                           cudaStream_t st, float *mass = nullptr);
+                           cudaStream_t st, float *mass = nullptr,
+                           const int32_t *lens = nullptr);
 // Decode path (few query tokens per sequence): HBM-streaming index scoring and
 // one-CTA-per-kept-block attention feeding the same combine.
 bool decode_index_supported(const Shape &s);
 cudaError_t launch_decode_index(const Shape &s, const void *q_idx, const void *k_idx, float *bs,
-                                cudaStream_t st);
+                                cudaStream_t st, const KeyRows *rows = nullptr,
+                                const int32_t *lens = nullptr);
 bool decode_attn_supported(const Shape &s);
 size_t decode_attn_workspace(const Shape &s);
 cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, const void *V,
                                const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
-                               cudaStream_t st, float *mass = nullptr);
-cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st);
+                               cudaStream_t st, float *mass = nullptr,
+                               const KeyRows *rows = nullptr, const int32_t *lens = nullptr);
+cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st,
+                        const int32_t *lens = nullptr);
+// Page-table check of a paged call: lens_ok[b] = lens[b] when s.T <= lens[b]
+// <= s.S and every page id the sequence uses lies in [0, rows.num_pages),
+// otherwise 0 (the sequence does no work) with MSA_ERR_BAD_PAGE_TABLE recorded.
+cudaError_t launch_paged_check(const Shape &s, const int32_t *lens, const KeyRows &rows,
+                               int32_t *lens_ok, uint32_t *err, cudaStream_t st);
 cudaError_t launch_attn_simt(const Shape &s, const void *Q, const void *K, const void *V,
                              const int32_t *ids, void *O, float *lse, uint32_t *err,
                              cudaStream_t st, float *mass = nullptr);

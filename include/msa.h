@@ -59,7 +59,8 @@ typedef enum {
     MSA_ERR_CUDA = 3,            /* a CUDA runtime call failed                */
     MSA_ERR_DEVICE_TIMEOUT = 4,  /* a bounded device wait gave up             */
     MSA_ERR_WORKSPACE = 5,       /* workspace missing or too small            */
-    MSA_ERR_BAD_BLOCK_IDS = 6    /* caller ids out of range / not causal      */
+    MSA_ERR_BAD_BLOCK_IDS = 6,   /* caller ids out of range / not causal      */
+    MSA_ERR_BAD_PAGE_TABLE = 7   /* paged call: a length or page id invalid   */
 } msa_status_t;
 
 typedef enum { MSA_F32 = 0, MSA_BF16 = 1 } msa_dtype_t;
@@ -119,9 +120,10 @@ MSA_EXPORT msa_status_t msa_topk_blocks(const msa_params_t *params, const float 
                              int32_t *block_ids, void *stream);
 
 /* Workspace needs, in bytes, of msa_sparse_attn_fwd (which = 0) and
- * msa_forward (which = 1) for these shapes, or the device buffer of
- * msa_forward_host (which = 2, MSA_WS_FORWARD_HOST, defined with that call);
- * 0 for invalid shapes. */
+ * msa_forward (which = 1) for these shapes, the device buffer of
+ * msa_forward_host (which = 2, MSA_WS_FORWARD_HOST, defined with that call)
+ * or the workspace of msa_decode_paged (which = 3, MSA_WS_DECODE_PAGED);
+ * 0 for invalid shapes or shapes the call does not support. */
 #define MSA_WS_SPARSE_ATTN 0
 #define MSA_WS_FORWARD 1
 MSA_EXPORT size_t msa_workspace_size(const msa_params_t *params, int which);
@@ -299,6 +301,57 @@ MSA_EXPORT msa_status_t msa_forward_host(const msa_params_t *params, const void 
                                          const void *V, int32_t *block_ids, void *O, float *lse,
                                          void *device_buffer, size_t device_buffer_bytes,
                                          void *stream);
+
+/*
+ * Decode steps over a PAGED KV cache with per-sequence lengths: the forward
+ * pass of msa_forward (index scores, per-group Top-k with the current block
+ * kept, sparse attention with LSE) for a batch of sequences of different
+ * lengths whose index keys, K and V live in fixed-size pages.  The method is
+ * that of "MiniMax Sparse Attention" (Summary, second paragraph; Key points,
+ * "Efficiency at 1M context": decoding); the paged layout and the variable
+ * lengths have no counterpart in the paper and follow common serving
+ * practice.
+ *
+ * Sequence b holds L_b = seq_lens[b] keys; its key j (0 <= j < L_b) is row
+ * j % page_size of page block_table[b, j / page_size] in each cache.  Its T
+ * query tokens sit at positions L_b - T + t (the last T positions), so
+ * cb(t) = (L_b - T + t) / block and every definition above applies with S
+ * replaced by L_b.  L_b need not be a multiple of block: the last block of
+ * a sequence may be partial (its missing keys do not exist, and no query
+ * sits past them).  Outputs are those of msa_forward on each sequence's
+ * keys laid out densely.
+ *
+ * params: B sequences, T query tokens each (T * Hkv <= 32), S the capacity:
+ *   a multiple of block with T <= L_b <= S; bf16, d = 128, d_idx in {64, 128}
+ *   (otherwise MSA_ERR_UNSUPPORTED).
+ * seq_lens     [B]                               int32 (device, read)
+ * block_table  [B, max_pages]                    int32 (device, read); only
+ *              the first ceil(L_b / page_size) entries of row b are read
+ * page_size, max_pages, num_pages: max_pages * page_size >= S; page ids
+ *              must lie in [0, num_pages)
+ * q_idx        [B, T, G, d_idx]                  dtype (read)
+ * k_idx_cache  [num_pages, page_size, d_idx]     dtype (read)
+ * Q            [B, T, Hq, d]                     dtype (read)
+ * K_cache, V_cache [num_pages, page_size, Hkv, d] dtype (read)
+ * block_ids    [B, T, G, topk] int32 (written; may be NULL)
+ * O            [B, T, Hq, d] (written), lse [B, T, Hq] float32 (written)
+ * workspace    msa_workspace_size(params, MSA_WS_DECODE_PAGED) bytes,
+ *              256-byte aligned; first 256 bytes: the device error word.
+ *
+ * The lengths and page ids are checked on the device before any key is
+ * read: a sequence whose length is outside [T, S] or which uses a page id
+ * outside [0, num_pages) is skipped (its ids -1, O = 0, lse = -infinity)
+ * and the error word records MSA_ERR_BAD_PAGE_TABLE; the other sequences
+ * are computed as usual.
+ */
+#define MSA_WS_DECODE_PAGED 3
+MSA_EXPORT msa_status_t msa_decode_paged(const msa_params_t *params, const int32_t *seq_lens,
+                                         const int32_t *block_table, int32_t page_size,
+                                         int32_t max_pages, int32_t num_pages, const void *q_idx,
+                                         const void *k_idx_cache, const void *Q,
+                                         const void *K_cache, const void *V_cache,
+                                         int32_t *block_ids, void *O, float *lse,
+                                         void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Diagnostics: the query pieces a call splits its work into, computed on the

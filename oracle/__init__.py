@@ -51,8 +51,11 @@ def bind(path: str):
     lib.oracle_attention.argtypes = [i64] * 8 + [i32, dbl, vp, vp, vp, vp, vp, i64, vp, vp]
     lib.oracle_forward.argtypes = [i64] * 9 + [i32, dbl] + [vp] * 6 + [i64, vp, vp, vp, vp]
     lib.oracle_block_mass.argtypes = [i64] * 8 + [i32, dbl, vp, vp, vp, vp, vp, i64, vp]
+    lib.oracle_forward_paged.argtypes = [i64] * 9 + [i32, dbl, vp, vp, i64, i64, i64] + [vp] * 8
+    lib.oracle_select_hierarchical.argtypes = [i64] * 8 + [i32, vp, vp, vp, i64, vp]
     for f in (lib.oracle_block_scores, lib.oracle_select_blocks, lib.oracle_attention,
-              lib.oracle_forward, lib.oracle_block_mass, lib.oracle_num_threads):
+              lib.oracle_forward, lib.oracle_block_mass, lib.oracle_forward_paged,
+              lib.oracle_select_hierarchical, lib.oracle_num_threads):
         f.restype = ctypes.c_int
     return lib
 
@@ -202,3 +205,54 @@ def forward(q_idx_rows, k_idx, Q_rows, K, V, rows, *, T: int, block: int, topk: 
     if rc != 0:
         raise ValueError(f"oracle_forward failed ({rc})")
     return (ids, O, lse, bs) if want_scores else (ids, O, lse)
+
+
+def forward_paged(q_idx, k_idx_cache, Q, K_cache, V_cache, seq_lens, block_table, *, S: int,
+                  block: int, topk: int, scale: float = 0.0, lib=None):
+    """Forward pass over a paged cache with per-sequence lengths:
+    (ids [B, T, G, topk], O [B, T, Hq, d], lse [B, T, Hq]).
+
+    q_idx [B, T, G, d_idx]; k_idx_cache [num_pages, page_size, d_idx];
+    Q [B, T, Hq, d]; K_cache, V_cache [num_pages, page_size, Hkv, d];
+    seq_lens [B] and block_table [B, max_pages] int32 (host); S the capacity."""
+    qi, dt = _as_raw(q_idx)
+    ki, _ = _as_raw(k_idx_cache)
+    q, _ = _as_raw(Q)
+    k, _ = _as_raw(K_cache)
+    v, _ = _as_raw(V_cache)
+    lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32).reshape(-1))
+    table = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    B, T, Hq, d = q.shape
+    num_pages, page_size, Hkv, _ = k.shape
+    d_idx = qi.shape[-1]
+    max_pages = table.shape[1]
+    ids = np.empty((B, T, Hkv, topk), np.int32)
+    O = np.empty((B, T, Hq, d), np.float64)
+    lse = np.empty((B, T, Hq), np.float64)
+    rc = (lib or _load()).oracle_forward_paged(
+        B, T, S, Hq, Hkv, d, d_idx, block, topk, dt, float(scale), _ptr(lens), _ptr(table),
+        page_size, max_pages, num_pages, _ptr(qi), _ptr(ki), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(ids), _ptr(O), _ptr(lse))
+    if rc != 0:
+        raise ValueError(f"oracle_forward_paged failed ({rc})")
+    return ids, O, lse
+
+
+def select_hierarchical(q_idx_rows, k_idx, rows, *, T: int, block: int, topk: int, kc: int,
+                        lib=None) -> np.ndarray:
+    """Coarse-to-fine block selection: ids [nrows, G, topk] int32 (ascending,
+    -1 padded).  Coarse: index query . the block's mean index key; the kc - 1
+    best earlier blocks are the candidates; fine: their exact max-pooled
+    scores; kept: the current block and the topk - 1 best candidates."""
+    q, dt = _as_raw(q_idx_rows)
+    k, dt2 = _as_raw(k_idx)
+    assert dt == dt2, "q_idx and k_idx must share a dtype"
+    r = _rows(rows)
+    nrows, G, d_idx = q.shape
+    B, S, _ = k.shape
+    ids = np.empty((nrows, G, topk), np.int32)
+    rc = (lib or _load()).oracle_select_hierarchical(B, T, S, G, d_idx, block, topk, kc, dt,
+                                                     _ptr(q), _ptr(k), _ptr(r), nrows, _ptr(ids))
+    if rc != 0:
+        raise ValueError(f"oracle_select_hierarchical failed ({rc})")
+    return ids

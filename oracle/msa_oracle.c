@@ -397,6 +397,165 @@ int oracle_forward(int64_t B, int64_t T, int64_t S, int64_t Hq, int64_t Hkv,
     return rc;
 }
 
+/*
+ * Hierarchical (coarse-to-fine) block selection, an index-cost reducer
+ * ("LongCat Sparse Attention", Abstract, item (3): a coarse-to-fine scoring
+ * scheme narrows the candidate set of each query, cutting the indexing
+ * work).  The page names no formula; the reading taken here, for MSA's
+ * max-pooled block scores, in three steps per (row, group):
+ *   1. coarse: block n < cb is scored by the dot product of the index query
+ *      with the block's MEAN index key, (1 / block) * sum over the block's
+ *      tokens of k_idx[j] -- d_idx multiply-adds per block instead of
+ *      block * d_idx;
+ *   2. candidates: the kc - 1 best blocks n < cb by coarse score (larger
+ *      score first, lower id on ties);
+ *   3. fine: each candidate's exact block score (the max-pooled token dot
+ *      product of oracle_block_scores); kept = {cb} plus the topk - 1 best
+ *      candidates by fine score (same order), written ascending, -1 padded.
+ * Candidates are whole blocks before the current one, so every token of a
+ * candidate is causal.  With kc - 1 >= cb every earlier block is a
+ * candidate and the result is oracle_select_blocks' on the exact scores.
+ * Requires 1 <= topk <= kc.  ids [nrows, G, topk].
+ */
+int oracle_select_hierarchical(int64_t B, int64_t T, int64_t S, int64_t G,
+                               int64_t d_idx, int64_t block, int64_t topk, int64_t kc,
+                               int dtype, const void *q_idx_rows, const void *k_idx,
+                               const int64_t *rows, int64_t nrows, int32_t *ids)
+{
+    if (B <= 0 || T <= 0 || S <= 0 || T > S || G <= 0 || d_idx <= 0 || block <= 0 ||
+        topk <= 0 || kc < topk || nrows < 0 || (dtype != ORACLE_F32 && dtype != ORACLE_BF16))
+        return -1;
+    const int64_t NB = ceil_div(S, block);
+    int bad = 0;
+#pragma omp parallel
+    {
+        cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * (size_t)NB);
+        double *mean = (double *)malloc(sizeof(double) * (size_t)d_idx);
+        if (!cand || !mean) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t ri = 0; ri < nrows; ++ri) {
+            if (!cand || !mean) continue;
+            const int64_t r = rows[ri];
+            if (r < 0 || r >= B * T) { bad = 1; continue; }
+            const int64_t b = r / T, t = r % T;
+            const int64_t cb = query_pos(T, S, t) / block;
+            for (int64_t g = 0; g < G; ++g) {
+                const int64_t q0 = (ri * G + g) * d_idx;
+                int32_t *out = ids + (ri * G + g) * topk;
+                /* 1. coarse scores of the blocks before the current one */
+                for (int64_t n = 0; n < cb; ++n) {
+                    for (int64_t ii = 0; ii < d_idx; ++ii) {
+                        double sum = 0.0;
+                        for (int64_t j = n * block; j < (n + 1) * block; ++j)
+                            sum += widen(k_idx, dtype, (b * S + j) * d_idx + ii);
+                        mean[ii] = sum / (double)block;
+                    }
+                    double dot = 0.0;
+                    for (int64_t ii = 0; ii < d_idx; ++ii)
+                        dot += widen(q_idx_rows, dtype, q0 + ii) * mean[ii];
+                    cand[n].score = dot;
+                    cand[n].id = n;
+                }
+                /* 2. the kc - 1 best by coarse score */
+                qsort(cand, (size_t)cb, sizeof *cand, cand_better_first);
+                const int64_t nc = (cb < kc - 1) ? cb : kc - 1;
+                /* 3. exact max-pooled scores of the candidates, then the topk - 1 best */
+                for (int64_t c = 0; c < nc; ++c) {
+                    const int64_t n = cand[c].id;
+                    double best = -INFINITY;
+                    for (int64_t j = n * block; j < (n + 1) * block; ++j) {
+                        double dot = 0.0;
+                        for (int64_t ii = 0; ii < d_idx; ++ii)
+                            dot += widen(q_idx_rows, dtype, q0 + ii) *
+                                   widen(k_idx, dtype, (b * S + j) * d_idx + ii);
+                        best = dot > best ? dot : best;
+                    }
+                    cand[c].score = best;
+                }
+                qsort(cand, (size_t)nc, sizeof *cand, cand_better_first);
+                const int64_t take = (nc < topk - 1) ? nc : topk - 1;
+                for (int64_t i = 0; i < take; ++i) out[i] = (int32_t)cand[i].id;
+                qsort(out, (size_t)take, sizeof(int32_t), id_ascending);
+                out[take] = (int32_t)cb;
+                for (int64_t slot = take + 1; slot < topk; ++slot) out[slot] = -1;
+            }
+        }
+        free(cand);
+        free(mean);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * The forward pass over a PAGED cache with per-sequence lengths (decode
+ * steps of a serving batch).  The pages do not describe paging: this is the
+ * same method ("MiniMax Sparse Attention", Summary, second paragraph) with
+ * each sequence's keys read through a block table.
+ *
+ * Sequence b has L = seq_lens[b] keys; its key j < L is row j % page_size of
+ * page block_table[b * max_pages + j / page_size] of each cache:
+ *   k_idx_cache [num_pages, page_size, d_idx]
+ *   K_cache, V_cache [num_pages, page_size, Hkv, d]
+ * Its T queries (q_idx [B, T, Hkv, d_idx], Q [B, T, Hq, d]) sit at the last
+ * T positions L - T + t.  Each sequence is the dense problem with S = L:
+ * its keys are copied out of the pages in order, and oracle_forward runs on
+ * them (a partial last block is allowed there).  Outputs:
+ *   ids [B, T, Hkv, topk] int32, O [B, T, Hq, d], lse [B, T, Hq] (double).
+ * A length outside [T, S] or a page id outside [0, num_pages) is an error
+ * (-4); nothing is computed for any sequence then.
+ */
+int oracle_forward_paged(int64_t B, int64_t T, int64_t S, int64_t Hq, int64_t Hkv,
+                         int64_t d, int64_t d_idx, int64_t block, int64_t topk,
+                         int dtype, double scale, const int32_t *seq_lens,
+                         const int32_t *block_table, int64_t page_size,
+                         int64_t max_pages, int64_t num_pages, const void *q_idx,
+                         const void *k_idx_cache, const void *Q, const void *K_cache,
+                         const void *V_cache, int32_t *ids, double *O, double *lse)
+{
+    if (B <= 0 || T <= 0 || S <= 0 || page_size <= 0 || max_pages <= 0 ||
+        num_pages <= 0 || max_pages * page_size < S ||
+        (dtype != ORACLE_F32 && dtype != ORACLE_BF16))
+        return -1;
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t L = seq_lens[b];
+        if (L < T || L > S) return -4;
+        for (int64_t i = 0; i < (L + page_size - 1) / page_size; ++i) {
+            const int64_t pg = block_table[b * max_pages + i];
+            if (pg < 0 || pg >= num_pages) return -4;
+        }
+    }
+    const size_t esz = dtype == ORACLE_BF16 ? 2 : 4;
+    const size_t ki_row = (size_t)d_idx * esz, kv_row = (size_t)Hkv * d * esz;
+    char *ki = (char *)malloc(ki_row * (size_t)S);
+    char *kk = (char *)malloc(kv_row * (size_t)S);
+    char *vv = (char *)malloc(kv_row * (size_t)S);
+    int64_t *rows = (int64_t *)malloc(sizeof(int64_t) * (size_t)T);
+    int rc = (ki && kk && vv && rows) ? 0 : -2;
+    for (int64_t t = 0; t < T && rc == 0; ++t) rows[t] = t;
+    for (int64_t b = 0; b < B && rc == 0; ++b) {
+        const int64_t L = seq_lens[b];
+        /* the sequence's keys, densely: row j of page table entry j / page_size */
+        for (int64_t j = 0; j < L; ++j) {
+            const int64_t pg = block_table[b * max_pages + j / page_size];
+            const int64_t src = pg * page_size + j % page_size;
+            memcpy(ki + (size_t)j * ki_row, (const char *)k_idx_cache + (size_t)src * ki_row,
+                   ki_row);
+            memcpy(kk + (size_t)j * kv_row, (const char *)K_cache + (size_t)src * kv_row, kv_row);
+            memcpy(vv + (size_t)j * kv_row, (const char *)V_cache + (size_t)src * kv_row, kv_row);
+        }
+        rc = oracle_forward(1, T, L, Hq, Hkv, d, d_idx, block, topk, dtype, scale,
+                            (const char *)q_idx + (size_t)(b * T * Hkv * d_idx) * esz, ki,
+                            (const char *)Q + (size_t)(b * T * Hq * d) * esz, kk, vv, rows, T,
+                            ids + b * T * Hkv * topk, O + b * T * Hq * d, lse + b * T * Hq,
+                            NULL);
+    }
+    free(ki);
+    free(kk);
+    free(vv);
+    free(rows);
+    return rc;
+}
+
 /* Number of OpenMP threads the oracle runs with (for reporting). */
 int oracle_num_threads(void)
 {

@@ -360,5 +360,129 @@ def pin_block_mass(lib):
         np.testing.assert_allclose(mass[..., i], want, rtol=1e-12, atol=1e-15)
 
 
+def make_paged(rng, dense_rows_list, page_size, spare_pages=3):
+    """Scatter each sequence's rows (a list of [L_b, ...] arrays) over pages
+    in a random order.  Returns (cache [num_pages, page_size, ...],
+    block_table [B, max_pages]); unused table entries hold a valid page id."""
+    B = len(dense_rows_list)
+    n_pages = [-(-len(x) // page_size) for x in dense_rows_list]
+    max_pages = max(n_pages) + 1
+    num_pages = sum(n_pages) + spare_pages
+    order = rng.permutation(num_pages)
+    tail = dense_rows_list[0].shape[1:]
+    cache = rng.standard_normal((num_pages, page_size) + tail).astype(np.float32)
+    table = np.zeros((B, max_pages), dtype=np.int32)
+    k = 0
+    for b, x in enumerate(dense_rows_list):
+        for i in range(n_pages[b]):
+            pg = int(order[k])
+            k += 1
+            table[b, i] = pg
+            rows = x[i * page_size:(i + 1) * page_size]
+            cache[pg, :len(rows)] = rows
+    return cache, table
+
+
+def pin_paged_addressing(lib):
+    """The paged forward equals, sequence by sequence, the method on that
+    sequence's keys laid out densely, computed without the oracle: block
+    scores from the full score matrix, kept sets by counting, attention by
+    SDPA with the kept-block mask.  Lengths not a multiple of the block,
+    pages scattered in random order, page sizes below and above the block."""
+    rng = np.random.default_rng(23)
+    T, Hq, Hkv, d, d_idx, block, k, S = 2, 4, 2, 16, 8, 16, 4, 160
+    for page_size, lens in [(8, [160, 123, 40]), (24, [97, 160, 2])]:
+        B = len(lens)
+        q_idx = _grid(rng, (B, T, Hkv, d_idx))
+        Q = rng.standard_normal((B, T, Hq, d)).astype(np.float32)
+        kd = [_grid(rng, (L, d_idx)) for L in lens]
+        Kd = [rng.standard_normal((L, Hkv, d)).astype(np.float32) for L in lens]
+        Vd = [rng.standard_normal((L, Hkv, d)).astype(np.float32) for L in lens]
+        kc, table = make_paged(rng, kd, page_size)
+        # one table for all three caches: K and V on the index keys' pages
+        Kc = np.zeros((kc.shape[0], page_size, Hkv, d), np.float32)
+        Vc = np.zeros((kc.shape[0], page_size, Hkv, d), np.float32)
+        for b, L in enumerate(lens):
+            for j in range(L):
+                pg, off = table[b, j // page_size], j % page_size
+                Kc[pg, off], Vc[pg, off] = Kd[b][j], Vd[b][j]
+        ids, O, lse = orc.forward_paged(q_idx, kc, Q, Kc, Vc, np.array(lens), table, S=S,
+                                        block=block, topk=k, lib=lib)
+        for b, L in enumerate(lens):
+            bs = brute_block_scores(q_idx[b:b + 1], kd[b][None], T, block)[0]     # [T, G, NB]
+            for t in range(T):
+                cb = (L - T + t) // block
+                for g in range(Hkv):
+                    want = sorted(brute_kept_sets(bs[t, g], cb, k))
+                    got = [int(x) for x in ids[b, t, g] if x >= 0]
+                    assert got == want, (page_size, b, t, g, got, want)
+                    assert all(x == -1 for x in ids[b, t, g, len(want):])
+            allowed = _allowed_from_ids(ids[b].reshape(T, Hkv, k), 1, T, L, Hq, Hkv, block)
+            O_ref, lse_ref = _sdpa_reference(Q[b:b + 1], Kd[b][None], Vd[b][None], allowed,
+                                             1.0 / np.sqrt(d))
+            np.testing.assert_allclose(O[b], O_ref[0], rtol=0, atol=1e-10)
+            np.testing.assert_allclose(lse[b], lse_ref[0], rtol=0, atol=1e-10)
+
+
+def brute_hierarchical(q_idx, k_idx, T, block, k, kc):
+    """Coarse-to-fine kept sets [B, T, G] of python sets, by numpy and by
+    counting: block means by reshape, coarse scores by matmul, candidates
+    = earlier blocks with fewer than kc - 1 better coarse scores, kept = the
+    current block and the candidates with fewer than k - 1 better fine
+    (exact max-pooled) scores among the candidates."""
+    B, _, G, d_idx = q_idx.shape
+    S = k_idx.shape[1]
+    NB = S // block
+    mean = k_idx.astype(np.float64).reshape(B, NB, block, d_idx).mean(axis=2)   # [B, NB, d]
+    coarse = np.einsum("btgi,bni->btgn", q_idx.astype(np.float64), mean)
+    fine = brute_block_scores(q_idx, k_idx, T, block)
+    out = np.empty((B, T, G), dtype=object)
+    for b in range(B):
+        for t in range(T):
+            cb = (S - T + t) // block
+            for g in range(G):
+                c = coarse[b, t, g]
+                cands = [n for n in range(cb)
+                         if sum(1 for m in range(cb)
+                                if c[m] > c[n] or (c[m] == c[n] and m < n)) < kc - 1]
+                f = fine[b, t, g]
+                kept = {n for n in cands
+                        if sum(1 for m in cands
+                               if f[m] > f[n] or (f[m] == f[n] and m < n)) < k - 1}
+                out[b, t, g] = kept | {cb}
+    return out
+
+
+def pin_hierarchical_selection(lib):
+    """The coarse-to-fine selection equals the brute-force count on tiny
+    inputs (several candidate counts), and with every earlier block a
+    candidate it is the exact selection."""
+    rng = np.random.default_rng(29)
+    for B, T, S, G, d_idx, block, k, kcs in [(1, 40, 160, 2, 8, 8, 3, (3, 5, 9)),
+                                            (2, 24, 96, 1, 4, 16, 2, (2, 4))]:
+        q_idx = _grid(rng, (B, T, G, d_idx))
+        k_idx = _grid(rng, (B, S, d_idx))
+        rows = _rows_all(B, T)
+        NB = S // block
+        for kc in kcs + (NB + 1,):
+            ids = orc.select_hierarchical(q_idx.reshape(B * T, G, d_idx), k_idx, rows, T=T,
+                                          block=block, topk=k, kc=kc, lib=lib)
+            want = brute_hierarchical(q_idx, k_idx, T, block, k, kc)
+            for r in range(B * T):
+                for g in range(G):
+                    got = ids[r, g]
+                    kept = sorted(want[r // T, r % T, g])
+                    assert list(got[:len(kept)]) == kept, (kc, r, g, got, kept)
+                    assert all(x == -1 for x in got[len(kept):])
+        # every earlier block a candidate: the exact selection
+        exact = orc.select_blocks(orc.block_scores(q_idx.reshape(B * T, G, d_idx), k_idx, rows,
+                                                   T=T, block=block, lib=lib),
+                                  rows, T=T, S=S, block=block, topk=k, lib=lib)
+        full = orc.select_hierarchical(q_idx.reshape(B * T, G, d_idx), k_idx, rows, T=T,
+                                       block=block, topk=k, kc=NB, lib=lib)
+        assert np.array_equal(full, exact)
+
+
 ALL_PINS = [pin_brute_force_selection, pin_dense_limit, pin_masked_attention,
-            pin_closed_forms, pin_permutation_invariance, pin_bf16_widening, pin_block_mass]
+            pin_closed_forms, pin_permutation_invariance, pin_bf16_widening, pin_block_mass,
+            pin_paged_addressing, pin_hierarchical_selection]

@@ -21,7 +21,7 @@ def test_header_declares_the_calls():
     for want in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd", "msa_forward",
                  "msa_workspace_size", "msa_status_string", "msa_get_device_error",
                  "msa_kernel_launches", "msa_selftest_wait_timeout", "msa_forward_host",
-                 "msa_sparse_attn_fwd_mass", "msa_forward_mass"):
+                 "msa_sparse_attn_fwd_mass", "msa_forward_mass", "msa_decode_paged"):
         assert want in names
 
 
@@ -148,3 +148,34 @@ def test_missing_library_fails_loudly(tmp_path):
                        cwd=str(tmp_path), capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "ImportError" in r.stderr and "libmsa.so" in r.stderr
+
+
+def test_decode_paged_rejected_on_host():
+    """msa_decode_paged validates its page arguments, shapes and workspace on
+    the host before anything is enqueued (no pointer is dereferenced)."""
+    import torch
+    from block_sparse_long_03_b200 import binding
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x20000)
+
+    def call(p, page_size=64, max_pages=64, num_pages=100, ws_bytes=1 << 30, lens=fake):
+        return lib.msa_decode_paged(ctypes.byref(p), lens, fake, page_size, max_pages, num_pages,
+                                    fake, fake, fake, fake, fake, None, fake, fake, ws, ws_bytes,
+                                    None)
+
+    p = _p(B=4, T=1, S=4096, Hq=32, Hkv=8, block=64, topk=8)
+    need = binding.msa_workspace_size(p, binding.MSA_WS_DECODE_PAGED)
+    assert need > 256
+    assert call(p, page_size=0) == 1
+    assert call(p, page_size=64, max_pages=63) == 1          # 63 * 64 < S
+    assert call(p, num_pages=0) == 1
+    assert call(p, lens=None) == 1
+    assert call(p, lens=ctypes.c_void_p(0x10004)) == 1       # misaligned
+    assert call(p, ws_bytes=need - 1) == 5
+    p32 = _p(B=4, T=1, S=4096, Hq=32, Hkv=8, block=64, topk=8, dtype=torch.float32)
+    assert call(p32) == 2
+    assert binding.msa_workspace_size(p32, binding.MSA_WS_DECODE_PAGED) == 0
+    wide = _p(B=4, T=8, S=4096, Hq=32, Hkv=8, block=64, topk=8)   # T * G = 64 > 32
+    assert call(wide) == 2
+    assert call(_p(T=0)) == 1

@@ -160,3 +160,23 @@ def test_non_causal_caller_ids_counted(name):
     assert msa.msa_get_device_error(ws2) == 6
     assert msa.msa_get_device_error(ws3) == 0
     assert torch.equal(lse2, lse3) and torch.equal(O2, O3)
+
+
+@pytest.mark.parametrize("NB,k,ties", [(4100, 17, False), (4099, 100, False), (2052, 33, True),
+                                       (8192, 65, False), (3000, 66, True)])
+def test_topk_long_rows(NB, k, ties):
+    """Rows of more than 2048 blocks (the streaming warp kernel): threshold
+    path (k - 1 <= 64), radix path (k - 1 > 64 or heavy ties), 16-byte and
+    scalar row loads (NB % 4), against the oracle's selection."""
+    msa = _msa()
+    block, T, G = 64, 6, 2
+    S = NB * block
+    g = torch.Generator().manual_seed(NB + k)
+    if ties:
+        bs = (torch.randint(-2, 3, (1, T, G, NB), generator=g) * 0.5).float()
+    else:
+        bs = torch.randn((1, T, G, NB), generator=g).float()
+    ids = msa.topk_blocks(bs.cuda(), S=S, block=block, topk=k).cpu().numpy()
+    rows = np.arange(T)
+    ref = orc.select_blocks(bs[0].numpy().astype(np.float64), rows, T=T, S=S, block=block, topk=k)
+    parity.assert_ids_equal(ids[0], ref, f"long rows NB={NB} k={k}")

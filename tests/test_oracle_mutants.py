@@ -40,6 +40,16 @@ MUTANTS = {
                         "if (j > S) break;"),
     "mass_wrong_head_of_group": ("const int64_t h = g * R + hh;", "const int64_t h = hh * Hkv + g;"),
     "mass_unscaled_scores": ("head_sum += exp(scale * dot - l);", "head_sum += exp(dot - l);"),
+    "hier_one_candidate_too_few": ("const int64_t nc = (cb < kc - 1) ? cb : kc - 1;",
+                                   "const int64_t nc = (cb < kc - 2) ? cb : kc - 2;"),
+    "hier_coarse_drops_a_term": ("dot += widen(q_idx_rows, dtype, q0 + ii) * mean[ii];",
+                                 "dot += (ii == 0) ? 0.0 : widen(q_idx_rows, dtype, q0 + ii) * mean[ii];"),
+    "hier_no_fine_rescoring": ("                    cand[c].score = best;\n",
+                               "                    (void)best;\n"),
+    "paged_offset_in_page": ("const int64_t src = pg * page_size + j % page_size;",
+                             "const int64_t src = pg * page_size + (j + 1) % page_size;"),
+    "paged_wrong_table_entry": ("block_table[b * max_pages + j / page_size];\n",
+                                "block_table[b * max_pages + (j / page_size + 1) % max_pages];\n"),
 }
 # "current_block_not_forced" needs a two-part edit: candidates include cb and
 # the forced append is dropped.
