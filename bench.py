@@ -84,10 +84,10 @@ def partial_floor_bytes(w) -> float:
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the sparse
 # attention call's two main kernels, from a one-pass ncu capture of ONE row
-# chunk (the last, 8037 rows, every row keeping k blocks) of the workload
-# `prefill_32k_h64` (the 128K prefill's heads, group size and k at 32K tokens:
-# each chunk is one of the same 8065-row passes the 128K call makes, and Q is
-# larger than L2 as there):
+# chunk (the fourth of five: rows 24195..32259, 8065 rows like every full
+# chunk of the 128K call, every row keeping k blocks) of the workload
+# `prefill_32k_h64` (the 128K prefill's heads, group size and k at 32K tokens;
+# Q is larger than L2 as there):
 #   python bench.py --workload prefill_32k_h64 --attn-call-once
 # under ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
 # dram__bytes_write.sum -k regex:"attn_tc_kernel|combine_kernel" -s 6 -c 2.
@@ -323,6 +323,38 @@ class Problem:
         torch.cuda.empty_cache()
 
 
+def index_reducers(prob, args, ws: int, kc: int) -> dict:
+    """The index branch's cost at this shape, exact (msa_forward minus its
+    attention call, which takes the same ids) against coarse-to-fine
+    selection with kc candidates (msa_index_hierarchical), and the recall of
+    the latter: the share of the exact selection's non-forced ids it keeps,
+    over sampled rows."""
+    m, i, w = prob.msa, prob.inp, prob.w
+    steps = max(2, min(args.steps, 3))
+    fwd_ms = time_steps(prob.step, steps, args.warmup, ws)
+    attn_ms = time_steps(lambda: m.msa_sparse_attn_fwd(prob.params, i.Q, i.K, i.V, prob.ids,
+                                                       prob.O, prob.lse, prob.ws_attn),
+                         steps, args.warmup, ws)
+    hids = torch.empty_like(prob.ids)
+    hws = m.alloc_workspace(prob.params, m.MSA_WS_INDEX_HIER)
+    hier_ms = time_steps(lambda: m.msa_index_hierarchical(prob.params, kc, i.q_idx, i.k_idx,
+                                                          hids, hws),
+                         steps, args.warmup, ws)
+    prob.step()                                   # the exact ids of these inputs
+    torch.cuda.synchronize()
+    g = torch.Generator(device="cuda").manual_seed(3)
+    rows = torch.randint(w.block * w.topk, w.T, (4096,), generator=g, device="cuda")
+    ex = prob.ids[0, rows].long()                 # [n, G, k]; slot k - 1 is the current block
+    hi = hids[0, rows].long()
+    hit = (ex[..., :-1, None] == hi[..., None, :-1]).any(-1).float().mean().item()
+    del hws
+    return {"workload": w.name, "kc": kc, "exact_index_topk_ms": fwd_ms - attn_ms,
+            "hierarchical_ms": hier_ms, "attention_ms": attn_ms, "forward_ms": fwd_ms,
+            "speedup": (fwd_ms - attn_ms) / hier_ms,
+            "recall_of_exact_ids": hit,
+            "recall_rows": "4096 sampled rows with every slot filled (t >= block * k)"}
+
+
 def time_steps(fn, steps: int, warmup: int, ws: int):
     for _ in range(warmup):
         fn()
@@ -532,6 +564,7 @@ def run_ours(args, rank: int, ws: int):
             "tokens_per_s": aggregate_tokens_per_s(p1.w.B * p1.w.T, ms1, ws),
             "ms_per_step": ms1, "attention_flops": attention_flops(p1.w),
             "index_flops": index_flops(p1.w), "clocks": c1.summary()}
+        long_ctx["index_reducers"] = index_reducers(p1, args, ws, kc=64)
         p1.free()
         del p1
         d1 = Problem("decode_1m", seed=rank_seed(rank) + 3)

@@ -18,6 +18,7 @@ if not _os.path.exists(_LIB):
 
 __all__ = [
     "EXPORTS", "MSA_BF16", "MSA_F32", "MSA_OK", "MSA_WS_DECODE_PAGED", "MSA_WS_FORWARD",
+    "MSA_WS_INDEX_HIER", "index_hierarchical", "msa_index_hierarchical",
     "MSA_WS_FORWARD_HOST", "MSA_WS_SPARSE_ATTN", "MsaError", "Params", "alloc_workspace",
     "decode_paged", "forward", "msa_decode_paged",
     "forward_with_mass", "index_block_scores", "make_params", "msa_forward", "msa_forward_host",

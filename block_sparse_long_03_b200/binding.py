@@ -14,11 +14,14 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmsa.so")
+# MSA_LIBRARY=checked selects the bounds-checked build (libmsa_checked.so)
+LIB_PATH = os.path.join(_HERE, "libmsa_checked.so" if os.environ.get("MSA_LIBRARY") == "checked"
+                        else "libmsa.so")
 
 MSA_OK = 0
 MSA_F32, MSA_BF16 = 0, 1
 MSA_WS_SPARSE_ATTN, MSA_WS_FORWARD, MSA_WS_FORWARD_HOST, MSA_WS_DECODE_PAGED = 0, 1, 2, 3
+MSA_WS_INDEX_HIER = 4
 STATUS_NAMES = {0: "MSA_OK", 1: "MSA_ERR_INVALID_ARG", 2: "MSA_ERR_UNSUPPORTED", 3: "MSA_ERR_CUDA",
                 4: "MSA_ERR_DEVICE_TIMEOUT", 5: "MSA_ERR_WORKSPACE", 6: "MSA_ERR_BAD_BLOCK_IDS",
                 7: "MSA_ERR_BAD_PAGE_TABLE"}
@@ -28,7 +31,8 @@ EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_workspace_size", "msa_sparse_attn_fwd", "msa_forward", "msa_get_device_error",
            "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
            "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass",
-           "msa_query_pieces", "msa_decode_paged")
+           "msa_query_pieces", "msa_decode_paged", "msa_index_hierarchical",
+           "msa_bounds_failures")
 
 
 class MsaError(RuntimeError):
@@ -71,12 +75,16 @@ def _load():
     i32 = ctypes.c_int32
     lib.msa_decode_paged.argtypes = [P, vp, vp, i32, i32, i32] + [vp] * 8 + [vp, sz, vp]
     lib.msa_decode_paged.restype = st
+    lib.msa_index_hierarchical.argtypes = [P, i32, vp, vp, vp, vp, sz, vp]
+    lib.msa_index_hierarchical.restype = st
     lib.msa_query_pieces.argtypes = [P, ctypes.c_int, vp, ctypes.c_int64]
     lib.msa_query_pieces.restype = ctypes.c_int64
     lib.msa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.msa_selftest_wait_timeout.restype = st
     lib.msa_kernel_launches.argtypes = []
     lib.msa_kernel_launches.restype = ctypes.c_uint64
+    lib.msa_bounds_failures.argtypes = []
+    lib.msa_bounds_failures.restype = ctypes.c_uint32
     for name in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd",
                  "msa_forward", "msa_get_device_error"):
         getattr(lib, name).restype = st
@@ -199,6 +207,15 @@ def msa_decode_paged(params: Params, seq_lens, block_table, page_size: int, num_
            "msa_decode_paged")
 
 
+def msa_index_hierarchical(params: Params, kc: int, q_idx, k_idx, block_ids, workspace,
+                           stream=None):
+    """Coarse-to-fine block selection (block means, kc candidates, exact
+    rescoring) into block_ids [B, T, G, topk]."""
+    _check(lib.msa_index_hierarchical(ctypes.byref(params), int(kc), _ptr(q_idx), _ptr(k_idx),
+                                      _ptr(block_ids), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)), "msa_index_hierarchical")
+
+
 def msa_get_device_error(workspace, stream=None) -> int:
     """The status recorded on the device by the last call that used `workspace`."""
     return int(lib.msa_get_device_error(_ptr(workspace), _stream(stream)))
@@ -299,3 +316,15 @@ def decode_paged(q_idx, k_idx_cache, Q, K_cache, V_cache, seq_lens, block_table,
     msa_decode_paged(p, seq_lens, block_table, page_size, num_pages, q_idx, k_idx_cache, Q,
                      K_cache, V_cache, ids, O, lse, ws)
     return O, lse, ids, ws
+
+
+def index_hierarchical(q_idx, k_idx, *, block: int, topk: int, kc: int):
+    """Coarse-to-fine block selection; returns (block_ids, workspace)."""
+    B, T, G, d_idx = q_idx.shape
+    S = k_idx.shape[1]
+    p = make_params(B=B, T=T, S=S, Hq=G, Hkv=G, d=64, d_idx=d_idx, block=block, topk=topk,
+                    dtype=q_idx.dtype)
+    ids = torch.empty((B, T, G, topk), dtype=torch.int32, device=q_idx.device)
+    ws = alloc_workspace(p, MSA_WS_INDEX_HIER, q_idx.device)
+    msa_index_hierarchical(p, kc, q_idx, k_idx, ids, ws)
+    return ids, ws

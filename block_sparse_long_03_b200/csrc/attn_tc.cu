@@ -35,8 +35,9 @@ constexpr int kThreads = 512;        // four warpgroups: loads + MMA, two softma
 constexpr int kRun = 8;              // consecutive tiles per CTA turn (K/V reuse)
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Validity of the kept slots lane and lane + 32 of a row (topk <= 64),
-// computed by one warp: in range, holding a causal token, and not a repeat
+// Validity of the kept slots lane and lane + 32 of a row (topk <= 64; the
+// hot merge path, which keeps these few values in registers), computed by
+// one warp: in range, holding a causal token, and not a repeat
 // (a strictly ascending row, the form msa_topk_blocks writes, cannot repeat;
 // otherwise earlier slots are scanned).  bad = an id >= NB, an id above cb
 // (a block with no causal token) or a repeat; bad slots are skipped and
@@ -45,7 +46,7 @@ struct SlotPair {
     int id0, id1;
     bool ok0, ok1, bad0, bad1;
 };
-__device__ __forceinline__ SlotPair warp_slots(const int32_t *row, int topk, int NB, int cb,
+__device__ __forceinline__ SlotPair warp_slots2(const int32_t *row, int topk, int NB, int cb,
                                                int lane) {
     SlotPair r;
     r.id0 = lane < topk ? row[lane] : -1;
@@ -78,10 +79,64 @@ __device__ __forceinline__ SlotPair warp_slots(const int32_t *row, int topk, int
     return r;
 }
 
+// The same for the kept slots lane + 32 k (k < kPer, topk <= 32 kPer) of a
+// row, computed by one warp: in range, holding a causal token, and not a
+// repeat (a strictly ascending row, the form msa_topk_blocks writes, cannot
+// repeat; otherwise earlier slots are scanned).  bad = an id >= NB, an id
+// above cb (a block with no causal token) or a repeat; bad slots are skipped
+// and counted in the error word.  okmask[k] bit l: slot 32 k + l is valid.
+template <int kPer>
+struct SlotSet {
+    int id[kPer];
+    bool ok[kPer], bad[kPer];
+    uint32_t okmask[kPer];
+    __device__ __forceinline__ bool valid(int sl) const {      // slot sl of the row
+        uint32_t m = 0;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k)
+            if (k == (sl >> 5)) m = okmask[k];
+        return (m >> (sl & 31)) & 1u;
+    }
+};
+template <int kPer>
+__device__ __forceinline__ SlotSet<kPer> warp_slots(const int32_t *row, int topk, int NB, int cb,
+                                                    int lane) {
+    SlotSet<kPer> r;
+    int carry = -1;                               // largest id of the earlier 32-slot groups
+    bool dis = false;                             // some slot not above every earlier one
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int id = 32 * k + lane < topk ? row[32 * k + lane] : -1;
+        r.id[k] = id;
+        int pm = id;                              // inclusive prefix max over the lanes
+        for (int off = 1; off < 32; off *= 2) {
+            const int o = __shfl_up_sync(0xffffffffu, pm, off);
+            if (lane >= off) pm = max(pm, o);
+        }
+        const int up = __shfl_up_sync(0xffffffffu, pm, 1);
+        const int before = lane > 0 ? max(carry, up) : carry;
+        dis |= id >= 0 && (32 * k + lane > 0) && id <= before;
+        carry = max(carry, __shfl_sync(0xffffffffu, pm, 31));
+    }
+    const bool asc = !__any_sync(0xffffffffu, dis);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int id = r.id[k];
+        bool rep = false;
+        if (!asc)
+            for (int q = 0; q < 32 * k + lane && id >= 0; ++q) rep |= row[q] == id;
+        r.bad[k] = id >= NB || id > cb || (id >= 0 && rep);
+        r.ok[k] = id >= 0 && !r.bad[k];
+        r.okmask[k] = __ballot_sync(0xffffffffu, r.ok[k]);
+    }
+    return r;
+}
+
 // ---------------------------------------------------------------- CSR build
 
 // counts[(b*G + g)*NB + n] += 1 for every valid kept slot of the chunk's rows;
 // one warp per (row, group), one lane per slot.
+template <int kPer>
 __global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restrict__ counts,
                                  uint32_t *err, int64_t r0, int64_t rc, int T_, int S, int G,
                                  int NB, int block, int topk) {
@@ -92,11 +147,15 @@ __global__ void csr_count_kernel(const int32_t *__restrict__ ids, int *__restric
     const int g = (int)(x % G);
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
-    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const SlotSet<kPer> sp = warp_slots<kPer>(ids + (r * G + g) * topk, topk, NB, cb, lane);
     int *base = counts + ((int64_t)b * G + g) * NB;
-    if (sp.ok0) atomicAdd(base + sp.id0, 1);
-    if (sp.ok1) atomicAdd(base + sp.id1, 1);
-    if (sp.bad0 || sp.bad1) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        if (sp.ok[k]) atomicAdd(base + sp.id[k], 1);
+        bad |= sp.bad[k];
+    }
+    if (bad) record_error(err, MSA_ERR_BAD_BLOCK_IDS, 1);
 }
 
 // Single-CTA exclusive scan: tile_offs = scan(ceil(counts / tpt)); tile_offs[L]
@@ -132,10 +191,11 @@ __host__ __device__ constexpr int rec_ints(int tpt) { return 4 + tpt; }
 
 // Every valid kept slot of the chunk's rows into its list's next free record
 // entry; one warp per (row, group), one lane per slot.
+template <int kPer>
 __global__ void csr_fill_kernel(const int32_t *__restrict__ ids,
                                 const int *__restrict__ tile_offs, int *__restrict__ cursor,
                                 int *__restrict__ recs, int64_t r0, int64_t rc, int T_, int S,
-                                int G, int NB, int block, int topk, int tpt) {
+                                int G, int NB, int block, int topk, int tpt, int64_t rec_cap) {
     const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
@@ -143,19 +203,17 @@ __global__ void csr_fill_kernel(const int32_t *__restrict__ ids,
     const int g = (int)(x % G);
     const int b = (int)(r / T_), t = (int)(r % T_);
     const int cb = (int)(((int64_t)S - T_ + t) / block);
-    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const SlotSet<kPer> sp = warp_slots<kPer>(ids + (r * G + g) * topk, topk, NB, cb, lane);
     const int64_t lbase = ((int64_t)b * G + g) * NB;
     const int tag = (int)((r - r0) << 8);
-    if (sp.ok0) {
-        const int64_t list = lbase + sp.id0;
-        const int pos = atomicAdd(&cursor[list], 1);
-        recs[(int64_t)(tile_offs[list] + pos / tpt) * rec_ints(tpt) + 4 + pos % tpt] = tag | lane;
-    }
-    if (sp.ok1) {
-        const int64_t list = lbase + sp.id1;
-        const int pos = atomicAdd(&cursor[list], 1);
-        recs[(int64_t)(tile_offs[list] + pos / tpt) * rec_ints(tpt) + 4 + pos % tpt] =
-            tag | (lane + 32);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        if (sp.ok[k]) {
+            const int64_t list = lbase + sp.id[k];
+            const int pos = atomicAdd(&cursor[list], 1);
+            const int64_t at = (int64_t)(tile_offs[list] + pos / tpt) * rec_ints(tpt) + 4 + pos % tpt;
+            if (MSA_IN_BOUNDS(at, rec_cap)) recs[at] = tag | (32 * k + lane);
+        }
     }
 }
 
@@ -178,6 +236,234 @@ __global__ void csr_tiles_kernel(const int *__restrict__ counts, const int *__re
 namespace msa {
 namespace {
 
+// Phase 2: the LSE-weighted merge of a (query row, group)'s partials over
+// its valid kept slots, for each of the group's R heads: weights
+// exp(lse_i - max lse) give the softmax over the union of the slots' keys.
+// Four warps share a (row, group), each merging a quarter of the d/8 16-byte
+// channel chunks.  Lane l owns head l % R and slots l / R, l / R + 32 / R, ...;
+// with the blocked chunk layout every load of the warp is 512 contiguous
+// bytes, and all loads of a warp are independent (issued together).
+// Needs R | 32 and kPer >= topk / 32; lanes take their slots in batches of
+// kMaxPer.  Run by combine_kernel, and by the spare
+// CTAs of the attention kernel for the previous row chunk.
+struct CombineArgs {
+    const int32_t *ids;
+    const __nv_bfloat16 *part_o;
+    const float *part_lse;
+    __nv_bfloat16 *O;
+    float *lse;
+    int64_t r0, rc;                               // the chunk's query rows
+    int T_, S, Hq, G, R, NB, block, topk;
+    const int32_t *lens;
+};
+
+constexpr int kCombineChunksPerWarp = 4;          // 16-byte channel chunks per warp
+// Warps that merge one (row, group).
+template <int D> constexpr int combine_warps_per_row() { return D / 8 / kCombineChunksPerWarp; }
+
+// The merge of one (row, group) quarter: warp unit `wid` of the chunk
+// (wid < rc * G * combine_warps_per_row<D>()).  kMaxPer: slots per lane,
+// >= topk * R / 32.
+template <int D, int kMaxPer>
+__device__ __forceinline__ void combine_unit(const CombineArgs &c, int64_t wid, int lane) {
+    constexpr int kChunksPerWarp = kCombineChunksPerWarp;
+    constexpr int kWarpsPerRow = combine_warps_per_row<D>();
+    const int32_t *__restrict__ ids = c.ids;
+    const __nv_bfloat16 *__restrict__ part_o = c.part_o;
+    const float *__restrict__ part_lse = c.part_lse;
+    __nv_bfloat16 *__restrict__ O = c.O;
+    float *__restrict__ lse = c.lse;
+    const int64_t r0 = c.r0;
+    const int T_ = c.T_, S = c.S, Hq = c.Hq, G = c.G, R = c.R, NB = c.NB, block = c.block;
+    const int topk = c.topk;
+    const int32_t *__restrict__ lens = c.lens;
+    const int part = (int)(wid % kWarpsPerRow);
+    const int64_t rgl = wid / kWarpsPerRow;
+    const int64_t rl = rgl / G;                   // row within the chunk
+    const int g = (int)(rgl % G);
+    const int64_t r = r0 + rl;
+    const int t = (int)(r % T_);
+    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / block);
+    const SlotPair sp = warp_slots2(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (topk + sstep - 1) / sstep;
+    const int64_t base = (rl * G + g) * topk * R;
+    float li[kMaxPer], m = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        const int sl = s0 + k * sstep;
+        const bool okk = __shfl_sync(0xffffffffu, sl < 32 ? sp.ok0 : sp.ok1, sl & 31);
+        const bool ok = k < per && sl < topk && okk;
+        li[k] = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+        m = fmaxf(m, li[k]);
+    }
+    for (int off = R; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float w[kMaxPer], lsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        w[k] = li[k] == -INFINITY ? 0.f : expf(li[k] - m);
+        lsum += w[k];
+    }
+    for (int off = R; off < 32; off *= 2) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const uint4 *src = (const uint4 *)part_o;
+    __nv_bfloat16 *dst = O + (r * Hq + (int64_t)g * R + h) * D;
+    float acc[kChunksPerWarp][8];
+#pragma unroll
+    for (int c = 0; c < kChunksPerWarp; ++c)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[c][q] = 0.f;
+    // k < per is uniform across the warp, so the loads are issued together;
+    // a slot that holds no partial (weight 0) issues no load and adds 0
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        if (k < per) {
+            const int64_t prow = base + (int64_t)(s0 + k * sstep) * R + h;
+            const bool use = w[k] > 0.f && MSA_IN_BOUNDS(prow, c.rc * G * topk * R);
+#pragma unroll
+            for (int c = 0; c < kChunksPerWarp; ++c) {
+                uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                if (use) u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
+                const __nv_bfloat162 *hp = (const __nv_bfloat162 *)&u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __bfloat1622float2(hp[q]);
+                    acc[c][2 * q] = fmaf(w[k], f.x, acc[c][2 * q]);
+                    acc[c][2 * q + 1] = fmaf(w[k], f.y, acc[c][2 * q + 1]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < kChunksPerWarp; ++c) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            for (int off = R; off < 32; off *= 2)
+                acc[c][q] += __shfl_xor_sync(0xffffffffu, acc[c][q], off);
+        if (s0 == 0) {
+            __nv_bfloat162 o2[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o2[q] = __floats2bfloat162_rn(acc[c][2 * q] * inv, acc[c][2 * q + 1] * inv);
+            *(uint4 *)(dst + (part * kChunksPerWarp + c) * 8) = *(const uint4 *)o2;
+        }
+    }
+    if (part == 0 && s0 == 0) lse[r * Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
+}
+
+// The merge for rows of more than 64 kept blocks: slots taken in batches of
+// kMaxPer per lane; pass 1 finds the maximum LSE, pass 2 weighs and adds.
+template <int D, int kMaxPer, int kPer>
+__device__ __forceinline__ void combine_unit_batched(const CombineArgs &c, int64_t wid, int lane) {
+    constexpr int kChunksPerWarp = kCombineChunksPerWarp;
+    constexpr int kWarpsPerRow = combine_warps_per_row<D>();
+    const int32_t *__restrict__ ids = c.ids;
+    const __nv_bfloat16 *__restrict__ part_o = c.part_o;
+    const float *__restrict__ part_lse = c.part_lse;
+    __nv_bfloat16 *__restrict__ O = c.O;
+    float *__restrict__ lse = c.lse;
+    const int64_t r0 = c.r0;
+    const int T_ = c.T_, S = c.S, Hq = c.Hq, G = c.G, R = c.R, NB = c.NB, block = c.block;
+    const int topk = c.topk;
+    const int32_t *__restrict__ lens = c.lens;
+    const int part = (int)(wid % kWarpsPerRow);
+    const int64_t rgl = wid / kWarpsPerRow;
+    const int64_t rl = rgl / G;                   // row within the chunk
+    const int g = (int)(rgl % G);
+    const int64_t r = r0 + rl;
+    const int t = (int)(r % T_);
+    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / block);
+    const SlotSet<kPer> sp = warp_slots<kPer>(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (topk + sstep - 1) / sstep;   // slots per lane (uniform across the warp)
+    const int64_t base = (rl * G + g) * topk * R;
+    float li0[kMaxPer], m = -INFINITY;            // the first batch's LSEs stay in registers
+    for (int k0 = 0; k0 < per; k0 += kMaxPer) {
+#pragma unroll
+        for (int k = 0; k < kMaxPer; ++k) {
+            const int sl = s0 + (k0 + k) * sstep;
+            const bool ok = k0 + k < per && sl < topk && sp.valid(sl);
+            const float l = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+            if (k0 == 0) li0[k] = l;
+            m = fmaxf(m, l);
+        }
+    }
+    for (int off = R; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const uint4 *src = (const uint4 *)part_o;
+    __nv_bfloat16 *dst = O + (r * Hq + (int64_t)g * R + h) * D;
+    float acc[kChunksPerWarp][8];
+#pragma unroll
+    for (int c = 0; c < kChunksPerWarp; ++c)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[c][q] = 0.f;
+    float lsum = 0.f;
+    for (int k0 = 0; k0 < per; k0 += kMaxPer) {
+        float w[kMaxPer];
+#pragma unroll
+        for (int k = 0; k < kMaxPer; ++k) {
+            float l = li0[k];
+            if (k0 > 0) {
+                const int sl = s0 + (k0 + k) * sstep;
+                const bool ok = k0 + k < per && sl < topk && sp.valid(sl);
+                l = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+            }
+            w[k] = l == -INFINITY ? 0.f : expf(l - m);
+            lsum += w[k];
+        }
+        // k0 + k < per is uniform across the warp, so the loads are issued
+        // together; a slot that holds no partial (weight 0) issues no load
+#pragma unroll
+        for (int k = 0; k < kMaxPer; ++k) {
+            if (k0 + k < per) {
+                const int64_t prow = base + (int64_t)(s0 + (k0 + k) * sstep) * R + h;
+                const bool use = w[k] > 0.f && MSA_IN_BOUNDS(prow, c.rc * G * topk * R);
+#pragma unroll
+                for (int c = 0; c < kChunksPerWarp; ++c) {
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (use) u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
+                    const __nv_bfloat162 *hp = (const __nv_bfloat162 *)&u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 f = __bfloat1622float2(hp[q]);
+                        acc[c][2 * q] = fmaf(w[k], f.x, acc[c][2 * q]);
+                        acc[c][2 * q + 1] = fmaf(w[k], f.y, acc[c][2 * q + 1]);
+                    }
+                }
+            }
+        }
+    }
+    for (int off = R; off < 32; off *= 2) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+    for (int c = 0; c < kChunksPerWarp; ++c) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            for (int off = R; off < 32; off *= 2)
+                acc[c][q] += __shfl_xor_sync(0xffffffffu, acc[c][q], off);
+        if (s0 == 0) {
+            __nv_bfloat162 o2[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                o2[q] = __floats2bfloat162_rn(acc[c][2 * q] * inv, acc[c][2 * q + 1] * inv);
+            *(uint4 *)(dst + (part * kChunksPerWarp + c) * 8) = *(const uint4 *)o2;
+        }
+    }
+    if (part == 0 && s0 == 0) lse[r * Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
+}
+
+// kPer == 0: rows of at most 64 kept blocks and at most kMaxPer slots per
+// lane, one batch; otherwise batches of kMaxPer over up to 32 kPer kept blocks.
+template <int D, int kMaxPer, int kPer>
+__global__ void __launch_bounds__(256, kMaxPer <= 8 ? 3 : 2)
+combine_kernel(CombineArgs c) {
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    if (wid >= c.rc * c.G * combine_warps_per_row<D>()) return;
+    if (kPer == 0) combine_unit<D, kMaxPer>(c, wid, threadIdx.x % 32);
+    else combine_unit_batched<D, kMaxPer, (kPer > 0 ? kPer : 1)>(c, wid, threadIdx.x % 32);
+}
+
 struct AttnArgs {
     const __nv_bfloat16 *Q;     // [B, T, Hq, D]
     const int *recs;            // tile records (rec_ints(tpt) ints each)
@@ -185,6 +471,7 @@ struct AttnArgs {
     __nv_bfloat16 *part_o;      // normalised partial O, blocked chunks (partial_chunk)
     float *part_lse;            // [n_prows]
     int64_t n_prows;            // rc * G * topk * R
+    int64_t q_rows;             // B * T (rows of Q)
     uint32_t *err;
     int64_t r0;
     int T, S, Hq, G, R, NB, topk, tpt;
@@ -192,19 +479,21 @@ struct AttnArgs {
     float scale, scale_log2;
 };
 
-__device__ __forceinline__ int run_tile(int i) {
+// The CTA's i-th tile: runs of kRun consecutive tiles dealt round-robin
+// over the CTAs.
+__device__ __forceinline__ int run_tile(const AttnArgs &, int i) {
     return (i / kRun) * (gridDim.x * kRun) + blockIdx.x * kRun + (i % kRun);
 }
 
 // Header {list, count} of a CTA's i-th tile ({-1, 0} past the end) and entry
 // k (< tpt) of its record (0 past the end); independent loads.
 __device__ __forceinline__ int2 load_head(const AttnArgs &a, int i, int total) {
-    const int tile = run_tile(i);
+    const int tile = run_tile(a, i);
     return tile < total ? __ldg((const int2 *)(a.recs + (int64_t)tile * rec_ints(a.tpt)))
                         : make_int2(-1, 0);
 }
 __device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int k) {
-    const int tile = run_tile(i);
+    const int tile = run_tile(a, i);
     return tile < total && k < a.tpt ? __ldg(a.recs + (int64_t)tile * rec_ints(a.tpt) + 4 + k) : 0;
 }
 
@@ -287,13 +576,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // K/V blocks by TMA (warp 0, lane 0) whenever the list changes, and
             // the tile's Q rows gathered by warps 0 and 3 with 16-byte
             // cp.async copies straight into the 128-byte-swizzled K-major
-            // layout the MMA reads.  Each warp instruction copies two whole
-            // 256-byte rows; lane l always copies 16-byte chunk l % 16.  A
+            // layout the MMA reads.  Each warp instruction copies kRPI whole
+            // rows of D / 8 16-byte chunks (two rows for D = 128, four for
+            // D = 64); lane l always copies chunk l % (D / 8).  A
             // thread's copies arrive on q_full when they complete
             // (cp.async.mbarrier.arrive.noinc), so no warp waits for its own
             // copies and loads run up to three tiles ahead.
+            constexpr int kCPR = D / 8, kRPI = 32 / kCPR;   // chunks per row, rows per instruction
             const int gw = warp == 0 ? 0 : 1;          // gather warp 0..1
-            const int cc = lane % 16;
+            const int cc = lane % kCPR;
             const uint32_t q_swz = (uint32_t)(cc / 8) * 1024;
             const int lr = __ffs(a.R) - 1;             // log2 R
             // A token's Q rows are read once per kept block: keep them in L2
@@ -371,16 +662,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const uint32_t dst = tc::smem_u32(sQ + qb * kQBytes) + q_swz;
                 const int rows = count << lr;
                 const int64_t head0 = (int64_t)g * a.R;
-                // row pair q = rows 2q, 2q + 1 (lanes 0-15 / 16-31); both rows'
-                // tokens sit in the same 32-token block, so one register holds
-                // their entries and a shuffle hands each lane its token's entry
-                for (int q = gw; 2 * q < rows; q += 2) {
-                    const int r = 2 * q + lane / 16;
+                // row group q = rows kRPI q .. kRPI q + kRPI - 1 (lane / kCPR);
+                // their tokens sit in the same 32-token block, so one register
+                // holds their entries and a shuffle hands each lane its token's
+                // entry
+                for (int q = gw; kRPI * q < rows; q += 2) {
+                    const int r = kRPI * q + lane / kCPR;
                     const int tk = r >> lr, hh = r & (a.R - 1);
-                    const int kk = (2 * q) >> (lr + 5);
+                    const int kk = (kRPI * q) >> (lr + 5);
                     const int ev = kk == 0 ? e[0] : kk == 1 ? e[1] : kk == 2 ? e[2] : e[3];
                     const int ent = __shfl_sync(0xffffffffu, ev, tk & 31);
-                    if (r < rows) {
+                    if (r < rows && MSA_IN_BOUNDS(a.r0 + (ent >> 8), a.q_rows)) {
                         const __nv_bfloat16 *src =
                             a.Q + ((a.r0 + (ent >> 8)) * a.Hq + head0 + hh) * D + cc * 8;
                         const uint32_t sa = dst + (r / 8) * kGroupBytes + (r % 8) * 128 +
@@ -584,7 +876,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t tO = tmem + kOCol + lane_off;
         // partials are read back only by the combine: first out of L2
         const uint64_t st_pol = tc::policy_evict_first();
-        for (int i = 0; run_tile(i) < total; ++i) {
+        for (int i = 0; run_tile(a, i) < total; ++i) {
             if (!tc::mbar_wait(o_full, i & 1, a.err, abort_flag)) break;
             tc::tc_fence_after();
             uint32_t ov[D];
@@ -606,7 +898,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                                           __uint_as_float(ov[c + 1]) * inv);
                 ov[c / 2] = *(uint32_t *)&hv;
             }
-            if (prow >= 0) {
+            if (prow >= 0 && MSA_IN_BOUNDS(prow, a.n_prows)) {
                 uint4 *dst = (uint4 *)a.part_o + partial_chunk(prow, 0, D);
 #pragma unroll
                 for (int c = 0; c < D / 2; c += 4)
@@ -630,101 +922,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 namespace msa {
 namespace {
 
-// Phase 2: the LSE-weighted merge of a (query row, group)'s partials over
-// its valid kept slots, for each of the group's R heads: weights
-// exp(lse_i - max lse) give the softmax over the union of the slots' keys.
-// Four warps share a (row, group), each merging a quarter of the d/8 16-byte
-// channel chunks.  Lane l owns head l % R and slots l / R, l / R + 32 / R, ...;
-// with the blocked chunk layout every load of the warp is 512 contiguous
-// bytes, and all loads of a warp are independent (issued together).
-// Needs R | 32 and topk <= 64.
-template <int D, int kMaxPer>
-__global__ void __launch_bounds__(256, kMaxPer <= 8 ? 3 : 2)
-combine_kernel(const int32_t *__restrict__ ids, const __nv_bfloat16 *__restrict__ part_o,
-                               const float *__restrict__ part_lse, __nv_bfloat16 *__restrict__ O,
-                               float *__restrict__ lse, int64_t r0, int64_t rc, int T_, int S,
-                               int Hq, int G, int R, int NB, int block, int topk,
-                               const int32_t *__restrict__ lens) {
-    constexpr int kChunksPerWarp = 4;             // kMaxPer: slots per lane, >= topk * R / 32
-    constexpr int kWarpsPerRow = D / 8 / kChunksPerWarp;
-    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-    const int lane = threadIdx.x % 32;
-    if (wid >= rc * G * kWarpsPerRow) return;
-    const int part = (int)(wid % kWarpsPerRow);
-    const int64_t rgl = wid / kWarpsPerRow;
-    const int64_t rl = rgl / G;                   // row within the chunk
-    const int g = (int)(rgl % G);
-    const int64_t r = r0 + rl;
-    const int t = (int)(r % T_);
-    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
-    const int cb = p < 0 ? -1 : (int)(p / block);
-    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
-    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
-    const int per = (topk + sstep - 1) / sstep;
-    const int64_t base = (rl * G + g) * topk * R;
-    float li[kMaxPer], m = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-        const int sl = s0 + k * sstep;
-        const bool okk = __shfl_sync(0xffffffffu, sl < 32 ? sp.ok0 : sp.ok1, sl & 31);
-        const bool ok = k < per && sl < topk && okk;
-        li[k] = ok ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
-        m = fmaxf(m, li[k]);
-    }
-    for (int off = R; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    float w[kMaxPer], lsum = 0.f;
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-        w[k] = li[k] == -INFINITY ? 0.f : expf(li[k] - m);
-        lsum += w[k];
-    }
-    for (int off = R; off < 32; off *= 2) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    const uint4 *src = (const uint4 *)part_o;
-    __nv_bfloat16 *dst = O + (r * Hq + (int64_t)g * R + h) * D;
-    float acc[kChunksPerWarp][8];
-#pragma unroll
-    for (int c = 0; c < kChunksPerWarp; ++c)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[c][q] = 0.f;
-    // k < per is uniform across the warp, so the loads are issued together;
-    // a slot that holds no partial (weight 0) issues no load and adds 0
-#pragma unroll
-    for (int k = 0; k < kMaxPer; ++k) {
-        if (k < per) {
-            const int64_t prow = base + (int64_t)(s0 + k * sstep) * R + h;
-            const bool use = w[k] > 0.f;
-#pragma unroll
-            for (int c = 0; c < kChunksPerWarp; ++c) {
-                uint4 u = make_uint4(0u, 0u, 0u, 0u);
-                if (use) u = src[partial_chunk(prow, part * kChunksPerWarp + c, D)];
-                const __nv_bfloat162 *hp = (const __nv_bfloat162 *)&u;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __bfloat1622float2(hp[q]);
-                    acc[c][2 * q] = fmaf(w[k], f.x, acc[c][2 * q]);
-                    acc[c][2 * q + 1] = fmaf(w[k], f.y, acc[c][2 * q + 1]);
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int c = 0; c < kChunksPerWarp; ++c) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            for (int off = R; off < 32; off *= 2)
-                acc[c][q] += __shfl_xor_sync(0xffffffffu, acc[c][q], off);
-        if (s0 == 0) {
-            __nv_bfloat162 o2[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                o2[q] = __floats2bfloat162_rn(acc[c][2 * q] * inv, acc[c][2 * q + 1] * inv);
-            *(uint4 *)(dst + (part * kChunksPerWarp + c) * 8) = *(const uint4 *)o2;
-        }
-    }
-    if (part == 0 && s0 == 0) lse[r * Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
-}
-
 // The indexer's KL target for query rows [r0, r0 + rc), run after their
 // merge: slot sl's share of head h's softmax is exp(part_lse - lse) of that
 // slot (0 for slots no tile served), averaged over the group's R heads.  One
@@ -743,7 +940,7 @@ block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ par
     const int t = (int)(r % T_);
     const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
     const int cb = p < 0 ? -1 : (int)(p / block);
-    const SlotPair sp = warp_slots(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const SlotPair sp = warp_slots2(ids + (r * G + g) * topk, topk, NB, cb, lane);
     const int h = lane % R, s0 = lane / R, sstep = 32 / R;
     const int per = (topk + sstep - 1) / sstep;
     const float l = lse[r * Hq + (int64_t)g * R + h];
@@ -765,6 +962,63 @@ block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ par
         for (int off = 1; off < R; off *= 2) share += __shfl_xor_sync(0xffffffffu, share, off);
         if (h == 0 && sl < topk) mrow[sl] = share / (float)R;
     }
+}
+
+// More than 64 kept blocks or 16 slots per lane: the same, slots taken in
+// batches of 16 per lane.
+__global__ void __launch_bounds__(256)
+block_mass_wide_kernel(const int32_t *__restrict__ ids, const float *__restrict__ part_lse,
+                  const float *__restrict__ lse, float *__restrict__ mass, int64_t r0, int64_t rc,
+                  int T_, int S, int Hq, int G, int R, int NB, int block, int topk,
+                  const int32_t *__restrict__ lens) {
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (x >= rc * G) return;
+    const int64_t rl = x / G, r = r0 + rl;
+    const int g = (int)(x % G);
+    const int t = (int)(r % T_);
+    const int64_t p = seq_len(lens, (int)(r / T_), S) - T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / block);
+    const SlotSet<8> sp = warp_slots<8>(ids + (r * G + g) * topk, topk, NB, cb, lane);
+    const int h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (topk + sstep - 1) / sstep;
+    const float l = lse[r * Hq + (int64_t)g * R + h];
+    const int64_t base = x * topk * R;
+    float *mrow = mass + (r * G + g) * topk;
+    constexpr int kMaxPer = 16;                     // slots per lane and batch
+    for (int k0 = 0; k0 < per; k0 += kMaxPer) {
+        float li[kMaxPer];                          // every load of a batch issued before any use
+#pragma unroll
+        for (int k = 0; k < kMaxPer; ++k) {
+            const int sl = s0 + (k0 + k) * sstep;
+            li[k] = (k0 + k < per && sl < topk && sp.valid(sl))
+                        ? part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+        }
+#pragma unroll
+        for (int k = 0; k < kMaxPer; ++k) {
+            if (k0 + k >= per) break;               // per is uniform across the warp
+            const int sl = s0 + (k0 + k) * sstep;
+            float share = (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
+            for (int off = 1; off < R; off *= 2) share += __shfl_xor_sync(0xffffffffu, share, off);
+            if (h == 0 && sl < topk) mrow[sl] = share / (float)R;
+        }
+    }
+}
+
+int combine_per(const Shape &s) { return (s.topk + 32 / s.R - 1) / (32 / s.R); }  // slots per lane
+bool combine_wide(const Shape &s) { return combine_per(s) > 8; }
+// More than 64 kept blocks, or more than 16 slots per merging lane: batches.
+bool combine_batched(const Shape &s) { return s.topk > 64 || combine_per(s) > 16; }
+
+CombineArgs combine_args(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
+                         const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
+                         const int32_t *lens) {
+    CombineArgs c;
+    c.ids = ids; c.part_o = part_o; c.part_lse = part_lse; c.O = (__nv_bfloat16 *)O; c.lse = lse;
+    c.r0 = r0; c.rc = rc;
+    c.T_ = s.T; c.S = s.S; c.Hq = s.Hq; c.G = s.G; c.R = s.R; c.NB = s.NB; c.block = s.block;
+    c.topk = s.topk; c.lens = lens;
+    return c;
 }
 
 constexpr size_t kPartialBudget = (size_t)4 << 30;   // bytes of partials per chunk
@@ -847,11 +1101,13 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         if (e != cudaSuccess) return e;
         const int64_t nrow = rc * s.G;                      // one warp each
         const unsigned g1 = (unsigned)((nrow * 32 + 255) / 256);
-        csr_count_kernel<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB,
-                                             s.block, s.topk);
+        auto count_k = s.topk > 64 ? csr_count_kernel<8> : csr_count_kernel<2>;
+        auto fill_k = s.topk > 64 ? csr_fill_kernel<8> : csr_fill_kernel<2>;
+        count_k<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB, s.block,
+                                    s.topk);
         csr_scan_kernel<<<1, 1024, 0, st>>>(counts, toffs, L, pl.tpt);
-        csr_fill_kernel<<<g1, 256, 0, st>>>(ids, toffs, cursor, recs, r0, rc, s.T, s.S, s.G,
-                                            s.NB, s.block, s.topk, pl.tpt);
+        fill_k<<<g1, 256, 0, st>>>(ids, toffs, cursor, recs, r0, rc, s.T, s.S, s.G, s.NB,
+                                   s.block, s.topk, pl.tpt, (int64_t)(pl.part_o - pl.recs) / 4);
         csr_tiles_kernel<<<(L + 255) / 256, 256, 0, st>>>(counts, toffs, recs, L, pl.tpt);
         AttnArgs a{};
         a.Q = (const __nv_bfloat16 *)Q;
@@ -859,6 +1115,7 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         a.n_tiles = toffs + L;
         a.part_o = part_o; a.part_lse = part_lse; a.err = err; a.r0 = r0;
         a.n_prows = rc * s.G * s.topk * s.R;
+        a.q_rows = s.rows();
         a.T = s.T; a.S = s.S; a.Hq = s.Hq; a.G = s.G; a.R = s.R; a.NB = s.NB; a.topk = s.topk;
         a.tpt = pl.tpt;
         a.q_box4 = q_box4;
@@ -876,35 +1133,75 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 }  // namespace
 
+cudaError_t launch_block_mass(const Shape &s, const int32_t *ids, const float *part_lse,
+                              const float *lse, float *mass, int64_t r0, int64_t rc,
+                              cudaStream_t st, const int32_t *lens) {
+    const unsigned mgrid = (unsigned)((rc * s.G * 32 + 255) / 256);
+    auto k = combine_batched(s) ? block_mass_wide_kernel : block_mass_kernel;
+    k<<<mgrid, 256, 0, st>>>(ids, part_lse, lse, mass, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
+                             s.block, s.topk, lens);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
                            const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st, float *mass, const int32_t *lens) {
-    const int64_t warps = rc * s.G * (128 / 32);
+    const int64_t warps = rc * s.G * (s.d / 8 / kCombineChunksPerWarp);
     const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
-    const int per = (s.topk + 32 / s.R - 1) / (32 / s.R);
-    auto kern = per <= 8 ? combine_kernel<128, 8> : combine_kernel<128, 16>;
-    kern<<<grid, 256, 0, st>>>(ids, part_o, part_lse, (__nv_bfloat16 *)O, lse, r0, rc, s.T, s.S,
-                               s.Hq, s.G, s.R, s.NB, s.block, s.topk, lens);
+    // slots per merging lane: one batch of 8 or 16, or batches of 8 past 64 kept blocks
+    const bool batched = combine_batched(s);
+    auto kern = s.d == 64 ? (batched ? combine_kernel<64, 8, 8>
+                             : combine_wide(s) ? combine_kernel<64, 16, 0>
+                                               : combine_kernel<64, 8, 0>)
+                          : (batched ? combine_kernel<128, 8, 8>
+                             : combine_wide(s) ? combine_kernel<128, 16, 0>
+                                               : combine_kernel<128, 8, 0>);
+    kern<<<grid, 256, 0, st>>>(combine_args(s, ids, part_o, part_lse, O, lse, r0, rc, lens));
     count_launches(1);
     if (mass != nullptr) {
         const cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        const unsigned mgrid = (unsigned)((rc * s.G * 32 + 255) / 256);
-        block_mass_kernel<<<mgrid, 256, 0, st>>>(ids, part_lse, lse, mass, r0, rc, s.T, s.S, s.Hq,
-                                                 s.G, s.R, s.NB, s.block, s.topk, lens);
-        count_launches(1);
+        return launch_block_mass(s, ids, part_lse, lse, mass, r0, rc, st, lens);
     }
     return cudaGetLastError();
 }
 
+cudaError_t launch_slot_csr(const Shape &s, const int32_t *ids, int tpt, int64_t r0, int64_t rc,
+                            int *counts, int *cursor, int *toffs, int *recs, uint32_t *err,
+                            cudaStream_t st) {
+    const int L = s.B * s.G * s.NB;
+    cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int) * (size_t)L, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(cursor, 0, sizeof(int) * (size_t)L, st);
+    if (e != cudaSuccess) return e;
+    const unsigned g1 = (unsigned)((rc * s.G * 32 + 255) / 256);
+    auto count_k = s.topk > 64 ? csr_count_kernel<8> : csr_count_kernel<2>;
+    auto fill_k = s.topk > 64 ? csr_fill_kernel<8> : csr_fill_kernel<2>;
+    count_k<<<g1, 256, 0, st>>>(ids, counts, err, r0, rc, s.T, s.S, s.G, s.NB, s.block, s.topk);
+    csr_scan_kernel<<<1, 1024, 0, st>>>(counts, toffs, L, tpt);
+    fill_k<<<g1, 256, 0, st>>>(ids, toffs, cursor, recs, r0, rc, s.T, s.S, s.G, s.NB, s.block,
+                               s.topk, tpt,
+                               (int64_t)(slot_csr_records(s, rc, tpt) * rec_ints(tpt)));
+    csr_tiles_kernel<<<(L + 255) / 256, 256, 0, st>>>(counts, toffs, recs, L, tpt);
+    count_launches(4);
+    return cudaGetLastError();
+}
+
+size_t slot_csr_records(const Shape &s, int64_t rc, int tpt) {
+    const size_t slots = (size_t)rc * s.G * s.topk;
+    return (slots + tpt - 1) / tpt + (size_t)s.B * s.G * s.NB;
+}
+
+int slot_csr_record_ints(int tpt) { return rec_ints(tpt); }
+
 bool combine_supported(const Shape &s) {
     return (s.R == 1 || s.R == 2 || s.R == 4 || s.R == 8 || s.R == 16 || s.R == 32) &&
-           s.topk <= 64 && (s.topk + 32 / s.R - 1) / (32 / s.R) <= 16;
+           s.topk <= 256;
 }
 
 bool attn_tc_supported(const Shape &s) {
-    return s.dtype == MSA_BF16 && s.d == 128 && (s.block == 128 || s.block == 64) && s.R <= 16 &&
-           combine_supported(s);
+    return s.dtype == MSA_BF16 && (s.d == 128 || s.d == 64) && (s.block == 128 || s.block == 64) &&
+           s.R <= 16 && combine_supported(s);
 }
 
 size_t attn_tc_workspace(const Shape &s) { return make_plan(s).total; }
@@ -914,6 +1211,9 @@ int64_t attn_tc_rows_per_pass(const Shape &s) { return make_plan(s).rows_per_chu
 cudaError_t launch_attn_tc(const Shape &s, const void *Q, const void *K, const void *V,
                            const int32_t *ids, void *O, float *lse, uint32_t *err, void *ws,
                            cudaStream_t st, float *mass) {
+    if (s.d == 64)
+        return s.block == 128 ? run_chunks<64, 128>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass)
+                              : run_chunks<64, 64>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass);
     if (s.block == 128)
         return run_chunks<128, 128>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass);
     return run_chunks<128, 64>(s, Q, K, V, ids, O, lse, err, (char *)ws, st, mass);

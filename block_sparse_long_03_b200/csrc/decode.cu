@@ -73,11 +73,12 @@ __device__ __forceinline__ int swz(int r, int c, int row_bytes) {
 // double-buffered in shared memory.  Key rows are found through `rows`
 // (dense or paged); keys at or past the sequence's length L are never read
 // (zero in shared memory, and masked: every query sits before L).
-template <int DIDX, int NCG, int WARPS>
+template <int DIDX, int NCG, int WARPS, bool kPaged>
 __global__ void __launch_bounds__(WARPS * 32)
 decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16 *__restrict__ k_idx,
                     float *__restrict__ bs, int T_, int S, int G, int NB, int block,
-                    int blocks_per_warp, KeyRows rows, const int32_t *__restrict__ lens) {
+                    int blocks_per_warp, KeyRows rows, const int32_t *__restrict__ lens,
+                    int64_t kv_rows) {
     constexpr int kRowBytes = DIDX * 2;
     constexpr int kChunks = DIDX / 8;
     constexpr int kSub = 64;                               // keys per staged sub-block
@@ -128,14 +129,22 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
     const int spb = block / kSub;                          // sub-blocks per block
     const int first = first_blk * spb, last = last_blk * spb;
     auto stage = [&](int sb, uint8_t *dst) {
-        for (int c = lane; c < kSub * kChunks; c += 32) {
-            const int r = c / kChunks, ch = c % kChunks;
-            const int64_t j = (int64_t)sb * kSub + r;
-            const int64_t row = j < L ? rows.row(b, j) : -1;
-            if (row >= 0)
-                cp_async16(dst + swz(r, ch, kRowBytes), k_idx + row * DIDX + ch * 8);
-            else
-                *(uint4 *)(dst + swz(r, ch, kRowBytes)) = make_uint4(0u, 0u, 0u, 0u);
+        if (!kPaged) {                                     // whole sequences of S keys
+            const __nv_bfloat16 *src = k_idx + ((int64_t)b * S + (int64_t)sb * kSub) * DIDX;
+            for (int c = lane; c < kSub * kChunks; c += 32) {
+                const int r = c / kChunks, ch = c % kChunks;
+                cp_async16(dst + swz(r, ch, kRowBytes), src + (int64_t)r * DIDX + ch * 8);
+            }
+        } else {
+            for (int c = lane; c < kSub * kChunks; c += 32) {
+                const int r = c / kChunks, ch = c % kChunks;
+                const int64_t j = (int64_t)sb * kSub + r;
+                const int64_t row = j < L ? rows.row(b, j) : -1;
+                if (row >= 0 && MSA_IN_BOUNDS(row, kv_rows))
+                    cp_async16(dst + swz(r, ch, kRowBytes), k_idx + row * DIDX + ch * 8);
+                else
+                    *(uint4 *)(dst + swz(r, ch, kRowBytes)) = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
         cp_async_commit();
     };
@@ -201,13 +210,14 @@ constexpr int kAttnThreads = 128;
 // group's query heads (the width of one mma tile): the partial softmax of
 // those heads over that block's causal keys.  With R = 16 two CTAs share a
 // slot, heads 0-7 and 8-15.
-template <int D, int BLOCK>
+template <int D, int BLOCK, bool kPaged>
 __global__ void __launch_bounds__(kAttnThreads)
 decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
                     const __nv_bfloat16 *__restrict__ V, const int32_t *__restrict__ ids,
                     __nv_bfloat16 *__restrict__ part_o, float *__restrict__ part_lse, uint32_t *err,
                     int T_, int S, int Hq, int Hkv, int R, int NB, int topk, float scale_log2,
-                    float scale, int64_t n_prows, KeyRows rows, const int32_t *__restrict__ lens) {
+                    float scale, int64_t n_prows, KeyRows rows, const int32_t *__restrict__ lens,
+                    int64_t kv_rows) {
     constexpr int kRowBytes = D * 2;
     constexpr int kChunks = D / 8;
     extern __shared__ __align__(128) uint8_t sm[];
@@ -246,8 +256,9 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     // stage K and V rows of the block (zero rows past the last causal key)
     for (int c = tid; c < BLOCK * kChunks; c += kAttnThreads) {
         const int r = c / kChunks, ch = c % kChunks;
-        const int64_t kr = r < nk ? rows.row(b, j0 + r) : -1;
-        if (kr >= 0) {
+        const int64_t kr = r >= nk ? -1
+                           : kPaged ? rows.row(b, j0 + r) : (int64_t)b * S + j0 + r;
+        if (kr >= 0 && MSA_IN_BOUNDS(kr, kv_rows)) {
             const int64_t src = (kr * Hkv + g) * D + ch * 8;
             cp_async16(sK + swz(r, ch, kRowBytes), K + src);
             cp_async16(sV + swz(r, ch, kRowBytes), V + src);
@@ -383,9 +394,10 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
     const int64_t prow0 = (rg * topk + slot) * R + h0;
     for (int c = tid; c < Rh * kChunks; c += kAttnThreads) {
         const int h = c % Rh, ch = c / Rh;
-        ((uint4 *)part_o)[partial_chunk(prow0 + h, ch, D)] = *(const uint4 *)(sO + h * D + ch * 8);
+        if (MSA_IN_BOUNDS(prow0 + h, n_prows))
+            ((uint4 *)part_o)[partial_chunk(prow0 + h, ch, D)] = *(const uint4 *)(sO + h * D + ch * 8);
     }
-    if (tid < Rh) {
+    if (tid < Rh && MSA_IN_BOUNDS(prow0 + tid, n_prows)) {
         const int h = tid;
         const float l = sRed[h] + sRed[8 + h] + sRed[16 + h] + sRed[24 + h];
         part_lse[prow0 + h] = sMax[h] * scale + logf(l);
@@ -397,13 +409,16 @@ cudaError_t launch_index_t(const Shape &s, const void *q_idx, const void *k_idx,
                            cudaStream_t st, const KeyRows &rows, const int32_t *lens) {
     constexpr int W = DIDX == 64 ? 8 : 4;
     const size_t smem = (size_t)W * 2 * 64 * DIDX * 2;
-    auto k = decode_index_kernel<DIDX, NCG, W>;
+    auto k = rows.table ? decode_index_kernel<DIDX, NCG, W, true>
+                        : decode_index_kernel<DIDX, NCG, W, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int bpw = 4;                                     // blocks per warp
     const dim3 grid((unsigned)((s.NB + W * bpw - 1) / (W * bpw)), (unsigned)s.B);
     k<<<grid, W * 32, smem, st>>>((const __nv_bfloat16 *)q_idx, (const __nv_bfloat16 *)k_idx, bs,
-                                  s.T, s.S, s.G, s.NB, s.block, bpw, rows, lens);
+                                  s.T, s.S, s.G, s.NB, s.block, bpw, rows, lens,
+                                  rows.table ? (int64_t)rows.num_pages * rows.page_size
+                                             : (int64_t)s.B * s.S);
     count_launches(1);
     return cudaGetLastError();
 }
@@ -426,7 +441,7 @@ cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const v
                            cudaStream_t st, const KeyRows &rows, const int32_t *lens) {
     constexpr int D = 128;
     const size_t smem = 2 * (size_t)BLOCK * D * 2 + 8 * BLOCK * 2 + 40 * 4 + 8 * D * 2;
-    auto k = decode_block_kernel<D, BLOCK>;
+    auto k = rows.table ? decode_block_kernel<D, BLOCK, true> : decode_block_kernel<D, BLOCK, false>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t ctas = s.index_rows() * s.topk * ((s.R + 7) / 8);
@@ -434,7 +449,8 @@ cudaError_t launch_block_t(const Shape &s, const void *Q, const void *K, const v
     k<<<(unsigned)ctas, kAttnThreads, smem, st>>>(
         (const __nv_bfloat16 *)Q, (const __nv_bfloat16 *)K, (const __nv_bfloat16 *)V, ids, part_o,
         part_lse, err, s.T, s.S, s.Hq, s.Hkv, s.R, s.NB, s.topk, scale_log2, s.scale,
-        (int64_t)s.index_rows() * s.topk * s.R, rows, lens);
+        (int64_t)s.index_rows() * s.topk * s.R, rows, lens,
+        rows.table ? (int64_t)rows.num_pages * rows.page_size : (int64_t)s.B * s.S);
     count_launches(1);
     return cudaGetLastError();
 }

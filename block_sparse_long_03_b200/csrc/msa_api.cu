@@ -11,6 +11,10 @@
 
 namespace msa {
 
+#if MSA_CHECKED
+__device__ unsigned int g_msa_bounds_failures = 0;
+#endif
+
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
@@ -52,9 +56,17 @@ size_t block_score_bytes(const Shape &s) { return sizeof(float) * (size_t)s.inde
 size_t block_id_bytes(const Shape &s) { return sizeof(int32_t) * (size_t)s.index_rows() * s.topk; }
 
 // Prefill shapes go to the tensor-core KV-block-outer kernel; decode-like
-// shapes (few query tokens per sequence) to the query-outer kernel.
-bool use_attn_tc(const Shape &s) { return attn_tc_supported(s) && s.T >= 64; }
+// shapes (few query tokens per sequence) to the query-outer kernel, or to the
+// tensor-core kernel where the decode kernel lacks the shape (d = 64).  fp32
+// runs on CUDA cores; a bf16 shape with neither tensor-core path (a group
+// size R outside {1, 2, 4, 8, 16}) is not supported rather than run there.
+bool use_attn_tc(const Shape &s) {
+    return attn_tc_supported(s) && (s.T >= 64 || !decode_attn_supported(s));
+}
 bool use_attn_decode(const Shape &s) { return !use_attn_tc(s) && decode_attn_supported(s); }
+bool attn_supported(const Shape &s) {
+    return s.dtype == MSA_F32 || use_attn_tc(s) || use_attn_decode(s);
+}
 size_t attn_scratch(const Shape &s) {
     if (use_attn_tc(s)) return align_up(attn_tc_workspace(s));
     if (use_attn_decode(s)) return align_up(decode_attn_workspace(s));
@@ -154,6 +166,8 @@ size_t host_ws_size(const Shape &s);
 // Workspace bytes of msa_decode_paged (defined with that call below); 0 when
 // the shapes have no paged path.
 size_t paged_ws_size(const Shape &s);
+// Workspace bytes of msa_index_hierarchical (defined with that call below).
+size_t hier_ws_size(const Shape &s);
 
 }  // namespace
 }  // namespace msa
@@ -179,10 +193,14 @@ const char *msa_status_string(msa_status_t status) {
 size_t msa_workspace_size(const msa_params_t *params, int which) {
     Shape s;
     if (make_shape(params, &s) != MSA_OK) return 0;
+    if ((which == MSA_WS_SPARSE_ATTN || which == MSA_WS_FORWARD || which == MSA_WS_FORWARD_HOST) &&
+        !attn_supported(s))
+        return 0;
     if (which == MSA_WS_SPARSE_ATTN) return attn_ws(s);
     if (which == MSA_WS_FORWARD) return forward_ws(s);
     if (which == MSA_WS_FORWARD_HOST) return host_ws_size(s);
     if (which == MSA_WS_DECODE_PAGED) return paged_ws_size(s);
+    if (which == MSA_WS_INDEX_HIER) return hier_ws_size(s);
     return 0;
 }
 
@@ -225,6 +243,7 @@ msa_status_t msa_sparse_attn_fwd_mass(const msa_params_t *params, const void *Q,
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(block_ids) ||
         !aligned16(O) || !aligned16(lse) || (block_mass && !aligned16(block_mass)))
         return MSA_ERR_INVALID_ARG;
+    if (!attn_supported(s)) return MSA_ERR_UNSUPPORTED;
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < attn_ws(s))
         return MSA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -256,6 +275,7 @@ msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx, con
         !aligned16(V) || !aligned16(O) || !aligned16(lse) ||
         (block_ids && !aligned16(block_ids)) || (block_mass && !aligned16(block_mass)))
         return MSA_ERR_INVALID_ARG;
+    if (!attn_supported(s)) return MSA_ERR_UNSUPPORTED;
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < forward_ws(s))
         return MSA_ERR_WORKSPACE;
     cudaStream_t st = (cudaStream_t)stream;
@@ -281,6 +301,17 @@ msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx, con
 }
 
 uint64_t msa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+uint32_t msa_bounds_failures(void) {
+#if MSA_CHECKED
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, msa::g_msa_bounds_failures, sizeof v) != cudaSuccess)
+        return 0xffffffffu;
+    return v;
+#else
+    return 0;
+#endif
+}
 
 msa_status_t msa_get_device_error(void *workspace, void *stream) {
     if (!workspace || ((uintptr_t)workspace % kAlign) != 0) return MSA_ERR_WORKSPACE;
@@ -524,6 +555,7 @@ extern "C" msa_status_t msa_forward_host(const msa_params_t *params, const void 
     Shape s;
     msa_status_t rc = make_shape(params, &s);
     if (rc != MSA_OK) return rc;
+    if (!attn_supported(s)) return MSA_ERR_UNSUPPORTED;
     const HostLayout L = host_layout(s);
     if (!device_buffer || ((uintptr_t)device_buffer % kAlign) != 0 ||
         device_buffer_bytes < L.total)
@@ -731,5 +763,107 @@ extern "C" msa_status_t msa_decode_paged(const msa_params_t *params, const int32
     if (e == cudaSuccess)
         e = launch_decode_attn(s, Q, K_cache, V_cache, ids, O, lse, err, ws + L.scratch, st,
                                nullptr, &rows, lens_ok);
+    return cuda_status(e);
+}
+
+// ---------------------------------------------------------------------------
+// msa_index_hierarchical: coarse-to-fine block selection (see include/msa.h
+// and hier.cu).  Each sequence is taken in the query pieces msa_forward
+// scores in (the coarse scores have the block scores' size); per piece:
+// coarse scores, the kc best candidates (Top-k kernel), their slot CSR,
+// their exact scores, and the final selection among them.
+// ---------------------------------------------------------------------------
+namespace msa {
+namespace {
+
+constexpr int kHierMaxKc = 64;
+constexpr int kHierTpt = 128;
+
+struct HierLayout {
+    size_t kmean, cs, cand, fine, counts, cursor, toffs, recs, total;
+};
+
+HierLayout hier_layout(const Shape &s) {
+    Shape s1 = s;
+    s1.B = 1;
+    int64_t rows = 0;                              // index rows of the largest piece
+    for (const Piece &p : score_pieces(s1))
+        rows = std::max<int64_t>(rows, (int64_t)(p.t1 - p.t0) * s.G);
+    Shape pk = s1;
+    pk.topk = kHierMaxKc;
+    const int64_t L = (int64_t)s.G * s.NB;
+    HierLayout H;
+    size_t o = kErrorBytes;
+    H.kmean = o;  o += align_up(sizeof(float) * (size_t)s.B * s.NB * s.d_idx);
+    H.cs = o;     o += align_up(score_bytes(s1));
+    H.cand = o;   o += align_up(sizeof(int32_t) * (size_t)rows * kHierMaxKc);
+    H.fine = o;   o += align_up(sizeof(float) * (size_t)rows * kHierMaxKc);
+    H.counts = o; o += align_up(sizeof(int) * (size_t)L);
+    H.cursor = o; o += align_up(sizeof(int) * (size_t)L);
+    H.toffs = o;  o += align_up(sizeof(int) * (size_t)(L + 1));
+    H.recs = o;
+    o += align_up(sizeof(int) * (size_t)slot_csr_record_ints(kHierTpt) *
+                  slot_csr_records(pk, rows / s.G, kHierTpt));
+    H.total = o;
+    return H;
+}
+
+size_t hier_ws_size(const Shape &s) {
+    return fine_scores_supported(s) ? hier_layout(s).total : 0;
+}
+
+}  // namespace
+}  // namespace msa
+
+extern "C" msa_status_t msa_index_hierarchical(const msa_params_t *params, int32_t kc,
+                                               const void *q_idx, const void *k_idx,
+                                               int32_t *block_ids, void *workspace,
+                                               size_t workspace_bytes, void *stream) {
+    Shape s;
+    msa_status_t rc = make_shape(params, &s);
+    if (rc != MSA_OK) return rc;
+    if (kc < s.topk) return MSA_ERR_INVALID_ARG;
+    if (kc > kHierMaxKc || !fine_scores_supported(s)) return MSA_ERR_UNSUPPORTED;
+    if (!q_idx || !k_idx || !block_ids) return MSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(block_ids))
+        return MSA_ERR_INVALID_ARG;
+    const HierLayout H = hier_layout(s);
+    if (!workspace || ((uintptr_t)workspace % kAlign) != 0 || workspace_bytes < H.total)
+        return MSA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char *ws = (char *)workspace;
+    uint32_t *err = (uint32_t *)ws;
+    float *kmean = (float *)(ws + H.kmean), *cs = (float *)(ws + H.cs);
+    float *fine = (float *)(ws + H.fine);
+    int32_t *cand = (int32_t *)(ws + H.cand);
+    int *counts = (int *)(ws + H.counts), *cursor = (int *)(ws + H.cursor);
+    int *toffs = (int *)(ws + H.toffs), *recs = (int *)(ws + H.recs);
+    const size_t e_sz = elem_bytes(s);
+    Shape s1 = s;
+    s1.B = 1;
+    const std::vector<Piece> pieces = score_pieces(s1);
+    cudaError_t e = cudaMemsetAsync(err, 0, kErrorBytes, st);
+    if (e == cudaSuccess) e = launch_coarse_keys(s, k_idx, kmean, st);
+    for (int b = 0; b < s.B && e == cudaSuccess; ++b) {
+        for (const Piece &p : pieces) {
+            if (e != cudaSuccess) break;
+            const Shape ps = piece_shape(s1, p);      // B = 1, T' = t1 - t0, S' = S - T + t1
+            Shape pk = ps;
+            pk.topk = kc;
+            const int64_t row0 = (int64_t)b * s.T + p.t0;
+            const char *q = (const char *)q_idx + row0 * s.G * s.d_idx * e_sz;
+            const char *k = (const char *)k_idx + (int64_t)b * s.S * s.d_idx * e_sz;
+            e = launch_coarse_scores(ps, q, kmean + (size_t)b * s.NB * s.d_idx, cs, st);
+            if (e == cudaSuccess) e = launch_topk(pk, cs, cand, st);
+            if (e == cudaSuccess)
+                e = launch_slot_csr(pk, cand, kHierTpt, 0, ps.rows(), counts, cursor, toffs,
+                                    recs, err, st);
+            if (e == cudaSuccess)
+                e = launch_fine_scores(ps, q, k, recs, toffs + (int64_t)ps.G * ps.NB, fine, kc,
+                                       st);
+            if (e == cudaSuccess)
+                e = launch_select_among(ps, cand, fine, kc, block_ids + row0 * s.G * s.topk, st);
+        }
+    }
     return cuda_status(e);
 }

@@ -27,6 +27,27 @@ struct Shape {
 //   word[3]: number of sequences a paged call skipped (bad length or page id)
 constexpr size_t kErrorBytes = 256;
 
+// Checked build (compiled with -DMSA_CHECKED=1 into libmsa_checked.so): every
+// global-memory index that comes from data -- block ids, CSR tile records,
+// page tables, per-sequence lengths -- is tested against the extent of its
+// buffer before the access; a failed test skips the access and counts in a
+// device counter (msa_bounds_failures), and nothing traps.  The normal build
+// compiles the tests away.
+#ifndef MSA_CHECKED
+#define MSA_CHECKED 0
+#endif
+#if MSA_CHECKED
+extern __device__ unsigned int g_msa_bounds_failures;
+__device__ __forceinline__ bool in_bounds_checked(int64_t i, int64_t n) {
+    if (i >= 0 && i < n) return true;
+    atomicAdd(&g_msa_bounds_failures, 1u);
+    return false;
+}
+#define MSA_IN_BOUNDS(i, n) ::msa::in_bounds_checked((int64_t)(i), (int64_t)(n))
+#else
+#define MSA_IN_BOUNDS(i, n) true
+#endif
+
 __device__ __forceinline__ void record_error(uint32_t *err, uint32_t code, int counter) {
     if (err == nullptr) return;
     atomicCAS(err, 0u, code);
@@ -108,7 +129,25 @@ __host__ __device__ __forceinline__ int64_t partial_chunk(int64_t prow, int c, i
     return (prow >> 5) * (int64_t)(d / 8) * 32 + (int64_t)c * 32 + (prow & 31);
 }
 
-// Shapes the combine kernel handles: R divides 32, topk <= 64, topk * R <= 512.
+// Slot lists per (batch, group, block) -- a CSR built on the device -- for
+// query rows [r0, r0 + rc) of ids [B*T, G, s.topk] (s.topk <= 256): counts
+// and cursor [L = B*G*NB] (zeroed here), tile_offs [L + 1] (tile_offs[L] =
+// the number of tiles), and tile records of slot_csr_record_ints(tpt) ints:
+// {list, entries in the tile, 0, 0, entry[0 .. tpt)} with entry =
+// (row - r0) << 8 | slot.  Slots with bad or non-causal ids are skipped and
+// counted in the error word.  slot_csr_records bounds the records needed.
+cudaError_t launch_slot_csr(const Shape &s, const int32_t *ids, int tpt, int64_t r0, int64_t rc,
+                            int *counts, int *cursor, int *toffs, int *recs, uint32_t *err,
+                            cudaStream_t st);
+size_t slot_csr_records(const Shape &s, int64_t rc, int tpt);
+int slot_csr_record_ints(int tpt);
+
+// The indexer's KL target of query rows [r0, r0 + rc) from their partial
+// LSEs and merged lse (run after their merge).
+cudaError_t launch_block_mass(const Shape &s, const int32_t *ids, const float *part_lse,
+                              const float *lse, float *mass, int64_t r0, int64_t rc,
+                              cudaStream_t st, const int32_t *lens = nullptr);
+// Shapes the combine kernel handles: R divides 32, topk <= 256.
 bool combine_supported(const Shape &s);
 // LSE-weighted combine of per-(row, head, kept slot) partials into O and lse
 // for query rows [r0, r0 + rc) (d = 128).
@@ -130,6 +169,23 @@ cudaError_t launch_decode_attn(const Shape &s, const void *Q, const void *K, con
                                const KeyRows *rows = nullptr, const int32_t *lens = nullptr);
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st,
                         const int32_t *lens = nullptr);
+// Coarse-to-fine selection, last step: from candidates cand [rows, kc]
+// (ascending ids from launch_topk with topk = kc) and their exact block
+// scores fine [rows, kc], ids [rows, s.topk]: the current block and the
+// s.topk - 1 best candidates below it.  kc <= 64.
+cudaError_t launch_select_among(const Shape &s, const int32_t *cand, const float *fine, int kc,
+                                int32_t *ids, cudaStream_t st);
+// Coarse-to-fine selection (hier.cu): block-mean index keys kmean
+// [B, NB, d_idx] fp32; coarse scores cs [T*G, NB] of ONE sequence (B = 1;
+// only n < cb(t) written); exact scores of the candidates listed by a slot
+// CSR (tpt = 128) into fine [T*G, kc].
+cudaError_t launch_coarse_keys(const Shape &s, const void *k_idx, float *kmean, cudaStream_t st);
+cudaError_t launch_coarse_scores(const Shape &s, const void *q_idx, const float *kmean,
+                                 float *cs, cudaStream_t st);
+bool fine_scores_supported(const Shape &s);
+cudaError_t launch_fine_scores(const Shape &s, const void *q_idx, const void *k_idx,
+                               const int *recs, const int *n_tiles, float *fine, int kc,
+                               cudaStream_t st);
 // Page-table check of a paged call: lens_ok[b] = lens[b] when s.T <= lens[b]
 // <= s.S and every page id the sequence uses lies in [0, rows.num_pages),
 // otherwise 0 (the sequence does no work) with MSA_ERR_BAD_PAGE_TABLE recorded.

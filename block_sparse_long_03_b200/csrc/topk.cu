@@ -21,7 +21,9 @@
 // ascending id order with ballots, so the output needs no sort; cb is
 // appended last (it is larger than every candidate) and unused slots get -1.
 // Rows of more than 2048 blocks are too long to stage per warp; their warp
-// streams the row from memory instead (topk_long_kernel).
+// streams the row from memory instead (topk_long_kernel), unless there are
+// too few rows to fill the GPU that way (decode), where a CTA of 256
+// threads takes each row (topk_cta_kernel).
 #include "msa_internal.cuh"
 
 namespace msa {
@@ -258,7 +260,9 @@ __device__ __forceinline__ float4 load4(const float *row, int n, int limit) {
                        n + 3 < limit ? __ldg(row + n + 3) : 0.f);
 }
 
-template <bool kVec>
+// kTop: keys each lane keeps in pass 1 (2, or 4 when M > 32, so that the
+// threshold of the M-th largest stays close to it and few candidates pass).
+template <bool kVec, int kTop>
 __global__ void __launch_bounds__(kLongWarps * 32)
 topk_long_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int64_t nrows, int T_,
                  int S, int G, int NB, int block, int topk, const int32_t *__restrict__ lens) {
@@ -290,7 +294,9 @@ topk_long_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int64_
     auto key_of = [&](float f, int n) -> uint32_t { return n < cb ? ordered_key(f) : 0u; };
 
     if (M <= 64) {
-        uint32_t b1 = 0u, b2 = 0u;
+        uint32_t bt[kTop];                          // this lane's largest keys, descending
+#pragma unroll
+        for (int q = 0; q < kTop; ++q) bt[q] = 0u;
         for (int c0 = lane; c0 < nchunk; c0 += 128) {
             float4 f[4];
 #pragma unroll
@@ -302,16 +308,18 @@ topk_long_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int64_
                                         key_of(f[u].z, n + 2), key_of(f[u].w, n + 3)};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    b2 = max(b2, min(k4[e], b1));
-                    b1 = max(b1, k4[e]);
+#pragma unroll
+                    for (int q = kTop - 1; q > 0; --q) bt[q] = max(bt[q], min(k4[e], bt[q - 1]));
+                    bt[0] = max(bt[0], k4[e]);
                 }
             }
         }
         uint32_t tau = 0u;
         for (int bit = 31; bit >= 16; --bit) {
             const uint32_t c = tau | (1u << bit);
-            const int cnt = __popc(__ballot_sync(0xffffffffu, b1 >= c)) +
-                            __popc(__ballot_sync(0xffffffffu, b2 >= c));
+            int cnt = 0;
+#pragma unroll
+            for (int q = 0; q < kTop; ++q) cnt += __popc(__ballot_sync(0xffffffffu, bt[q] >= c));
             if (cnt >= M) tau = c;
         }
         // candidates >= tau in ascending id order: lane l owns ids 4l .. 4l + 3
@@ -410,22 +418,262 @@ topk_long_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int64_
     if (lane == 0) out[M] = cb;
 }
 
-constexpr int kWarpRowMaxNB = 2048;       // beyond: topk_long_kernel
+constexpr int kWarpRowMaxNB = 2048;       // beyond: topk_long_kernel, or
+constexpr int kLongMinRows = 4096;        // topk_cta_kernel for fewer rows than this
+
+// Last step of the coarse-to-fine selection: row r's candidates cand[r, 0..kc)
+// (ascending block ids, the current block last, -1 padding) with their
+// exact block scores fine[r, 0..kc).  Keeps the current block and the
+// topk - 1 best candidates below it, by (score descending, id ascending),
+// written ascending and -1 padded.  One warp per row, through the same
+// ballot selection as the Top-k kernels (kc <= 64 candidates).
+constexpr int kSelWarps = 8;
+
+__global__ void __launch_bounds__(kSelWarps * 32)
+select_among_kernel(const int32_t *__restrict__ cand, const float *__restrict__ fine,
+                    int32_t *__restrict__ ids, int64_t nrows, int T_, int S, int G, int block,
+                    int kc, int topk) {
+    __shared__ uint32_t s_buf[kSelWarps][2 * kMaxCand];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t r = (int64_t)blockIdx.x * kSelWarps + warp;
+    if (r >= nrows) return;
+    uint32_t *ck = s_buf[warp], *ci = s_buf[warp] + kMaxCand;
+    const int t = (int)((r / G) % T_);
+    const int cb = (int)(((int64_t)S - T_ + t) / block);
+    const int M = topk - 1;
+    int32_t *out = ids + r * topk;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    int C = 0;
+    for (int c0 = 0; c0 < kc; c0 += 32) {
+        const int c = c0 + lane;
+        const int n = c < kc ? cand[r * kc + c] : -1;
+        const bool ok = n >= 0 && n < cb;
+        const unsigned fb = __ballot_sync(0xffffffffu, ok);
+        const int pos = C + __popc(fb & lt_mask);
+        if (ok) {
+            ck[pos] = ordered_key(fine[r * kc + c]);
+            ci[pos] = (uint32_t)n;
+        }
+        C += __popc(fb);
+    }
+    __syncwarp();
+    if (C <= M) {                     // every candidate is kept
+        for (int i = lane; i < topk; i += 32)
+            out[i] = i < C ? (int32_t)ci[i] : (i == C ? cb : -1);
+        return;
+    }
+    select_candidates(ck, ci, C, M, cb, out, lane);
+}
+
+// Few rows with many candidates (decode at the 1M context: too few rows to
+// fill the GPU one warp per row): one CTA of kCtaThreads
+// threads per row runs the same selection (the threshold filter first, the
+// radix select when it leaves more than 128 candidates), the histogram and the
+// ordered emission shared by its warps; leading bits shared by every
+// candidate need no radix pass.
+constexpr int kCtaThreads = 256;
+
+__global__ void __launch_bounds__(kCtaThreads)
+topk_cta_kernel(const float *__restrict__ bs, int32_t *__restrict__ ids, int T_, int S, int G,
+                int NB, int block, int topk, const int32_t *__restrict__ lens) {
+    extern __shared__ uint32_t sm[];
+    constexpr int kWarps = kCtaThreads / 32;
+    uint32_t *keys = sm;                          // [NB]
+    uint32_t *hist = keys + NB;                   // [256]
+    uint32_t *red = hist + 256;                   // [2 * kWarps] reductions / warp counts
+    int *sel = (int *)(red + 2 * kWarps);         // [3]: digit, gt_count, (spare)
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int64_t r = blockIdx.x;
+    const int t = (int)((r / G) % T_);
+    const int64_t p = seq_len(lens, (int)(r / G / T_), S) - T_ + t;
+    const int cb = (int)(p / block);
+    const int M = topk - 1;
+    int32_t *out = ids + r * topk;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    if (p < 0) {
+        for (int i = tid; i < topk; i += kCtaThreads) out[i] = -1;
+        return;
+    }
+    if (M == 0) {
+        if (tid == 0) out[0] = cb;
+        return;
+    }
+    if (cb <= M) {
+        for (int i = tid; i < topk; i += kCtaThreads) out[i] = (i <= cb) ? i : -1;
+        return;
+    }
+    const float *row = bs + r * NB;
+    uint32_t all_and = 0xffffffffu, all_or = 0u;
+    uint32_t b1 = 0u, b2 = 0u;                    // this thread's two largest keys (0: none)
+    for (int n = tid; n < cb; n += kCtaThreads) {
+        const uint32_t v = ordered_key(row[n]);
+        keys[n] = v;
+        all_and &= v;
+        all_or |= v;
+        b2 = max(b2, min(v, b1));
+        b1 = max(b1, v);
+    }
+    all_and = __reduce_and_sync(0xffffffffu, all_and);
+    all_or = __reduce_or_sync(0xffffffffu, all_or);
+    if (lane == 0) { red[warp] = all_and; red[kWarps + warp] = all_or; }
+    __syncthreads();
+    all_and = 0xffffffffu; all_or = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) { all_and &= red[w]; all_or |= red[kWarps + w]; }
+    if (M <= 64) {
+        // As in the warp kernel: a lower bound tau of the M-th largest key
+        // (the M-th largest of the threads' top-2 keys, on its top 16 bits),
+        // the candidates >= tau compacted in id order, and if at most 128,
+        // warp 0 selects among them.  Counts cross the warps through a
+        // double-buffered shared array (one barrier per step).
+        __shared__ int cnt[2][kWarps];
+        uint32_t tau = 0u;
+        for (int bit = 31, it = 0; bit >= 16; --bit, ++it) {
+            const uint32_t c = tau | (1u << bit);
+            const int n_ge = __popc(__ballot_sync(0xffffffffu, b1 >= c)) +
+                             __popc(__ballot_sync(0xffffffffu, b2 >= c));
+            if (lane == 0) cnt[it & 1][warp] = n_ge;
+            __syncthreads();
+            int total = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) total += cnt[it & 1][w];
+            if (total >= M) tau = c;
+        }
+        uint32_t *ck = hist, *ci = hist + kMaxCand;   // the radix path re-zeroes hist
+        int C = 0;
+        for (int base = 0, it = 0; base < cb; base += kCtaThreads, ++it) {
+            const int n = base + tid;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool f = n < cb && v >= tau;
+            const unsigned fb = __ballot_sync(0xffffffffu, f);
+            if (lane == 0) cnt[it & 1][warp] = __popc(fb);
+            __syncthreads();
+            int before = C, total = C;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                before += w < warp ? cnt[it & 1][w] : 0;
+                total += cnt[it & 1][w];
+            }
+            const int pos = before + __popc(fb & lt_mask);
+            if (f && pos < kMaxCand) {
+                ck[pos] = v;
+                ci[pos] = (uint32_t)n;
+            }
+            C = total;
+        }
+        __syncthreads();
+        if (C <= kMaxCand) {                      // C is the same in every thread
+            if (warp == 0) select_candidates(ck, ci, C, M, cb, out, lane);
+            return;
+        }
+        __syncthreads();                          // hist is reused below
+    }
+    const uint32_t diff = all_and ^ all_or;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t prefix = 0, mask = 0;
+    int first_shift = 24;
+    while (first_shift > 0 && first_shift > top) first_shift -= 8;
+    if (first_shift + 8 <= 31) {
+        mask = 0xffffffffu << (first_shift + 8);
+        prefix = all_and & mask;
+    }
+    int remaining = M;
+    for (int shift = first_shift; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += kCtaThreads) hist[i] = 0;
+        __syncthreads();
+        for (int base = 0; base < cb; base += kCtaThreads) {
+            const int n = base + tid;
+            const uint32_t v = n < cb ? keys[n] : 0u;
+            const bool in = n < cb && (v & mask) == prefix;
+            if (in) atomicAdd(&hist[(v >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t c[8], lane_sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { c[i] = hist[lane * 8 + i]; lane_sum += c[i]; }
+            uint32_t incl = lane_sum;
+#pragma unroll
+            for (int off = 1; off < 32; off *= 2) {
+                const uint32_t o = __shfl_down_sync(0xffffffffu, incl, off);
+                if (lane + off < 32) incl += o;
+            }
+            const uint32_t above = incl - lane_sum;
+            int found = -1;
+            uint32_t gt_count = 0;
+            if (above < (uint32_t)remaining && above + lane_sum >= (uint32_t)remaining) {
+                uint32_t acc = above;
+                for (int i = 7; i >= 0; --i) {
+                    if (acc + c[i] >= (uint32_t)remaining) { found = lane * 8 + i; gt_count = acc; break; }
+                    acc += c[i];
+                }
+            }
+            if (found >= 0) { sel[0] = found; sel[1] = (int)gt_count; }
+        }
+        __syncthreads();
+        prefix |= (uint32_t)sel[0] << shift;
+        mask |= 255u << shift;
+        remaining -= sel[1];
+        __syncthreads();                              // sel and hist are reused
+    }
+    // ordered emission: per chunk of kCtaThreads ids, ranks from the warps'
+    // ballot counts
+    int ties_seen = 0, written = 0;
+    for (int base = 0; base < cb; base += kCtaThreads) {
+        const int n = base + tid;
+        const uint32_t v = (n < cb) ? keys[n] : 0u;
+        const bool eq = (n < cb) && v == prefix;
+        const unsigned eq_b = __ballot_sync(0xffffffffu, eq);
+        if (lane == 0) red[warp] = __popc(eq_b);
+        __syncthreads();
+        int eq_before = ties_seen, eq_total = ties_seen;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            eq_before += w < warp ? (int)red[w] : 0;
+            eq_total += (int)red[w];
+        }
+        const int tie_rank = eq_before + __popc(eq_b & lt_mask);
+        const bool take = (n < cb) && (v > prefix || (eq && tie_rank < remaining));
+        const unsigned tk_b = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) red[kWarps + warp] = __popc(tk_b);
+        __syncthreads();
+        int tk_before = written, tk_total = written;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            tk_before += w < warp ? (int)red[kWarps + w] : 0;
+            tk_total += (int)red[kWarps + w];
+        }
+        const int pos = tk_before + __popc(tk_b & lt_mask);
+        if (take && pos < M) out[pos] = n;
+        ties_seen = eq_total;
+        written = tk_total;
+        __syncthreads();                              // red is reused
+    }
+    if (tid == 0) out[M] = cb;
+}
 
 }  // namespace
 
 cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStream_t st,
                         const int32_t *lens) {
     const int64_t nrows = s.index_rows();
+    if (s.NB > kWarpRowMaxNB && nrows < kLongMinRows) {
+        const size_t smem = sizeof(uint32_t) * ((size_t)s.NB + 256 + 2 * (kCtaThreads / 32) + 4);
+        if (smem > 220 * 1024) return cudaErrorInvalidConfiguration;
+        cudaFuncSetAttribute(topk_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        topk_cta_kernel<<<(unsigned)nrows, kCtaThreads, smem, st>>>(bs, ids, s.T, s.S, s.G, s.NB,
+                                                                     s.block, s.topk, lens);
+        count_launches(1);
+        return cudaGetLastError();
+    }
     if (s.NB > kWarpRowMaxNB) {
         const unsigned grid = (unsigned)((nrows + kLongWarps - 1) / kLongWarps);
-        if ((s.NB & 3) == 0 && ((uintptr_t)bs & 15) == 0)
-            topk_long_kernel<true><<<grid, kLongWarps * 32, 0, st>>>(bs, ids, nrows, s.T, s.S, s.G,
-                                                                     s.NB, s.block, s.topk, lens);
-        else
-            topk_long_kernel<false><<<grid, kLongWarps * 32, 0, st>>>(bs, ids, nrows, s.T, s.S,
-                                                                      s.G, s.NB, s.block, s.topk,
-                                                                      lens);
+        const bool vec = (s.NB & 3) == 0 && ((uintptr_t)bs & 15) == 0, wide = s.topk - 1 > 32;
+        auto k = vec ? (wide ? topk_long_kernel<true, 4> : topk_long_kernel<true, 2>)
+                     : (wide ? topk_long_kernel<false, 4> : topk_long_kernel<false, 2>);
+        k<<<grid, kLongWarps * 32, 0, st>>>(bs, ids, nrows, s.T, s.S, s.G, s.NB, s.block, s.topk,
+                                            lens);
         count_launches(1);
         return cudaGetLastError();
     }
@@ -438,6 +686,16 @@ cudaError_t launch_topk(const Shape &s, const float *bs, int32_t *ids, cudaStrea
     const int64_t grid = (nrows + warps - 1) / warps;
     topk_kernel<<<(unsigned)grid, warps * 32, smem, st>>>(bs, ids, nrows, s.T, s.S, s.G, s.NB,
                                                           s.block, s.topk, warps, lens);
+    count_launches(1);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_among(const Shape &s, const int32_t *cand, const float *fine, int kc,
+                                int32_t *ids, cudaStream_t st) {
+    if (kc > 2 * 32 || kc < s.topk) return cudaErrorInvalidValue;
+    const int64_t nrows = s.index_rows();
+    select_among_kernel<<<(unsigned)((nrows + kSelWarps - 1) / kSelWarps), kSelWarps * 32, 0, st>>>(
+        cand, fine, ids, nrows, s.T, s.S, s.G, s.block, kc, s.topk);
     count_launches(1);
     return cudaGetLastError();
 }

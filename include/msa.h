@@ -122,8 +122,9 @@ MSA_EXPORT msa_status_t msa_topk_blocks(const msa_params_t *params, const float 
 /* Workspace needs, in bytes, of msa_sparse_attn_fwd (which = 0) and
  * msa_forward (which = 1) for these shapes, the device buffer of
  * msa_forward_host (which = 2, MSA_WS_FORWARD_HOST, defined with that call)
- * or the workspace of msa_decode_paged (which = 3, MSA_WS_DECODE_PAGED);
- * 0 for invalid shapes or shapes the call does not support. */
+ * the workspace of msa_decode_paged (which = 3, MSA_WS_DECODE_PAGED) or of
+ * msa_index_hierarchical (which = 4, MSA_WS_INDEX_HIER); 0 for invalid
+ * shapes or shapes the call does not support. */
 #define MSA_WS_SPARSE_ATTN 0
 #define MSA_WS_FORWARD 1
 MSA_EXPORT size_t msa_workspace_size(const msa_params_t *params, int which);
@@ -303,6 +304,42 @@ MSA_EXPORT msa_status_t msa_forward_host(const msa_params_t *params, const void 
                                          void *stream);
 
 /*
+ * Coarse-to-fine block selection: an index-cost reducer that replaces
+ * msa_index_block_scores + msa_topk_blocks ("LongCat Sparse Attention",
+ * Abstract, item (3): hierarchical indexing narrows each query's candidate
+ * set by coarse-to-fine scoring; applied here to the max-pooled block scores
+ * of "MiniMax Sparse Attention", Summary, second paragraph).  The page gives
+ * no formula; this call computes, per (b, t, g):
+ *   1. coarse score of each block n < cb(t): q_idx[b, t, g, :] . kmean[n],
+ *      kmean[n] the mean of block n's index keys (d_idx multiply-adds per
+ *      block instead of block * d_idx);
+ *   2. candidates: the kc - 1 best blocks n < cb(t) by coarse score (larger
+ *      first, lower id on ties);
+ *   3. the exact block score (as msa_index_block_scores) of each candidate;
+ *      kept = {cb(t)} plus the topk - 1 best candidates by that score, same
+ *      order; min(topk, cb(t) + 1) ids ascending, -1 padded.
+ * With kc - 1 >= cb(t) every earlier block is a candidate and the row's ids
+ * equal msa_topk_blocks' on msa_index_block_scores' scores.  The result is
+ * an approximation of that selection otherwise; its recall depends on how
+ * well block means rank blocks.  Feed the ids to msa_sparse_attn_fwd (for
+ * this layer, or for following layers that reuse them).
+ *
+ * kc: candidates per (query, group), current block included: topk <= kc
+ *     <= 64 (otherwise MSA_ERR_INVALID_ARG / MSA_ERR_UNSUPPORTED).
+ * bf16 only, d_idx in {64, 128} (otherwise MSA_ERR_UNSUPPORTED).
+ * q_idx [B, T, G, d_idx], k_idx [B, S, d_idx] (read); block_ids
+ * [B, T, G, topk] int32 (written).  workspace: at least
+ * msa_workspace_size(params, MSA_WS_INDEX_HIER) bytes (enough for any kc),
+ * 256-byte aligned; its first 256 bytes are the device error word.  Long
+ * prefills are processed in the query pieces msa_forward scores in.
+ */
+#define MSA_WS_INDEX_HIER 4
+MSA_EXPORT msa_status_t msa_index_hierarchical(const msa_params_t *params, int32_t kc,
+                                               const void *q_idx, const void *k_idx,
+                                               int32_t *block_ids, void *workspace,
+                                               size_t workspace_bytes, void *stream);
+
+/*
  * Decode steps over a PAGED KV cache with per-sequence lengths: the forward
  * pass of msa_forward (index scores, per-group Top-k with the current block
  * kept, sparse attention with LSE) for a batch of sequences of different
@@ -385,6 +422,17 @@ MSA_EXPORT msa_status_t msa_selftest_wait_timeout(void *workspace, size_t worksp
  * the kernels a region of work issued.
  */
 MSA_EXPORT uint64_t msa_kernel_launches(void);
+
+/*
+ * Diagnostics: the number of device bounds checks that failed since the
+ * library was loaded, in the checked build (libmsa_checked.so, compiled with
+ * MSA_CHECKED=1: every global-memory index derived from data -- block ids,
+ * the attention's tile records, page tables, sequence lengths -- is tested
+ * against its buffer's extent; a failed test skips the access and counts
+ * here, nothing traps).  Always 0 in the normal build, which has no checks.
+ * Synchronises the device; 0xffffffff if the counter cannot be read.
+ */
+MSA_EXPORT uint32_t msa_bounds_failures(void);
 
 #ifdef __cplusplus
 }

@@ -36,5 +36,17 @@ def pytest_sessionstart(session):
     lib_build = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(lib_build)
     lib_build.build()
+    if os.environ.get("MSA_LIBRARY") == "checked":
+        lib_build.build(checked=True)
     import oracle
     oracle.build()
+
+
+@pytest.fixture(autouse=True)
+def _no_failed_bounds_checks(request):
+    """Under the checked build (MSA_LIBRARY=checked) every GPU test must end
+    with no failed device bounds check."""
+    yield
+    if os.environ.get("MSA_LIBRARY") == "checked" and "gpu" in request.keywords:
+        from block_sparse_long_03_b200 import binding
+        assert binding.lib.msa_bounds_failures() == 0, "a device bounds check failed"

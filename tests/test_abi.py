@@ -179,3 +179,22 @@ def test_decode_paged_rejected_on_host():
     wide = _p(B=4, T=8, S=4096, Hq=32, Hkv=8, block=64, topk=8)   # T * G = 64 > 32
     assert call(wide) == 2
     assert call(_p(T=0)) == 1
+
+
+def test_bf16_without_tensor_core_path_is_unsupported():
+    """A bf16 group size with no tensor-core path (R = 3) is rejected on the
+    host instead of running on CUDA cores; fp32 of the same shape is served."""
+    import torch
+    from block_sparse_long_03_b200 import binding
+    lib = binding.lib
+    fake = ctypes.c_void_p(0x10000)
+    ws = ctypes.c_void_p(0x20000)
+    p = _p(Hq=6, Hkv=2)
+    assert binding.msa_workspace_size(p, binding.MSA_WS_SPARSE_ATTN) == 0
+    assert binding.msa_workspace_size(p, binding.MSA_WS_FORWARD) == 0
+    assert lib.msa_sparse_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, ws,
+                                   1 << 30, None) == 2
+    assert lib.msa_forward(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, ws,
+                           1 << 30, None) == 2
+    p32 = _p(Hq=6, Hkv=2, dtype=torch.float32)
+    assert binding.msa_workspace_size(p32, binding.MSA_WS_FORWARD) > 0

@@ -15,7 +15,8 @@ pytestmark = pytest.mark.gpu
 
 CASES = ["tiny_fp32_prefill", "fp32_gqa8", "bf16_prefill_2x1024", "bf16_chunk_ragged",
          "bf16_prefill_R16", "bf16_prefill_odd_blocks", "bf16_prefill_B2_chunk",
-         "bf16_decode_small", "bf16_decode_T4", "bf16_decode_topk64", "bf16_decode_R16"]
+         "bf16_decode_small", "bf16_decode_T4", "bf16_decode_topk64", "bf16_decode_R16",
+         "bf16_prefill_topk128", "bf16_decode_topk128", "bf16_d64_R8", "bf16_prefill_R16_topk64"]
 
 
 def _msa():

@@ -65,6 +65,19 @@ def _case(name):
         # more than 2048 candidate blocks per row: the CTA-per-row Top-k
         "bf16_chunk_many_blocks": W("bf16_chunk_many_blocks", B=1, T=64, S=139264, Hq=8, Hkv=2,
                                     d=128, d_idx=64, block=64, topk=9, dtype=bf),
+        # more than 64 kept blocks (batched merge), 16 heads per group with 64
+        # kept blocks, head dimension 64 on the tensor-core path (TMA Q boxes
+        # and the cp.async Q gather), and T = 1 with d = 64 (tensor-core path)
+        "bf16_prefill_topk128": W("bf16_prefill_topk128", B=1, T=512, S=16384, Hq=16, Hkv=2,
+                                  d=128, d_idx=64, block=64, topk=128, dtype=bf),
+        "bf16_prefill_R16_topk64": W("bf16_prefill_R16_topk64", B=1, T=384, S=8192, Hq=32,
+                                     Hkv=2, d=128, d_idx=64, block=64, topk=64, dtype=bf),
+        "bf16_decode_topk128": W("bf16_decode_topk128", B=2, T=1, S=16384, Hq=16, Hkv=4, d=128,
+                                 d_idx=64, block=64, topk=128, dtype=bf),
+        "bf16_d64_R8": W("bf16_d64_R8", B=1, T=768, S=1024, Hq=16, Hkv=2, d=64, d_idx=64,
+                         block=128, topk=4, dtype=bf, hot_blocks_per_group=1),
+        "bf16_decode_d64": W("bf16_decode_d64", B=4, T=1, S=2048, Hq=8, Hkv=2, d=64, d_idx=64,
+                             block=64, topk=8, dtype=bf),
     }
     return cases[name]
 
@@ -73,7 +86,8 @@ CASES = ["tiny_fp32_prefill", "bf16_prefill_2x1024", "bf16_chunk_ragged", "bf16_
          "bf16_d64_mha", "bf16_dense_limit", "bf16_topk1", "fp32_gqa8", "bf16_prefill_R16",
          "bf16_prefill_R1_didx128", "bf16_prefill_B2_chunk", "bf16_decode_block128",
          "bf16_decode_T4", "bf16_decode_topk64", "bf16_prefill_odd_blocks",
-         "bf16_chunk_many_blocks", "bf16_decode_R16"]
+         "bf16_chunk_many_blocks", "bf16_decode_R16", "bf16_prefill_topk128",
+         "bf16_prefill_R16_topk64", "bf16_decode_topk128", "bf16_d64_R8", "bf16_decode_d64"]
 
 
 def _inputs(w, seed=0):
