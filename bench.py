@@ -366,6 +366,41 @@ def index_reducers(prob, args, ws: int, kc: int) -> dict:
             "recall_rows": "4096 sampled rows with every slot filled (t >= block * k)"}
 
 
+def paged_decode(prob, args, ws: int, page_size: int = 64) -> dict:
+    """The same decode batch through msa_decode_paged: the cache is a pool of
+    pages (the dense cache cut into page_size-token pages) reached through a
+    random page table, with sequence lengths drawn uniformly from [S/2, S]
+    (ragged, most not a multiple of the block).  Bytes per step count the
+    index keys and kept K/V rows of each sequence's own length."""
+    m, i, w = prob.msa, prob.inp, prob.w
+    g = torch.Generator(device="cuda").manual_seed(11)
+    n_pages = w.B * w.S // page_size
+    table = torch.randperm(n_pages, generator=g, device="cuda").to(torch.int32).view(w.B, -1)
+    lens = torch.randint(w.S // 2, w.S + 1, (w.B,), generator=g, device="cuda").to(torch.int32)
+    kc = i.k_idx.view(n_pages, page_size, w.d_idx)
+    Kc = i.K.view(n_pages, page_size, w.Hkv, w.d)
+    Vc = i.V.view(n_pages, page_size, w.Hkv, w.d)
+    pws = m.alloc_workspace(prob.params, m.MSA_WS_DECODE_PAGED)
+
+    def step():
+        m.msa_decode_paged(prob.params, lens, table, page_size, n_pages, i.q_idx, kc, i.Q, Kc, Vc,
+                           prob.ids, prob.O, prob.lse, pws)
+
+    us = time_steps(step, max(args.steps, 10), args.warmup, ws) * 1e3
+    L = lens.long().cpu()
+    e = 2
+    kept_keys = 0
+    for Lb in L.tolist():                            # per sequence: the forced block is partial
+        cb = (Lb - 1) // w.block
+        kept_keys += (min(w.topk, cb + 1) - 1) * w.block + (Lb - 1 - cb * w.block + 1)
+    nbytes = (int(L.sum()) * w.d_idx * e + w.G * kept_keys * w.d * e * 2 +
+              w.B * (w.G * w.d_idx * e + 2 * w.Hq * w.d * e + w.Hq * 4))
+    del pws
+    return {"page_size": page_size, "lengths": f"uniform in [{w.S // 2}, {w.S}]",
+            "us_per_step": us, "bytes_per_step": float(nbytes),
+            "frac": nbytes / (us / 1e6) / 1e9 / peaks()["hbm_gbs"]}
+
+
 def time_steps(fn, steps: int, warmup: int, ws: int):
     for _ in range(warmup):
         fn()
@@ -561,7 +596,7 @@ def run_ours(args, rank: int, ws: int):
         decode = {"workload": args.decode_workload, "us_per_step": dms * 1e3, "bytes_per_step": db,
                   "achieved_gbs": db / (dms / 1e3) / 1e9, "peak_gbs": pk["hbm_gbs"],
                   "frac": db / (dms / 1e3) / 1e9 / pk["hbm_gbs"], "stage_ms": dst,
-                  "clocks": dclk.summary()}
+                  "clocks": dclk.summary(), "paged": paged_decode(dp, args, ws)}
         dp.free()
 
     # the pages' own 1M-token shape (prefill, and decode steps of 16 sequences)

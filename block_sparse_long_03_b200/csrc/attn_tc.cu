@@ -796,25 +796,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (!tc::mbar_wait(&s_full[bsel], (i / kQBuf) & 1, a.err, abort_flag)) break;
             tc::tc_fence_after();
             const bool masked = valid && (j_base + BLOCK - 1 > p);
-            // S is read from TMEM twice, 64 columns at a time (a TMEM read is
-            // cheap; holding a whole 128-column row would cost 64 registers).
-            // Causal mask (only in a token's own block): keys past the query
-            // position read as -inf.
+            // S is read from TMEM twice, 32 columns at a time, in rolled loops:
+            // the code every warp of the sub-partition runs stays small enough
+            // for its instruction cache (the unrolled passes were not; a TMEM
+            // read is cheap).  Causal mask (only in a token's own block): keys
+            // past the query position read as -inf.
             // Pass 1: row maximum.
             float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-            for (int h0 = 0; h0 < BLOCK; h0 += 64) {
-                uint32_t v[64];
-                tc::tmem_ld32(tS + h0, *(uint32_t(*)[32])(v));
-                tc::tmem_ld32(tS + h0 + 32, *(uint32_t(*)[32])(v + 32));
+#pragma unroll 1
+            for (int h0 = 0; h0 < BLOCK; h0 += 32) {
+                uint32_t v[32];
+                tc::tmem_ld32(tS + h0, v);
                 tc::tmem_ld_wait();
                 if (masked) {
+                    const int lim = p - (j_base + h0);     // columns above lim are not causal
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (j_base + h0 + c > p) v[c] = __float_as_uint(-INFINITY);
+                    for (int c = 0; c < 32; ++c)
+                        if (c > lim) v[c] = __float_as_uint(-INFINITY);
                 }
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) {
+                for (int c = 0; c < 32; c += 8) {
                     m0 = tc::fmax3(m0, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
                     m1 = tc::fmax3(m1, __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
                     m2 = tc::fmax3(m2, __uint_as_float(v[c + 4]), __uint_as_float(v[c + 5]));
@@ -828,19 +829,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // already read, with four partial row sums.  Rows past the tile's
             // tokens hold no query and are never stored.
             float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-            for (int h0 = 0; h0 < BLOCK; h0 += 64) {
-                uint32_t v[64];
-                tc::tmem_ld32(tS + h0, *(uint32_t(*)[32])(v));
-                tc::tmem_ld32(tS + h0 + 32, *(uint32_t(*)[32])(v + 32));
+#pragma unroll 1
+            for (int h0 = 0; h0 < BLOCK; h0 += 32) {
+                uint32_t v[32];
+                tc::tmem_ld32(tS + h0, v);
                 tc::tmem_ld_wait();
                 if (masked) {
+                    const int lim = p - (j_base + h0);
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (j_base + h0 + c > p) v[c] = __float_as_uint(-INFINITY);
+                    for (int c = 0; c < 32; ++c)
+                        if (c > lim) v[c] = __float_as_uint(-INFINITY);
                 }
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
+                for (int c = 0; c < 32; c += 4) {
                     const float e0 = tc::ex2_approx(fmaf(__uint_as_float(v[c]), a.scale_log2, -mb));
                     const float e1 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 1]), a.scale_log2, -mb));
                     const float e2 = tc::ex2_approx(fmaf(__uint_as_float(v[c + 2]), a.scale_log2, -mb));
@@ -848,10 +850,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     l0 += e0; l1 += e1; l2 += e2; l3 += e3;
                     __nv_bfloat162 b0 = __floats2bfloat162_rn(e0, e1);
                     __nv_bfloat162 b1 = __floats2bfloat162_rn(e2, e3);
-                    v[c / 2] = *(uint32_t *)&b0;
-                    v[c / 2 + 1] = *(uint32_t *)&b1;
+                    pk[c / 2] = *(uint32_t *)&b0;
+                    pk[c / 2 + 1] = *(uint32_t *)&b1;
                 }
-                tc::tmem_st32(tS + h0 / 2, *(const uint32_t(*)[32])(v));
+                tc::tmem_st16(tS + h0 / 2, pk);
             }
             const float l = (l0 + l1) + (l2 + l3);
             // the partial's row, m and l for the epilogue
