@@ -97,11 +97,11 @@ def partial_floor_bytes(w) -> float:
 # with the SHA-256 of the attention source: null once that source changes.
 MEASURED_TRAFFIC = {
     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-    "source_sha256": "3f1951c4f56767f4093babca7175a18ecb6b7d9168b0df45a0143b52fd0b61cd",
+    "source_sha256": "90249312842bdf6235f7995e3db464799c1c4674bafbea34a708773c56d3d3d8",
     "workload": "prefill_32k_h64",
     "slots": 8065 * 8 * 32,                       # kept (row, group) slots of the chunk
-    "kernels": {"attn_tc_kernel": {"read": 573004032.0, "write": 4238815744.0},
-                "combine_kernel": {"read": 4302819072.0, "write": 130824704.0}},
+    "kernels": {"attn_tc_kernel": {"read": 339964672.0, "write": 4236807424.0},
+                "combine_kernel": {"read": 4303569152.0, "write": 131194624.0}},
 }
 
 

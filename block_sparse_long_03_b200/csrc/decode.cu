@@ -136,10 +136,22 @@ decode_index_kernel(const __nv_bfloat16 *__restrict__ q_idx, const __nv_bfloat16
                 cp_async16(dst + swz(r, ch, kRowBytes), src + (int64_t)r * DIDX + ch * 8);
             }
         } else {
+            // one page-table lookup per key row (lane l: rows l and l + 32),
+            // handed to the lanes copying that row's chunks by a shuffle
+            static_assert(kSub == 64, "two key rows per lane");
+            const int64_t j0 = (int64_t)sb * kSub;
+            int64_t rw0, rw1;
+            if (rows.page_size % kSub == 0) {              // the sub-block lies in one page
+                const int64_t base = rows.row(b, j0);      // one lookup, the same in every lane
+                rw0 = j0 + lane < L && base >= 0 ? base + lane : -1;
+                rw1 = j0 + lane + 32 < L && base >= 0 ? base + lane + 32 : -1;
+            } else {
+                rw0 = j0 + lane < L ? rows.row(b, j0 + lane) : -1;
+                rw1 = j0 + lane + 32 < L ? rows.row(b, j0 + lane + 32) : -1;
+            }
             for (int c = lane; c < kSub * kChunks; c += 32) {
-                const int r = c / kChunks, ch = c % kChunks;
-                const int64_t j = (int64_t)sb * kSub + r;
-                const int64_t row = j < L ? rows.row(b, j) : -1;
+                const int r = c / kChunks, ch = c % kChunks;     // r < 32 is uniform per step
+                const int64_t row = __shfl_sync(0xffffffffu, r < 32 ? rw0 : rw1, r & 31);
                 if (row >= 0 && MSA_IN_BOUNDS(row, kv_rows))
                     cp_async16(dst + swz(r, ch, kRowBytes), k_idx + row * DIDX + ch * 8);
                 else
@@ -253,11 +265,28 @@ decode_block_kernel(const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__
 
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int g4 = lane / 4, t4 = lane % 4;
-    // stage K and V rows of the block (zero rows past the last causal key)
+    // stage K and V rows of the block (zero rows past the last causal key);
+    // a paged cache takes one page-table lookup per key row, shared through
+    // shared memory
+    int64_t *s_rows = nullptr;
+    int64_t page_base = -1;                            // a block inside one page: its first row
+    const bool one_page = kPaged && rows.page_size % BLOCK == 0;
+    if constexpr (kPaged) {
+        if (one_page) {
+            page_base = nk > 0 ? rows.row(b, j0) : -1;
+        } else {
+            __shared__ int64_t s_rows_buf[BLOCK];
+            for (int r = tid; r < BLOCK; r += kAttnThreads)
+                s_rows_buf[r] = r < nk ? rows.row(b, j0 + r) : -1;
+            __syncthreads();
+            s_rows = s_rows_buf;
+        }
+    }
     for (int c = tid; c < BLOCK * kChunks; c += kAttnThreads) {
         const int r = c / kChunks, ch = c % kChunks;
         const int64_t kr = r >= nk ? -1
-                           : kPaged ? rows.row(b, j0 + r) : (int64_t)b * S + j0 + r;
+                           : !kPaged ? (int64_t)b * S + j0 + r
+                           : one_page ? (page_base >= 0 ? page_base + r : -1) : s_rows[r];
         if (kr >= 0 && MSA_IN_BOUNDS(kr, kv_rows)) {
             const int64_t src = (kr * Hkv + g) * D + ch * 8;
             cp_async16(sK + swz(r, ch, kRowBytes), K + src);
