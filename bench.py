@@ -97,11 +97,11 @@ def partial_floor_bytes(w) -> float:
 # with the SHA-256 of the attention source: null once that source changes.
 MEASURED_TRAFFIC = {
     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-    "source_sha256": "90249312842bdf6235f7995e3db464799c1c4674bafbea34a708773c56d3d3d8",
+    "source_sha256": "ba7c86cc02d2706559a19e5df23538a4a2991d9f993b026257dd457b30f792a2",
     "workload": "prefill_32k_h64",
     "slots": 8065 * 8 * 32,                       # kept (row, group) slots of the chunk
-    "kernels": {"attn_tc_kernel": {"read": 339964672.0, "write": 4236807424.0},
-                "combine_kernel": {"read": 4303569152.0, "write": 131194624.0}},
+    "kernels": {"attn_tc_kernel": {"read": 318543616.0, "write": 4236307456.0},
+                "combine_kernel": {"read": 4302752512.0, "write": 130685952.0}},
 }
 
 

@@ -498,10 +498,10 @@ __device__ __forceinline__ int load_ent(const AttnArgs &a, int i, int total, int
 }
 
 // Warp roles (four warpgroups, 512 threads):
-//   warpgroup 0     warp 0 loads the K/V blocks and Q rows (TMA; for fewer
-//                   than 8 heads per token, warps 0 and 3 gather Q with
-//                   cp.async), warp 1 issues the S products, warp 2 the PV
-//                   products;
+//   warpgroup 0     warp 0 loads the K/V blocks, warps 0 and 3 the Q rows
+//                   (TMA boxes, half the tokens each; for fewer than 8 heads
+//                   per token, a cp.async gather), warp 1 issues the S
+//                   products, warp 2 the PV products;
 //   warpgroups 1-2  softmax, tiles 0, 2, 4, ... and 1, 3, 5, ...;
 //   warpgroup 3     epilogue of every tile: O from TMEM to a bf16 partial.
 // TMEM: three S/P buffers (S: BLOCK fp32 columns; P: bf16 pairs in the first
@@ -546,7 +546,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kQBuf; ++i) {
-            tc::mbar_init(&q_full[i], a.R >= 8 ? 1 : 64);   // TMA: one; cp.async: per thread
+            tc::mbar_init(&q_full[i], a.R >= 8 ? 2 : 64);   // TMA: one per warp; cp.async: per thread
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_full[i], 128);
             tc::mbar_init(&s_free[i], 128);        // epilogue threads, after PV
@@ -571,11 +571,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // Each role sets its warpgroup's register budget first.
     if (wg == 0) {
         tc::regs_dec<kRegsLoad>();
-        if (warp == 0 || (warp == 3 && a.R < 8)) {
+        if (warp == 0 || warp == 3) {
             // ------------------------------------------------ loads
             // K/V blocks by TMA (warp 0, lane 0) whenever the list changes, and
-            // the tile's Q rows gathered by warps 0 and 3 with 16-byte
-            // cp.async copies straight into the 128-byte-swizzled K-major
+            // the tile's Q rows by warps 0 and 3: TMA boxes for 8 or more heads
+            // per token, else 16-byte cp.async copies straight into the
+            // 128-byte-swizzled K-major
             // layout the MMA reads.  Each warp instruction copies kRPI whole
             // rows of D / 8 16-byte chunks (two rows for D = 128, four for
             // D = 64); lane l always copies chunk l % (D / 8).  A
@@ -638,14 +639,22 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (a.R >= 8) {
                     // 8 or more heads per token: the token's heads in groups of 8
                     // rows, one TMA box per group holding both 64-channel atoms
-                    // (or one box per atom); lane k < count holds token k's entry.
+                    // (or one box per atom).  Warps 0 and 3 take the first and
+                    // the second half of the tile's tokens: one thread issues a
+                    // box every ~100 cycles, so two issuing warps halve the
+                    // time a tile's Q takes to leave.  Lane k holds token k's
+                    // entry; a shuffle hands each lane its token's.
+                    const int half = (count + 1) / 2;
+                    const int t0 = warp == 0 ? 0 : half, nt = warp == 0 ? half : count - half;
+                    const int ent_t = __shfl_sync(0xffffffffu, e[0], min(t0 + lane, 31));
                     if (lane == 0)
-                        tc::mbar_expect_tx(&q_full[qb], (uint32_t)count * a.R * D * 2);
+                        tc::mbar_expect_tx(&q_full[qb], (uint32_t)nt * a.R * D * 2);
                     __syncwarp();
-                    if (lane < count) {
-                        const int grow = (int)(a.r0 + (e[0] >> 8));
+                    if (lane < nt) {
+                        const int grow = (int)(a.r0 + (ent_t >> 8));
                         for (int j = 0; j < a.R / 8; ++j) {
-                            uint8_t *grp8 = sQ + qb * kQBytes + (lane * (a.R / 8) + j) * kGroupBytes;
+                            uint8_t *grp8 =
+                                sQ + qb * kQBytes + ((t0 + lane) * (a.R / 8) + j) * kGroupBytes;
                             if (a.q_box4) {
                                 tc::tma_load_4d_hint(grp8, &tm_q, &q_full[qb], 0, g * a.R + j * 8, 0,
                                                      grow, q_pol);
