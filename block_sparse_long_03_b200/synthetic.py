@@ -83,6 +83,8 @@ WORKLOADS = {
                            block=128, topk=32, dtype=torch.bfloat16, hot_blocks_per_group=8),
     "decode_4x128k": Workload("decode_4x128k", B=4, T=1, S=131072, Hq=32, Hkv=8, d=128,
                               d_idx=64, block=64, topk=32, dtype=torch.bfloat16),
+    "decode_16x128k": Workload("decode_16x128k", B=16, T=1, S=131072, Hq=32, Hkv=8, d=128,
+                               d_idx=64, block=64, topk=32, dtype=torch.bfloat16),
     # The 128K prefill's heads, group size and k at 32K tokens: four row
     # chunks of the same size as the 128K call's, Q still larger than L2.
     "prefill_32k_h64": Workload("prefill_32k_h64", B=1, T=32768, S=32768, Hq=64, Hkv=8, d=128,
