@@ -32,7 +32,7 @@ EXPORTS = ("msa_status_string", "msa_index_block_scores", "msa_topk_blocks",
            "msa_kernel_launches", "msa_forward_noalloc", "msa_forward_host",
            "msa_selftest_wait_timeout", "msa_sparse_attn_fwd_mass", "msa_forward_mass",
            "msa_query_pieces", "msa_decode_paged", "msa_index_hierarchical",
-           "msa_bounds_failures")
+           "msa_bounds_failures", "msa_profile_begin", "msa_profile_end")
 
 
 class MsaError(RuntimeError):
@@ -85,6 +85,10 @@ def _load():
     lib.msa_kernel_launches.restype = ctypes.c_uint64
     lib.msa_bounds_failures.argtypes = []
     lib.msa_bounds_failures.restype = ctypes.c_uint32
+    lib.msa_profile_begin.argtypes = []
+    lib.msa_profile_begin.restype = st
+    lib.msa_profile_end.argtypes = [vp, vp, vp, vp]
+    lib.msa_profile_end.restype = st
     for name in ("msa_index_block_scores", "msa_topk_blocks", "msa_sparse_attn_fwd",
                  "msa_forward", "msa_get_device_error"):
         getattr(lib, name).restype = st
@@ -241,6 +245,21 @@ def msa_query_pieces(params: Params, which: int) -> list:
 def msa_kernel_launches() -> int:
     """Kernels the library has launched in this process so far."""
     return int(lib.msa_kernel_launches())
+
+
+def msa_profile_begin():
+    _check(lib.msa_profile_begin(), "msa_profile_begin")
+
+
+def msa_profile_end() -> dict:
+    """Summed device time (ms) and launch counts of the tensor-core attention
+    and merge kernels launched since msa_profile_begin."""
+    am, mm = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    an, mn = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib.msa_profile_end(ctypes.byref(am), ctypes.byref(an), ctypes.byref(mm),
+                               ctypes.byref(mn)), "msa_profile_end")
+    return {"attn_ms": am.value, "attn_launches": an.value, "merge_ms": mm.value,
+            "merge_launches": mn.value}
 
 
 # ---- convenience wrappers that allocate outputs with torch ----------------

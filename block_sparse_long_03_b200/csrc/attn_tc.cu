@@ -1132,9 +1132,13 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
         a.q_box4 = q_box4;
         a.scale = s.scale;
         a.scale_log2 = s.scale * kLog2e;
+        if ((e = prof_mark(st, kProfAttn, false)) != cudaSuccess) return e;
         kern<<<sms, kThreads, smem, st>>>(tq, tk, tv, a);
+        if ((e = prof_mark(st, kProfAttn, true)) != cudaSuccess) return e;
+        if ((e = prof_mark(st, kProfMerge, false)) != cudaSuccess) return e;
         e = launch_combine(s, ids, part_o, part_lse, O, lse, r0, rc, st, mass);
         if (e != cudaSuccess) return e;
+        if ((e = prof_mark(st, kProfMerge, true)) != cudaSuccess) return e;
         count_launches(5);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;

@@ -5,6 +5,8 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
+#include <utility>
 #include <vector>
 
 #include "msa_internal.cuh"
@@ -17,6 +19,81 @@ __device__ unsigned int g_msa_bounds_failures = 0;
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// Per-launch timing (msa_profile_begin/end): event pairs per kind, recorded
+// on the launching stream, summed and released at the end.
+struct ProfState {
+    std::mutex mu;
+    std::atomic<bool> on{false};
+    cudaEvent_t open[2] = {nullptr, nullptr};
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> done[2];
+};
+static ProfState g_prof;
+
+static void prof_release_locked() {
+    for (int k = 0; k < 2; ++k) {
+        for (auto &pr : g_prof.done[k]) {
+            cudaEventDestroy(pr.first);
+            cudaEventDestroy(pr.second);
+        }
+        g_prof.done[k].clear();
+        if (g_prof.open[k]) cudaEventDestroy(g_prof.open[k]);
+        g_prof.open[k] = nullptr;
+    }
+}
+
+cudaError_t prof_mark(cudaStream_t st, int kind, bool end) {
+    if (!g_prof.on.load(std::memory_order_acquire)) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    if (!g_prof.on.load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaEvent_t ev;
+    cudaError_t e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ev, st)) != cudaSuccess) {
+        cudaEventDestroy(ev);
+        return e;
+    }
+    if (!end) {
+        if (g_prof.open[kind]) cudaEventDestroy(g_prof.open[kind]);
+        g_prof.open[kind] = ev;
+    } else if (g_prof.open[kind]) {
+        g_prof.done[kind].push_back({g_prof.open[kind], ev});
+        g_prof.open[kind] = nullptr;
+    } else {
+        cudaEventDestroy(ev);
+    }
+    return cudaSuccess;
+}
+
+cudaError_t prof_begin() {
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    prof_release_locked();
+    g_prof.on.store(true, std::memory_order_release);
+    return cudaSuccess;
+}
+
+cudaError_t prof_end(double ms[2], int64_t n[2]) {
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    g_prof.on.store(false, std::memory_order_release);
+    cudaError_t first = cudaSuccess;
+    for (int k = 0; k < 2; ++k) {
+        ms[k] = 0.0;
+        n[k] = 0;
+        for (auto &pr : g_prof.done[k]) {
+            float t = 0.f;
+            cudaError_t e = cudaEventSynchronize(pr.second);
+            if (e == cudaSuccess) e = cudaEventElapsedTime(&t, pr.first, pr.second);
+            if (e != cudaSuccess) {
+                if (first == cudaSuccess) first = e;
+                continue;
+            }
+            ms[k] += t;
+            ++n[k];
+        }
+    }
+    prof_release_locked();
+    return first;
+}
 
 namespace {
 
@@ -301,6 +378,20 @@ msa_status_t msa_forward_mass(const msa_params_t *params, const void *q_idx, con
 }
 
 uint64_t msa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+msa_status_t msa_profile_begin(void) { return msa::prof_begin() == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+msa_status_t msa_profile_end(double *attn_ms, int64_t *attn_launches, double *merge_ms,
+                             int64_t *merge_launches) {
+    double ms[2] = {0.0, 0.0};
+    int64_t n[2] = {0, 0};
+    const cudaError_t e = msa::prof_end(ms, n);
+    if (attn_ms) *attn_ms = ms[msa::kProfAttn];
+    if (attn_launches) *attn_launches = n[msa::kProfAttn];
+    if (merge_ms) *merge_ms = ms[msa::kProfMerge];
+    if (merge_launches) *merge_launches = n[msa::kProfMerge];
+    return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA;
+}
 
 uint32_t msa_bounds_failures(void) {
 #if MSA_CHECKED

@@ -99,6 +99,12 @@ __device__ __forceinline__ int64_t seq_len(const int32_t *lens, int b, int64_t S
 // Every kernel launch of the library is counted (msa_kernel_launches).
 void count_launches(int n);
 
+// Per-launch timing of the prefill attention (msa_profile_begin/end): an
+// event on `st` before (end = false) or after (end = true) a launch of kind
+// kProfAttn or kProfMerge; nothing while profiling is off.
+constexpr int kProfAttn = 0, kProfMerge = 1;
+cudaError_t prof_mark(cudaStream_t st, int kind, bool end);
+
 // Launchers (each returns a cudaError_t from the launch).
 cudaError_t launch_index_scores_simt(const Shape &s, const void *q_idx, const void *k_idx,
                                      float *bs, cudaStream_t st);

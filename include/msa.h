@@ -434,6 +434,23 @@ MSA_EXPORT uint64_t msa_kernel_launches(void);
  */
 MSA_EXPORT uint32_t msa_bounds_failures(void);
 
+/*
+ * Measurement: per-kernel device time of the prefill attention.  Between
+ * msa_profile_begin and msa_profile_end, every launch of the tensor-core
+ * attention kernel (the KV-block-outer tiles) and of the merge kernel that
+ * follows it is bracketed by two CUDA events recorded on the call's own
+ * stream; msa_profile_end waits for those events, returns the summed elapsed
+ * times (milliseconds) and launch counts, and releases the events.  Outputs
+ * are unchanged; the event records add no kernel.  This is the one piece of
+ * library state a caller switches (process-wide, guarded by a lock); calls
+ * on several threads while it is on all add to the same totals.  Any output
+ * pointer may be NULL.  Returns MSA_ERR_CUDA if an event call fails (the
+ * totals then cover the launches before the failure).
+ */
+MSA_EXPORT msa_status_t msa_profile_begin(void);
+MSA_EXPORT msa_status_t msa_profile_end(double *attn_ms, int64_t *attn_launches,
+                                        double *merge_ms, int64_t *merge_launches);
+
 #ifdef __cplusplus
 }
 #endif

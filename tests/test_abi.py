@@ -198,3 +198,13 @@ def test_bf16_without_tensor_core_path_is_unsupported():
                            1 << 30, None) == 2
     p32 = _p(Hq=6, Hkv=2, dtype=torch.float32)
     assert binding.msa_workspace_size(p32, binding.MSA_WS_FORWARD) > 0
+
+
+def test_profile_hook_without_launches():
+    """msa_profile_begin/end with nothing launched in between return zero
+    totals (no device is touched), and end without begin is harmless."""
+    from block_sparse_long_03_b200 import binding
+    binding.msa_profile_begin()
+    r = binding.msa_profile_end()
+    assert r == {"attn_ms": 0.0, "attn_launches": 0, "merge_ms": 0.0, "merge_launches": 0}
+    assert binding.msa_profile_end()["attn_launches"] == 0

@@ -106,3 +106,37 @@ def test_measured_traffic_guard(bench, monkeypatch):
     monkeypatch.setattr(bench, "MEASURED_TRAFFIC", dict(fake, source_sha256="0" * 64))
     assert bench.measured_traffic(w) is None
 
+
+
+def test_roofline_uses_the_kernels_own_time(bench, monkeypatch):
+    """The roofline names the attention kernel: selected flops over its own
+    event-timed launches per step; traffic per launch from the per-slot
+    capture; the whole call and the merge are reported beside it.  An
+    index-dominated shape falls back to whole calls."""
+    import hashlib
+    src = "block_sparse_long_03_b200/csrc/attn_tc.cu"
+    with open(os.path.join(ROOT, src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    fake = {"source": src, "source_sha256": sha, "workload": "prefill_32k_h64", "slots": 1000,
+            "kernels": {"attn_tc_kernel": {"read": 3000.0, "write": 5000.0},
+                        "combine_kernel": {"read": 6000.0, "write": 500.0}}}
+    monkeypatch.setattr(bench, "MEASURED_TRAFFIC", fake)
+    w = _workloads().WORKLOADS["prefill_128k"]
+    pk = {"bf16_tflops": 1600.0, "hbm_gbs": 6500.0, "source": "measured"}
+    stages = {"index_block_scores": 6.0, "topk_blocks": 1.5, "sparse_attn_fwd": 40.0}
+    prof = {"attn_ms": 5 * 22.0, "attn_launches": 5 * 17, "merge_ms": 5 * 15.0,
+            "merge_launches": 5 * 17}
+    fl = 1.7e13
+    r = bench.roofline(w, pk, stages, prof, 5, fl, 8.8e12)
+    assert r["kernel"] == "attn_tc_kernel" and r["launches_per_step"] == 17
+    assert abs(r["achieved"] - fl / 22e-3 / 1e12) < 1e-6 * r["achieved"]
+    assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
+    assert abs(r["call"]["tflops"] - fl / 40e-3 / 1e12) < 1e-6 * r["call"]["tflops"]
+    slots = bench.kept_slots(w)
+    assert abs(r["traffic"] - 8.0 * slots / 17) < 1e-3 * slots
+    assert abs(r["merge"]["bytes_per_step"] - 6.5 * slots) < 1e-3 * slots
+    assert r["call"]["traffic"] == bench.measured_traffic(w)["bytes"]
+    # index-dominated: whole calls, no per-kernel traffic
+    r2 = bench.roofline(w, pk, dict(stages, index_block_scores=50.0), prof, 5, fl, 8.8e12)
+    assert r2["kernel"] == "index_block_scores" and r2["traffic"] is None
+    assert abs(r2["achieved"] - 8.8e12 / 50e-3 / 1e12) < 1e-6 * r2["achieved"]
