@@ -24,7 +24,8 @@ __all__ = [
     "forward_with_mass", "index_block_scores", "make_params", "msa_forward", "msa_forward_host",
     "msa_forward_mass", "msa_query_pieces", "msa_sparse_attn_fwd_mass",
     "msa_get_device_error", "msa_index_block_scores", "msa_kernel_launches",
-    "msa_selftest_wait_timeout", "msa_sparse_attn_fwd",
+    "msa_selftest_wait_timeout", "msa_sparse_attn_fwd", "msa_profile_begin", "msa_profile_end",
+    "msa_bounds_failures",
     "msa_topk_blocks", "msa_workspace_size", "params_from", "sparse_attn_fwd", "status_string",
     "topk_blocks",
 ]

@@ -247,6 +247,11 @@ def msa_kernel_launches() -> int:
     return int(lib.msa_kernel_launches())
 
 
+def msa_bounds_failures() -> int:
+    """Failed device bounds checks since load (checked build; 0 otherwise)."""
+    return int(lib.msa_bounds_failures())
+
+
 def msa_profile_begin():
     _check(lib.msa_profile_begin(), "msa_profile_begin")
 

@@ -208,3 +208,11 @@ def test_profile_hook_without_launches():
     r = binding.msa_profile_end()
     assert r == {"attn_ms": 0.0, "attn_launches": 0, "merge_ms": 0.0, "merge_launches": 0}
     assert binding.msa_profile_end()["attn_launches"] == 0
+
+
+def test_package_names_resolve():
+    """Every name the package exports resolves to the binding (the library
+    loads without a device)."""
+    import block_sparse_long_03_b200 as msa
+    for name in msa.__all__:
+        assert getattr(msa, name) is not None, name
