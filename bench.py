@@ -97,11 +97,11 @@ def partial_floor_bytes(w) -> float:
 # with the SHA-256 of the attention source: null once that source changes.
 MEASURED_TRAFFIC = {
     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-    "source_sha256": "ba7c86cc02d2706559a19e5df23538a4a2991d9f993b026257dd457b30f792a2",
+    "source_sha256": "631d6a257b9b79b367d4c88116d10e69ff7260880cf0cac77c559b849594284d",
     "workload": "prefill_32k_h64",
     "slots": 8065 * 8 * 32,                       # kept (row, group) slots of the chunk
-    "kernels": {"attn_tc_kernel": {"read": 318543616.0, "write": 4236307456.0},
-                "combine_kernel": {"read": 4302752512.0, "write": 130685952.0}},
+    "kernels": {"attn_tc_kernel": {"read": 330041344.0, "write": 4236393216.0},
+                "combine_kernel": {"read": 4302755072.0, "write": 131347200.0}},
 }
 
 
@@ -119,8 +119,9 @@ def measured_traffic(w):
     rd = sum(k["read"] for k in m["kernels"].values()) / m["slots"] * slots
     wr = sum(k["write"] for k in m["kernels"].values()) / m["slots"] * slots
     per = {name: (k["read"] + k["write"]) / m["slots"] * slots for name, k in m["kernels"].items()}
+    per_w = {name: k["write"] / m["slots"] * slots for name, k in m["kernels"].items()}
     return {"bytes": rd + wr, "read_bytes": rd, "write_bytes": wr, "from": m["workload"],
-            "kernels": per}
+            "kernels": per, "kernel_writes": per_w}
 
 
 def decode_bytes(w) -> float:
@@ -543,7 +544,28 @@ def run_reference(args, rank: int, ws: int):
 NOMINAL_BF16_TFLOPS, NOMINAL_HBM_GBS = 2250.0, 8000.0
 
 
-def roofline(w, pk, stages, prof, steps, attn_fl, idx_fl) -> dict:
+def write_only_gbs(nbytes: int = 4 << 30, reps: int = 10) -> float:
+    """HBM bandwidth of a plain write-only stream on this GPU (torch fill of a
+    buffer larger than L2), measured with CUDA events: the reference for the
+    attention kernel, whose DRAM traffic is almost all partial-output writes."""
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        buf.fill_(1)
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(reps):
+        buf.fill_(1)
+    e1.record(s)
+    torch.cuda.synchronize()
+    gbs = nbytes / (e0.elapsed_time(e1) / reps / 1e3) / 1e9
+    del buf
+    torch.cuda.empty_cache()
+    return gbs
+
+
+def roofline(w, pk, stages, prof, steps, attn_fl, idx_fl, fill_gbs=None) -> dict:
     """The dominant kernel's roofline.  At the prefill shapes that is the
     tensor-core attention kernel: its selected flops per launch over its own
     launch time, measured live in the timed steps; the whole sparse-attention
@@ -589,6 +611,13 @@ def roofline(w, pk, stages, prof, steps, attn_fl, idx_fl) -> dict:
                   "bytes_per_step": float(merge_bytes),
                   "achieved_gbs": merge_bytes / (merge_ms / 1e3) / 1e9,
                   "frac_of_hbm": merge_bytes / (merge_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
+        # the kernel's DRAM traffic is almost all partial writes: their time at
+        # the write-only bandwidth measured in the same run is a second floor
+        "write_floor": None if (mt is None or not fill_gbs) else {
+            "bytes_per_step": mt["kernel_writes"]["attn_tc_kernel"],
+            "write_only_gbs": fill_gbs,
+            "ms": mt["kernel_writes"]["attn_tc_kernel"] / (fill_gbs * 1e9) * 1e3,
+            "frac": mt["kernel_writes"]["attn_tc_kernel"] / (fill_gbs * 1e9) * 1e3 / attn_ms},
         "stage_ms": stages,
         # the schedule's own floor: partials through HBM at the measured bandwidth
         "partial_traffic_floor": {
@@ -619,7 +648,7 @@ def run_ours(args, rank: int, ws: int):
     value = aggregate_tokens_per_s(w.B * w.T, ms, ws)
     stages = prob.stage_times_ms(max(2, args.steps))
     attn_fl, idx_fl = attention_flops(w), index_flops(w)
-    roof = roofline(w, pk, stages, prof, args.steps, attn_fl, idx_fl)
+    roof = roofline(w, pk, stages, prof, args.steps, attn_fl, idx_fl, write_only_gbs())
     # the indexer's KL target as a third output of the same pass
     kl_ms = time_steps(prob.step_mass, args.steps, args.warmup, ws)
     ref_ms = time_steps(prob.step, args.steps, args.warmup, ws)    # adjacent, same clocks

@@ -127,8 +127,12 @@ def test_roofline_uses_the_kernels_own_time(bench, monkeypatch):
     prof = {"attn_ms": 5 * 22.0, "attn_launches": 5 * 17, "merge_ms": 5 * 15.0,
             "merge_launches": 5 * 17}
     fl = 1.7e13
-    r = bench.roofline(w, pk, stages, prof, 5, fl, 8.8e12)
+    r = bench.roofline(w, pk, stages, prof, 5, fl, 8.8e12, fill_gbs=4000.0)
     assert r["kernel"] == "attn_tc_kernel" and r["launches_per_step"] == 17
+    wf = r["write_floor"]
+    assert abs(wf["bytes_per_step"] - 5.0 * bench.kept_slots(w)) < 1e-3 * bench.kept_slots(w)
+    assert abs(wf["ms"] - wf["bytes_per_step"] / 4e12 * 1e3) < 1e-9 * wf["ms"]
+    assert abs(wf["frac"] - wf["ms"] / 22.0) < 1e-12
     assert abs(r["achieved"] - fl / 22e-3 / 1e12) < 1e-6 * r["achieved"]
     assert abs(r["frac"] - r["achieved"] / 1600.0) < 1e-12
     assert abs(r["call"]["tflops"] - fl / 40e-3 / 1e12) < 1e-6 * r["call"]["tflops"]
