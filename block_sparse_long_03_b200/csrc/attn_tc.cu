@@ -244,8 +244,7 @@ namespace {
 // with the blocked chunk layout every load of the warp is 512 contiguous
 // bytes, and all loads of a warp are independent (issued together).
 // Needs R | 32 and kPer >= topk / 32; lanes take their slots in batches of
-// kMaxPer.  Run by combine_kernel, and by the spare
-// CTAs of the attention kernel for the previous row chunk.
+// kMaxPer.  Run by combine_kernel after each row chunk's attention kernel.
 struct CombineArgs {
     const int32_t *ids;
     const __nv_bfloat16 *part_o;
@@ -462,6 +461,104 @@ combine_kernel(CombineArgs c) {
     if (wid >= c.rc * c.G * combine_warps_per_row<D>()) return;
     if (kPer == 0) combine_unit<D, kMaxPer>(c, wid, threadIdx.x % 32);
     else combine_unit_batched<D, kMaxPer, (kPer > 0 ? kPer : 1)>(c, wid, threadIdx.x % 32);
+}
+
+// The merge in two passes, for R * d >= 256 (a warp's 32 lanes then cover
+// whole heads): pass 1 turns each (row, group)'s slot LSEs into normalised
+// weights w = exp(lse_i - lse) (0 for a slot no tile served), written over
+// the LSEs, and writes the row's final LSE; pass 2 streams the partials with
+// lanes = (head, 16-byte channel chunk), each lane summing w * O_i over the
+// slots for its own 8 output channels (no cross-lane reduction, no per-warp
+// LSE work).  Lanes of pass 1 are laid out as in the single-pass merge (head
+// l % R, slots l / R + k * 32 / R); kMaxPer (8 or 16) >= slots per lane.
+template <int kMaxPer>
+__global__ void __launch_bounds__(256) merge_weights_kernel(CombineArgs c, float *wts) {
+    const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (x >= c.rc * c.G) return;
+    const int64_t rl = x / c.G, r = c.r0 + rl;
+    const int g = (int)(x % c.G);
+    const int t = (int)(r % c.T_);
+    const int64_t p = seq_len(c.lens, (int)(r / c.T_), c.S) - c.T_ + t;
+    const int cb = p < 0 ? -1 : (int)(p / c.block);
+    const SlotPair sp = warp_slots2(c.ids + (r * c.G + g) * c.topk, c.topk, c.NB, cb, lane);
+    const int R = c.R, h = lane % R, s0 = lane / R, sstep = 32 / R;
+    const int per = (c.topk + sstep - 1) / sstep;        // slots per lane
+    const int64_t base = x * c.topk * R;
+    float li[kMaxPer], m = -INFINITY;                    // every load issued before any use
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        const int sl = s0 + k * sstep;
+        const bool okk = __shfl_sync(0xffffffffu, sl < 32 ? sp.ok0 : sp.ok1, sl & 31);
+        const bool ok = k < per && sl < c.topk && okk;
+        li[k] = ok ? c.part_lse[base + (int64_t)sl * R + h] : -INFINITY;
+        m = fmaxf(m, li[k]);
+    }
+    for (int off = R; off < 32; off *= 2) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    float lsum = 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        li[k] = li[k] == -INFINITY ? 0.f : expf(li[k] - m);
+        lsum += li[k];
+    }
+    for (int off = R; off < 32; off *= 2) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+    for (int k = 0; k < kMaxPer; ++k) {
+        const int sl = s0 + k * sstep;
+        if (k < per && sl < c.topk) wts[base + (int64_t)sl * R + h] = li[k] * inv;
+    }
+    if (s0 == 0) c.lse[r * c.Hq + (int64_t)g * R + h] = lsum > 0.f ? m + logf(lsum) : -INFINITY;
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(256) merge_apply_kernel(CombineArgs c, const float *wts) {
+    constexpr int C = 32 / R;                            // chunks per head in one warp
+    constexpr int W = D / 8 / C;                         // warps per (row, group)
+    static_assert(W >= 1, "the group's heads must fill a warp");
+    const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
+    const int lane = threadIdx.x % 32;
+    if (wid >= c.rc * c.G * W) return;
+    const int part = (int)(wid % W);
+    const int64_t x = wid / W;                           // (row in chunk, group)
+    const int64_t rl = x / c.G;
+    const int g = (int)(x % c.G);
+    const int h = lane / C, ch = part * C + lane % C;    // head, 16-byte channel chunk
+    const int64_t base = x * c.topk * R;
+    const uint4 *src = (const uint4 *)c.part_o;
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int s0 = 0; s0 < c.topk; s0 += 8) {
+        // a batch's weights, then its loads (a zero weight: no partial, no load)
+        float w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            w[k] = s0 + k < c.topk ? __ldg(wts + base + (int64_t)(s0 + k) * R + h) : 0.f;
+        uint4 u[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int64_t prow = base + (int64_t)(s0 + k) * R + h;
+            u[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (w[k] != 0.f && MSA_IN_BOUNDS(prow, c.rc * c.G * c.topk * R))
+                u[k] = src[partial_chunk(prow, ch, D)];
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const __nv_bfloat162 *hp = (const __nv_bfloat162 *)&u[k];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(hp[q]);
+                acc[2 * q] = fmaf(w[k], f.x, acc[2 * q]);
+                acc[2 * q + 1] = fmaf(w[k], f.y, acc[2 * q + 1]);
+            }
+        }
+    }
+    const int64_t r = c.r0 + rl;
+    __nv_bfloat162 o2[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) o2[q] = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    *(uint4 *)(c.O + (r * c.Hq + (int64_t)g * R + h) * D + ch * 8) = *(const uint4 *)o2;
 }
 
 struct AttnArgs {
@@ -935,14 +1032,15 @@ namespace {
 
 // The indexer's KL target for query rows [r0, r0 + rc), run after their
 // merge: slot sl's share of head h's softmax is exp(part_lse - lse) of that
-// slot (0 for slots no tile served), averaged over the group's R heads.  One
+// slot (0 for slots no tile served), averaged over the group's R heads; after
+// the two-pass merge (weights = true) part_lse already holds those shares.  One
 // warp per (row, group), lanes laid out as in the merge (head l % R, slots
 // l / R + k * 32 / R), so the head average is a shuffle over R lanes.
 __global__ void __launch_bounds__(256)
 block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ part_lse,
                   const float *__restrict__ lse, float *__restrict__ mass, int64_t r0, int64_t rc,
                   int T_, int S, int Hq, int G, int R, int NB, int block, int topk,
-                  const int32_t *__restrict__ lens) {
+                  const int32_t *__restrict__ lens, bool weights) {
     const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
@@ -969,7 +1067,8 @@ block_mass_kernel(const int32_t *__restrict__ ids, const float *__restrict__ par
     for (int k = 0; k < kMaxPer; ++k) {
         if (k >= per) break;                        // per is uniform across the warp
         const int sl = s0 + k * sstep;
-        float share = (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
+        float share = weights ? (li[k] == -INFINITY ? 0.f : li[k])
+                              : (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
         for (int off = 1; off < R; off *= 2) share += __shfl_xor_sync(0xffffffffu, share, off);
         if (h == 0 && sl < topk) mrow[sl] = share / (float)R;
     }
@@ -981,7 +1080,7 @@ __global__ void __launch_bounds__(256)
 block_mass_wide_kernel(const int32_t *__restrict__ ids, const float *__restrict__ part_lse,
                   const float *__restrict__ lse, float *__restrict__ mass, int64_t r0, int64_t rc,
                   int T_, int S, int Hq, int G, int R, int NB, int block, int topk,
-                  const int32_t *__restrict__ lens) {
+                  const int32_t *__restrict__ lens, bool weights) {
     const int64_t x = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
     const int lane = threadIdx.x % 32;
     if (x >= rc * G) return;
@@ -1009,7 +1108,8 @@ block_mass_wide_kernel(const int32_t *__restrict__ ids, const float *__restrict_
         for (int k = 0; k < kMaxPer; ++k) {
             if (k0 + k >= per) break;               // per is uniform across the warp
             const int sl = s0 + (k0 + k) * sstep;
-            float share = (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
+            float share = weights ? (li[k] == -INFINITY ? 0.f : li[k])
+                                  : (li[k] != -INFINITY && l != -INFINITY) ? expf(li[k] - l) : 0.f;
             for (int off = 1; off < R; off *= 2) share += __shfl_xor_sync(0xffffffffu, share, off);
             if (h == 0 && sl < topk) mrow[sl] = share / (float)R;
         }
@@ -1148,20 +1248,54 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 }  // namespace
 
+// The two-pass merge serves every group size whose heads fill whole warps.
+bool merge_two_pass(const Shape &s) { return s.R * s.d >= 256 && !combine_batched(s); }
+
+template <int D>
+cudaError_t launch_merge_apply(const Shape &s, const CombineArgs &ca, const float *wts,
+                               int64_t rc, cudaStream_t st) {
+    const int64_t warps = rc * s.G * (D / 8 / (32 / s.R));
+    const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
+    switch (s.R) {
+        case 2: if constexpr (D / 8 >= 16) merge_apply_kernel<D, 2><<<grid, 256, 0, st>>>(ca, wts); break;
+        case 4: if constexpr (D / 8 >= 8) merge_apply_kernel<D, 4><<<grid, 256, 0, st>>>(ca, wts); break;
+        case 8: merge_apply_kernel<D, 8><<<grid, 256, 0, st>>>(ca, wts); break;
+        case 16: merge_apply_kernel<D, 16><<<grid, 256, 0, st>>>(ca, wts); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_block_mass(const Shape &s, const int32_t *ids, const float *part_lse,
                               const float *lse, float *mass, int64_t r0, int64_t rc,
                               cudaStream_t st, const int32_t *lens) {
     const unsigned mgrid = (unsigned)((rc * s.G * 32 + 255) / 256);
     auto k = combine_batched(s) ? block_mass_wide_kernel : block_mass_kernel;
     k<<<mgrid, 256, 0, st>>>(ids, part_lse, lse, mass, r0, rc, s.T, s.S, s.Hq, s.G, s.R, s.NB,
-                             s.block, s.topk, lens);
+                             s.block, s.topk, lens, merge_two_pass(s));
     count_launches(1);
     return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
-                           const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
+                           float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st, float *mass, const int32_t *lens) {
+    if (merge_two_pass(s)) {
+        const CombineArgs ca = combine_args(s, ids, part_o, part_lse, O, lse, r0, rc, lens);
+        const unsigned g1 = (unsigned)((rc * s.G * 32 + 255) / 256);
+        if (combine_wide(s)) merge_weights_kernel<16><<<g1, 256, 0, st>>>(ca, part_lse);
+        else merge_weights_kernel<8><<<g1, 256, 0, st>>>(ca, part_lse);
+        const cudaError_t e = s.d == 64 ? launch_merge_apply<64>(s, ca, part_lse, rc, st)
+                                        : launch_merge_apply<128>(s, ca, part_lse, rc, st);
+        if (e != cudaSuccess) return e;
+        count_launches(2);
+        if (mass != nullptr) {
+            const cudaError_t e2 = cudaGetLastError();
+            if (e2 != cudaSuccess) return e2;
+            return launch_block_mass(s, ids, part_lse, lse, mass, r0, rc, st, lens);
+        }
+        return cudaGetLastError();
+    }
     const int64_t warps = rc * s.G * (s.d / 8 / kCombineChunksPerWarp);
     const unsigned grid = (unsigned)((warps * 32 + 255) / 256);
     // slots per merging lane: one batch of 8 or 16, or batches of 8 past 64 kept blocks

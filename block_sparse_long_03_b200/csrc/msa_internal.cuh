@@ -158,7 +158,7 @@ bool combine_supported(const Shape &s);
 // LSE-weighted combine of per-(row, head, kept slot) partials into O and lse
 // for query rows [r0, r0 + rc) (d = 128).
 cudaError_t launch_combine(const Shape &s, const int32_t *ids, const __nv_bfloat16 *part_o,
-                           const float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
+                           float *part_lse, void *O, float *lse, int64_t r0, int64_t rc,
                            cudaStream_t st, float *mass = nullptr,
                            const int32_t *lens = nullptr);
 // Decode path (few query tokens per sequence): HBM-streaming index scoring and
