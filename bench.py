@@ -83,25 +83,27 @@ def partial_floor_bytes(w) -> float:
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of the sparse
-# attention call's two main kernels, from a one-pass ncu capture of ONE row
+# attention call's main kernels, from a one-pass ncu capture of ONE row
 # chunk (the fourth of five: rows 24195..32259, 8065 rows like every full
 # chunk of the 128K call, every row keeping k blocks) of the workload
 # `prefill_32k_h64` (the 128K prefill's heads, group size and k at 32K tokens;
 # Q is larger than L2 as there):
 #   python bench.py --workload prefill_32k_h64 --attn-call-once
 # under ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,
-# dram__bytes_write.sum -k regex:"attn_tc_kernel|combine_kernel" -s 6 -c 2.
+# dram__bytes_write.sum -k regex:"attn_tc_kernel|merge_" -s 9 -c 3 (the
+# attention kernel and the merge's two passes of that chunk).
 # The figures are per kept (query, group) slot of the chunk; a call's traffic
-# is that times its kept slots (the partials, the Q gather and the combine's
+# is that times its kept slots (the partials, the Q gather and the merge's
 # reads all grow with the slots; K/V and the CSR kernels add < 1 %).  Held
 # with the SHA-256 of the attention source: null once that source changes.
 MEASURED_TRAFFIC = {
     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-    "source_sha256": "631d6a257b9b79b367d4c88116d10e69ff7260880cf0cac77c559b849594284d",
+    "source_sha256": "a15d5bea3824c7609ee5c1342bd6535d534e8e2050dab6144d6b492137eb3cfd",
     "workload": "prefill_32k_h64",
     "slots": 8065 * 8 * 32,                       # kept (row, group) slots of the chunk
-    "kernels": {"attn_tc_kernel": {"read": 330041344.0, "write": 4236393216.0},
-                "combine_kernel": {"read": 4302755072.0, "write": 131347200.0}},
+    "kernels": {"attn_tc_kernel": {"read": 314621696.0, "write": 4236021760.0},
+                "merge_weights_kernel": {"read": 74349312.0, "write": 6268928.0},
+                "merge_apply_kernel": {"read": 4294464768.0, "write": 127204096.0}},
 }
 
 
@@ -587,7 +589,7 @@ def roofline(w, pk, stages, prof, steps, attn_fl, idx_fl, fill_gbs=None) -> dict
     ach = attn_fl / (attn_ms / 1e3) / 1e12
     mt = measured_traffic(w)
     merge_ms = prof["merge_ms"] / steps
-    merge_bytes = (mt["kernels"]["combine_kernel"] if mt else
+    merge_bytes = (sum(v for k, v in mt["kernels"].items() if k != "attn_tc_kernel") if mt else
                    partial_floor_bytes(w) / 2)            # read back once, O written once
     call_tf = attn_fl / (call_ms / 1e3) / 1e12
     return {
@@ -607,7 +609,7 @@ def roofline(w, pk, stages, prof, steps, attn_fl, idx_fl, fill_gbs=None) -> dict
                  "frac": call_tf / pk["bf16_tflops"],
                  "frac_of_nominal": call_tf / NOMINAL_BF16_TFLOPS,
                  "traffic": None if mt is None else float(mt["bytes"])},
-        "merge": {"kernel": "combine_kernel", "ms_per_step": merge_ms,
+        "merge": {"kernels": "merge_weights_kernel + merge_apply_kernel", "ms_per_step": merge_ms,
                   "bytes_per_step": float(merge_bytes),
                   "achieved_gbs": merge_bytes / (merge_ms / 1e3) / 1e9,
                   "frac_of_hbm": merge_bytes / (merge_ms / 1e3) / 1e9 / pk["hbm_gbs"]},
