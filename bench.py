@@ -98,12 +98,12 @@ def partial_floor_bytes(w) -> float:
 # with the SHA-256 of the attention source: null once that source changes.
 MEASURED_TRAFFIC = {
     "source": "block_sparse_long_03_b200/csrc/attn_tc.cu",
-    "source_sha256": "a15d5bea3824c7609ee5c1342bd6535d534e8e2050dab6144d6b492137eb3cfd",
+    "source_sha256": "48e6c5e6d6552623caadd10f200e69635c6a3ce5357985d69407dff41f7e161f",
     "workload": "prefill_32k_h64",
     "slots": 8065 * 8 * 32,                       # kept (row, group) slots of the chunk
-    "kernels": {"attn_tc_kernel": {"read": 314621696.0, "write": 4236021760.0},
-                "merge_weights_kernel": {"read": 74349312.0, "write": 6268928.0},
-                "merge_apply_kernel": {"read": 4294464768.0, "write": 127204096.0}},
+    "kernels": {"attn_tc_kernel": {"read": 336722688.0, "write": 4236628480.0},
+                "merge_weights_kernel": {"read": 74349056.0, "write": 6138368.0},
+                "merge_apply_kernel": {"read": 4294501376.0, "write": 127399424.0}},
 }
 
 

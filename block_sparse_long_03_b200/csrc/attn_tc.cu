@@ -1248,8 +1248,14 @@ cudaError_t run_chunks(const Shape &s, const void *Q, const void *K, const void 
 
 }  // namespace
 
-// The two-pass merge serves every group size whose heads fill whole warps.
-bool merge_two_pass(const Shape &s) { return s.R * s.d >= 256 && !combine_batched(s); }
+// The two-pass merge serves prefill-shaped calls (64 or more queries per
+// sequence) whose group's heads fill whole warps; a decode step's few rows are
+// bound by launch latency, where one pass is faster.  The choice depends on
+// the call's shape only, never on how its rows are chunked, so a call split
+// into pieces gives the same bits as the whole call.
+bool merge_two_pass(const Shape &s) {
+    return s.R * s.d >= 256 && !combine_batched(s) && s.T >= 64;
+}
 
 template <int D>
 cudaError_t launch_merge_apply(const Shape &s, const CombineArgs &ca, const float *wts,
