@@ -17,6 +17,15 @@ max over ranks and `value` counts the tokens of all ranks.
 
 `--impl reference` times the fp64 CPU oracle on the host cores on a bounded
 row sample of the same workload (rank 0 only).
+
+`roofline` names the dominant kernel, the tensor-core attention kernel: its
+selected flops over its own launches, which the library brackets with CUDA
+events on the call's stream during the timed steps (msa_profile_begin/end).
+Beside it: the whole sparse-attention call (`call`), the merge kernels
+(`merge`), the kernel's DRAM bytes per launch from a one-chunk ncu capture
+(`traffic`, null once the attention source changes), and the time its
+partial writes need at a write-only HBM rate measured in the same run
+(`write_floor`).
 """
 from __future__ import annotations
 
